@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Paged decode step benchmark (B200, sm_100a).
+
+One step = the whole decode hot path over one batch: copy_blocks for pending
+copy-on-write pairs (none in the llama7b batch), reshape_and_cache of every
+sequence's new token, and paged_attention_decode (plus the split-K merge when
+the workload splits).  The default workload is the Llama-2-7B-shaped batch:
+256 sequences, 32 = 32 heads, head_dim 128, block_size 16, contexts uniform in
+[500, 1524], 32768-block pool.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama7b|gqa|bs_sweep_8|...]
+
+Prints ONE JSON line (rank 0).  value = K+V bytes the attention reads per step,
+summed over ranks, divided by the device time of the K timed steps (max over
+ranks).  Multi-GPU runs are independent replicas of the batch on every rank
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s (% of B200 HBM peak) and decode tokens/s"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b")
+    ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---- distributed plumbing -----------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(backend, world, device_index=None):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        kw = {}
+        if backend == "nccl" and device_index is not None:
+            import torch
+            kw["device_id"] = torch.device("cuda", device_index)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+
+
+def barrier(world, device_index=None):
+    if world > 1:
+        import torch.distributed as dist
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device_index])
+        else:
+            dist.barrier()
+
+
+def aggregate(ms: float, units: float, world: int, device=None):
+    """(max over ranks of the timed ms, sum over ranks of the units processed)."""
+    if world == 1:
+        return ms, units
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# ---- clocks --------------------------------------------------------------------------
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of one GPU's clocks and throttle reasons (read-only)."""
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + CLOCK_FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        # samples under load: power above the midpoint of the observed range
+        if power:
+            cut = (min(power) + max(power)) / 2
+            loaded = [num(r[1]) for r in rows if num(r[3]) is not None and num(r[3]) >= cut]
+        else:
+            loaded = sm
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded or sm) if sm else None,
+                "sm_max_mhz": num(rows[0][2]), "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def gpu_id_for(device_index: int) -> str:
+    import torch
+    props = torch.cuda.get_device_properties(device_index)
+    uuid = getattr(props, "uuid", None)
+    if uuid is not None:
+        s = str(uuid)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    return str(device_index)
+
+
+# ---- peaks and ncu traffic -------------------------------------------------------------
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this
+    exact kernel source; None otherwise."""
+    summary = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    src = os.path.join(ROOT, "paged_kv_cache_393_b200", "csrc", kernel_file)
+    if not os.path.exists(summary) or not os.path.exists(src):
+        return None
+    h = kernel_source_hash(src)
+    with open(summary) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel_file \
+                    and parts[1] == h and parts[2] == workload:
+                return float(parts[3])
+    return None
+
+
+# ---- the CUDA arm ------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    init_dist("nccl", world, local)
+    dev = torch.device("cuda", local)
+    import paged_kv_cache_393_b200 as pkv
+    from paged_kv_cache_393_b200.batch import PagedBatch
+    pkv.load_library()
+    w = wl.get(args.workload)
+    if w.lens == "cow":
+        raise SystemExit("the bench times fixed-length batches; the cow workload is a parity test")
+    gb = PagedBatch(w, dev)
+    part = w.partition_size
+    B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
+    need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, part)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    splits = need > 0
+    launches_per_step = 2 + (1 if splits else 0)   # reshape, attention[, merge]
+    G = H // Hk
+    kernel_file = "attention_mma.cu" if (2 <= G <= 8 and w.block_size >= 8) else "attention_simt.cu"
+
+    def attention():
+        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                                   gb.context_lens, w.scale, gb.max_context_len, part, ws,
+                                   stream=stream)
+
+    def cache_update():
+        pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots,
+                              stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        cache_update()
+        attention()
+    torch.cuda.synchronize(dev)
+    pkv.device_errors(clear=True)
+
+    K = args.steps
+    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    # keep the GPU busy while the sampler spins up, then time exactly K steps
+    for _ in range(20):
+        cache_update()
+        attention()
+    barrier(world, local)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(K):
+        cache_update()
+        ev_a[i][0].record(stream)
+        attention()
+        ev_a[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, local)
+    clocks = sampler.stop()
+    flags = pkv.device_errors(clear=True)
+    if flags:
+        raise SystemExit("device error flags %#x during the timed steps" % flags)
+
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = sum(a.elapsed_time(b) for a, b in ev_a) / K
+    kv_bytes = gb.kv_bytes()
+    ms_max, kv_all = aggregate(ms_total, float(kv_bytes) * K, world, dev)
+    ms_per_step = ms_max / K
+    value = kv_all / (ms_max / 1e3) / 1e9
+
+    # roofline of the attention kernel: its algorithmic bytes per launch
+    # (K+V rows read, q read, out written, table entries and lengths read)
+    nblk = (gb.lens_host + w.block_size - 1) // w.block_size
+    attn_bytes = (kv_bytes + 2 * B * H * D * 2 + int(nblk.sum()) * 4 + B * 4)
+    if splits:
+        parts = (gb.lens_host + part - 1) // part
+        attn_bytes += int(parts.sum()) * H * (D + 2) * 4 * 2    # partials written + read
+    peak, peak_kind = hbm_peak()
+    achieved = attn_bytes / (attn_ms / 1e3) / 1e9
+    traffic = recorded_traffic(kernel_file, args.workload)
+
+    # end to end through the public API: host buffers in, host result out
+    e2e = None
+    if args.e2e_steps > 0:
+        sess = pkv.DecodeSession(gb.key_cache, gb.value_cache, B, H, gb.max_blocks,
+                                 gb.max_context_len, part)
+        pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
+        hq, hk, hv = pin(gb.q_host), pin(gb.k_new_host), pin(gb.v_new_host)
+        hs, ht, hl = pin(gb.slots_host), pin(gb.tables_host), pin(gb.lens_host)
+        hout = torch.empty((B, H, D), dtype=torch.float16).pin_memory()
+        for _ in range(5):
+            sess.step(hq, hk, hv, hs, ht, hl, hout, stream=stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, local)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        E = args.e2e_steps
+        e0.record(stream)
+        for _ in range(E):
+            sess.step(hq, hk, hv, hs, ht, hl, hout, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms, e_bytes = aggregate(e0.elapsed_time(e1), float(kv_bytes) * E, world, dev)
+        e2e = {"value": round(e_bytes / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
+               "ms_per_step": round(e_ms / E, 4),
+               "h2d_bytes_per_step": sess.h2d_bytes(), "d2h_bytes_per_step": sess.d2h_bytes()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16", "accumulate": "f32", "data": "synthetic",
+            "config": {
+                "workload": "%s: %d seqs, %d query / %d kv heads, head_dim %d, block_size %d, "
+                            "contexts %s, %d-block pool" % (
+                                w.name, B, H, Hk, D, w.block_size,
+                                "%d..%d" % (gb.lens_host.min(), gb.lens_host.max()),
+                                w.num_blocks),
+                "seed": w.seed, "partition_size": part, "kv_bytes_per_step": kv_bytes,
+                "l2": "no flush: each step reads %.2f GB of K/V, far above the 126 MB L2"
+                      % (kv_bytes / 1e9),
+                "parallelism": "replicas x%d" % world},
+            "tokens_per_s": round(B * world / (ms_per_step / 1e3), 1),
+            "steps_per_s": round(1e3 / ms_per_step, 2),
+            "roofline": {"bound": "hbm", "kernel": kernel_file.replace(".cu", ""),
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                         "traffic": traffic, "algorithmic_bytes": attn_bytes,
+                         "avg_launch_ms": round(attn_ms, 5)},
+            "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+            "gpu_launches": K * launches_per_step,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---- the oracle: cpu_baseline leg and reference arm ---------------------------------------
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_sample(w, seconds, cores):
+    """Largest prefix of the batch whose oracle attention takes about `seconds`."""
+    from oracle.batch import OracleBatch
+    probe = OracleBatch(w, sample=[0, 1])
+    t = time.perf_counter()
+    probe.attention(nthreads=cores)
+    per_seq = max((time.perf_counter() - t) / 2, 1e-4)
+    n = int(max(2, min(w.num_seqs, seconds / per_seq)))
+    return OracleBatch(w, sample=list(range(n)))
+
+
+def cpu_baseline(w, seconds):
+    cores = _cores()
+    ob = _oracle_sample(w, seconds, cores)
+    t = time.perf_counter()
+    ob.attention(nthreads=cores)
+    dt = time.perf_counter() - t
+    kv = int(ob.lens.astype("int64").sum()) * wl.kv_bytes_per_token(w.num_kv_heads, w.head_dim)
+    return {"value": round(kv / dt / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "%d of %d sequences (all %d heads, %d tokens) of the %s batch; fp64 C "
+                      "oracle on %d threads; %.1f s" % (len(ob.sample), w.num_seqs, w.num_heads,
+                                                        int(ob.lens.sum()), w.name, cores, dt)}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    w = wl.get(args.workload)
+    cores = _cores()
+    steps, warm = args.steps, max(args.warmup, 3)
+    per_step = min(10.0, 150.0 / (steps + warm))
+    ob = _oracle_sample(w, per_step, cores)
+    bs = w.block_size
+    tables = ob.compact_tables
+    last = ob.lens - 1
+    slots = np.array([tables[j, L // bs] * bs + L % bs for j, L in enumerate(last)], np.int64)
+    kv_new = [wl.sequence_kv(w.seed, b, int(L) + 1, w.num_kv_heads, w.head_dim)
+              for b, L in zip(ob.sample, last)]
+    k_new = np.stack([k[-1] for k, _ in kv_new])
+    v_new = np.stack([v[-1] for _, v in kv_new])
+
+    def step():
+        kc, vc = oracle.reshape_and_cache(ob.key_cache, ob.value_cache, k_new, v_new, slots, bs)
+        return oracle.paged_attention(ob.q, kc, vc, tables, ob.lens, w.scale, bs, w.num_kv_heads,
+                                      nthreads=cores)
+    for _ in range(warm):
+        step()
+    t = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = (time.perf_counter() - t) / steps
+    kv = int(ob.lens.astype("int64").sum()) * wl.kv_bytes_per_token(w.num_kv_heads, w.head_dim)
+    value = kv / dt / 1e9
+    sample = ("%d of %d sequences (all %d heads, %d tokens) of the %s batch per step; fp64 C "
+              "oracle on %d threads" % (len(ob.sample), w.num_seqs, w.num_heads,
+                                        int(ob.lens.sum()), w.name, cores))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "seed": w.seed, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,267 @@
+/*
+ * pagedkv.h -- C ABI of the B200 paged-KV decode library (libpagedkv.so).
+ *
+ * Three GPU operations form the decode hot path of a paged KV cache:
+ *
+ *   paged_attention_decode   one query token per head attends over a KV cache held
+ *                            in fixed-size physical blocks, found through a
+ *                            per-sequence block table;
+ *   reshape_and_cache        each new token's K/V row is written into its slot;
+ *   copy_blocks              whole blocks are copied for copy-on-write.
+ *
+ * A host block manager (bm_*) hands out the physical blocks, slots and
+ * copy-on-write pairs that these operations consume; it is not on the GPU path.
+ *
+ * Conventions shared by every GPU entry point
+ * -------------------------------------------
+ *  - Every buffer is owned by the caller; the library allocates nothing of its
+ *    own on the GPU.  Pointers marked "device" must be device memory of the
+ *    current CUDA device; "host" pointers are ordinary host memory.
+ *  - fp16 means IEEE 754 binary16; the buffers are typed void* so that this
+ *    header needs no CUDA include.  fp16 buffers must be 16-byte aligned.
+ *  - KV pool layout: key_cache and value_cache are each
+ *        [num_blocks][num_kv_heads][block_size][head_dim]  fp16, contiguous,
+ *    so the rows of one (block, kv head) are one contiguous tile.  The pages
+ *    only say a block holds "block_size x num_kv_heads x head_dim" values
+ *    (lpnh.cn/news/2758356 §2.1); the head-major order inside a block is this
+ *    library's choice.
+ *  - A flat slot s addresses row s % block_size of physical block
+ *    s / block_size.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  The GPU
+ *    calls only enqueue work and return; they never synchronize.
+ *  - Return value: PAGEDKV_OK (0) or a negative PAGEDKV_E* code; nothing is
+ *    enqueued when an argument is rejected.  pagedkv_last_error() returns a
+ *    message for the calling thread's last failure.  No call throws.
+ *  - Values that live on the device cannot be checked before launch.  The
+ *    kernels check them (block ids, context lengths, slots) and, instead of
+ *    faulting, skip the bad access and set a bit in a per-device error word
+ *    that pagedkv_device_errors() reads.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PAGEDKV_API __attribute__((visibility("default")))
+#else
+#define PAGEDKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes --------------------------------------------------------- */
+#define PAGEDKV_OK 0
+#define PAGEDKV_EINVAL (-1)       /* invalid argument (null, misaligned, out of range) */
+#define PAGEDKV_EUNSUPPORTED (-2) /* shape outside the supported set */
+#define PAGEDKV_ECUDA (-3)        /* CUDA runtime or launch error */
+#define PAGEDKV_EWORKSPACE (-4)   /* workspace missing or smaller than required */
+#define PAGEDKV_ENOMEM (-5)       /* block pool exhausted (block manager) */
+#define PAGEDKV_ENOENT (-6)       /* unknown sequence id (block manager) */
+#define PAGEDKV_ERANGE (-7)       /* caller's output buffer too small */
+
+/* ---- bits of the per-device error word ------------------------------------ */
+#define PAGEDKV_DEVERR_BLOCK_ID 1u    /* a block id outside [0, num_blocks): block 0 read instead */
+#define PAGEDKV_DEVERR_CONTEXT_LEN 2u /* a context length <= 0 (output zeros) or beyond
+                                         max_context_len / the table (clamped) */
+#define PAGEDKV_DEVERR_SLOT 4u        /* a slot beyond the pool: that token was skipped */
+#define PAGEDKV_DEVERR_TIMEOUT 8u     /* a pipeline wait gave up after ~2 s; output invalid */
+
+/* Message of the calling thread's last failed call ("" if none). */
+PAGEDKV_API const char *pagedkv_last_error(void);
+
+/* Reads (and, if clear != 0, zeroes) the error word of the current device.
+ * Synchronizes the device first.  Returns PAGEDKV_OK or PAGEDKV_ECUDA. */
+PAGEDKV_API int pagedkv_device_errors(unsigned int *flags, int clear);
+
+/* ---- paged decode attention ------------------------------------------------
+ *
+ * For every sequence b < num_seqs and query head h < num_heads, with
+ * G = num_heads / num_kv_heads and kv head kvh = h / G (contiguous groups):
+ *
+ *     K_b[i] = key_cache  [block_tables[b][i / bs]][kvh][i % bs][:]   for i < L_b
+ *     V_b[i] = value_cache[block_tables[b][i / bs]][kvh][i % bs][:]
+ *     out[b][h][:] = softmax_i(scale * q[b][h][:] . K_b[i]) . V_b
+ *
+ * where L_b = context_lens[b] counts every cached token including the one
+ * written this step.  The attention reads each sequence's K/V through its block
+ * table ("查询其块表…动态地找到…高效地读取", lpnh.cn/news/1824136 §2.2 item 3 and
+ * §3.2 step 4; the table itself: 5688vip ch. 4 "PagedAttention：显存管理、分页机制、
+ * 块大小选择", section "分页机制：块表与物理块的组织方式"; lpnh.cn/news/2758356 §2.2).
+ * Accumulation is fp32; out is rounded once to fp16 (round to nearest even).
+ *
+ *   out            device fp16 [num_seqs][num_heads][head_dim]
+ *   q              device fp16 [num_seqs][num_heads][head_dim]
+ *   key_cache,
+ *   value_cache    device fp16 [num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_tables   device int32 [num_seqs][max_blocks_per_seq]; entries at and
+ *                  beyond ceil(L_b / block_size) are never read
+ *   context_lens   device int32 [num_seqs], 1 <= L_b <= max_context_len
+ *   scale          multiplies q.K (usually 1/sqrt(head_dim))
+ *   head_dim       64 or 128;  block_size 4, 8, 16, 32 or 64
+ *   num_heads      a multiple of num_kv_heads
+ *   max_context_len  an upper bound of every L_b, <= max_blocks_per_seq * block_size
+ *   partition_size 0 = chosen by the library; -1 = single pass; > 0 = split each
+ *                  context into partitions of this many tokens (a multiple of 16
+ *                  and of block_size), computed in parallel and merged by a
+ *                  second kernel.
+ *   workspace      device scratch of at least paged_attention_workspace_bytes(...)
+ *                  bytes (16-byte aligned) when the call splits; may be NULL when
+ *                  that function returns 0.  Its contents need no initialization
+ *                  and are garbage afterwards.
+ *
+ * num_seqs == 0 is a no-op.  Errors: EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+PAGEDKV_API int paged_attention_decode(void *out, const void *q,
+                           const void *key_cache, const void *value_cache,
+                           const int32_t *block_tables, const int32_t *context_lens,
+                           float scale, int block_size, int num_kv_heads,
+                           int num_seqs, int num_heads, int head_dim,
+                           int max_blocks_per_seq, int num_blocks, int max_context_len,
+                           int partition_size, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Workspace bytes paged_attention_decode needs for these arguments (0 when the
+ * call runs as a single pass).  Returns 0 for arguments it would reject too. */
+PAGEDKV_API size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_dim, int block_size, int max_context_len,
+                                       int partition_size);
+
+/* ---- reshape_and_cache -------------------------------------------------------
+ *
+ * For every token t < num_tokens with slot s = slot_mapping[t] >= 0:
+ *     key_cache  [s / bs][h][s % bs][:] = k[t][h][:]   for every kv head h
+ *     value_cache[s / bs][h][s % bs][:] = v[t][h][:]
+ * (the new token's K/V is scattered back into its block: lpnh.cn/news/1824136
+ * §3.1; a new block is used once the last one is full: 5688vip ch. 4, section
+ * "分页机制：块表与物理块的组织方式").  A slot of -1 marks padding and is
+ * skipped; a slot >= num_blocks * bs is skipped and flagged
+ * (PAGEDKV_DEVERR_SLOT).  Two tokens with the same slot race.
+ *
+ *   k, v          device fp16 [num_tokens][num_kv_heads][head_dim]
+ *   key_cache,
+ *   value_cache   device fp16 [num_blocks][num_kv_heads][block_size][head_dim]
+ *   slot_mapping  device int64 [num_tokens]
+ *   head_dim      a multiple of 8
+ *
+ * Bit-exact copy; num_tokens == 0 is a no-op.  Errors: EINVAL, ECUDA.
+ */
+PAGEDKV_API int reshape_and_cache(const void *k, const void *v, void *key_cache, void *value_cache,
+                      const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                      int head_dim, int block_size, int num_blocks, void *stream);
+
+/* ---- copy_blocks ---------------------------------------------------------------
+ *
+ * For every pair (src, dst) = src_dst_pairs[i] and every layer l:
+ *     key_caches[l][dst] = key_caches[l][src];  value_caches[l][dst] = value_caches[l][src]
+ * where a block is block_elems fp16 values (num_kv_heads * block_size * head_dim).
+ * This is the copy of copy-on-write: a writer of a shared, not yet full block
+ * gets a new block holding a copy of the old one (lpnh.cn/news/2758356 §4.2).
+ *
+ *   key_caches,
+ *   value_caches   HOST arrays of num_layers device pointers, each a pool of
+ *                  num_blocks blocks (16-byte aligned); num_layers <= 128
+ *   src_dst_pairs  device int64 [num_pairs][2]
+ *   block_elems    fp16 values per block, a multiple of 8
+ *
+ * Pairs must not overlap: no dst may repeat or appear as a src (the block
+ * manager never emits such pairs); overlapping pairs give unspecified block
+ * contents but stay in bounds.  An id outside [0, num_blocks) skips that pair
+ * and sets PAGEDKV_DEVERR_BLOCK_ID.  Bit-exact; num_pairs == 0 is a no-op.
+ * Errors: EINVAL, ECUDA.
+ */
+PAGEDKV_API int copy_blocks(void *const *key_caches, void *const *value_caches,
+                const int64_t *src_dst_pairs, int num_pairs, int num_layers,
+                size_t block_elems, int num_blocks, void *stream);
+
+/* ---- host block manager ----------------------------------------------------------
+ *
+ * Free list, reference counts, on-demand growth, fork and copy-on-write, after
+ * the pages' description (lpnh.cn/news/2758356 §3.1-§3.2, §4.2; the
+ * PagedKVManager concept model of n1n.ai "PagedAttention 对比传统 KV 缓存",
+ * section "实现逻辑代码示例"):
+ *
+ *  - the free list is a stack: allocation pops its last element and sets the
+ *    block's refcount to 1; release pushes blocks back in table order;
+ *  - a sequence grows one token at a time; a new block is taken when it has
+ *    none or its last block is full;
+ *  - fork makes children that share every block (refcount += children);
+ *  - writing into a shared (refcount > 1) last block that is not full first
+ *    copies it: a new block is taken, (src, dst) is queued for copy_blocks, the
+ *    old block's refcount drops by one and the writer's entry points to the new
+ *    block.  A shared full block needs no copy (the next token starts a fresh
+ *    block anyway);
+ *  - release decrements every block of the sequence; blocks reaching 0 return
+ *    to the free list.
+ *
+ * A failed call changes nothing.  Every call locks the manager, so reference
+ * counts stay consistent when several threads share one manager (the pages
+ * warn that unsynchronised counts corrupt shared blocks, lpnh.cn/news/2758356
+ * §4.3).  Sequence ids are small non-negative ints, never reused.
+ */
+typedef struct pagedkv_block_manager pagedkv_block_manager;
+
+/* free_order: host int32 [num_blocks], a permutation of 0..num_blocks-1 giving
+ * the initial free list (its LAST element is handed out first); NULL means
+ * 0..num_blocks-1.  Returns NULL on invalid arguments. */
+PAGEDKV_API pagedkv_block_manager *bm_create(int num_blocks, int block_size, const int32_t *free_order);
+PAGEDKV_API void bm_destroy(pagedkv_block_manager *bm);
+
+/* New sequence that already holds num_tokens tokens (ceil(num_tokens/bs)
+ * blocks).  Returns its id, or ENOMEM / EINVAL. */
+PAGEDKV_API int bm_add_seq(pagedkv_block_manager *bm, int num_tokens);
+
+/* Reserves the slot of the sequence's next token (allocating or copying on
+ * write as described above) and stores it in *slot_out.  Returns OK, ENOMEM,
+ * ENOENT or EINVAL. */
+PAGEDKV_API int bm_append_token(pagedkv_block_manager *bm, int seq, int64_t *slot_out);
+
+/* bm_append_token for seqs[0..n) in order, stopping at the first failure.
+ * Returns how many succeeded (slots_out[i] valid below that), or EINVAL. */
+PAGEDKV_API int bm_append_tokens(pagedkv_block_manager *bm, const int32_t *seqs, int n, int64_t *slots_out);
+
+/* n children sharing every block of seq; their ids go to ids_out[0..n).
+ * Returns OK, ENOENT or EINVAL. */
+PAGEDKV_API int bm_fork(pagedkv_block_manager *bm, int seq, int n, int32_t *ids_out);
+
+/* Releases the sequence.  Returns OK or ENOENT. */
+PAGEDKV_API int bm_free_seq(pagedkv_block_manager *bm, int seq);
+
+/* Copies the sequence's block table to out[0..n) and returns n; with out ==
+ * NULL only returns n.  ERANGE if cap < n, ENOENT for an unknown id. */
+PAGEDKV_API int bm_block_table(pagedkv_block_manager *bm, int seq, int32_t *out, int cap);
+
+/* Tokens held by the sequence, or ENOENT. */
+PAGEDKV_API int bm_seq_len(pagedkv_block_manager *bm, int seq);
+
+/* Packs the tables and lengths of seqs[0..n) into block_tables[n][max_blocks]
+ * (unused entries = -1) and context_lens[n].  OK, ENOENT, ERANGE or EINVAL. */
+PAGEDKV_API int bm_build_batch(pagedkv_block_manager *bm, const int32_t *seqs, int n,
+                   int32_t *block_tables, int max_blocks, int32_t *context_lens);
+
+/* Moves the queued copy-on-write pairs to pairs[0..2*count) as (src, dst) and
+ * returns count; with pairs == NULL only returns count.  ERANGE if cap (in
+ * pairs) < count, in which case nothing is moved. */
+PAGEDKV_API int bm_take_copies(pagedkv_block_manager *bm, int64_t *pairs, int cap);
+
+/* Reference count of a block (0 = free), or EINVAL. */
+PAGEDKV_API int bm_refcount(pagedkv_block_manager *bm, int block);
+
+/* Number of free blocks. */
+PAGEDKV_API int bm_num_free(pagedkv_block_manager *bm);
+
+/* Copies the free list (bottom to top) to out and returns its length; with
+ * out == NULL only returns the length.  ERANGE if cap is too small. */
+PAGEDKV_API int bm_free_list(pagedkv_block_manager *bm, int32_t *out, int cap);
+
+/* Message of the calling thread's last failed bm_* call ("" if none). */
+PAGEDKV_API const char *bm_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

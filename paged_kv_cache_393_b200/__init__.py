@@ -1,0 +1,30 @@
+"""B200-native paged KV cache: decode attention, slot-mapping scatter, copy-on-write.
+
+Thin Python binding over ``libpagedkv.so`` (C ABI in ``include/pagedkv.h``).
+Every step of the GPU path runs in the library's CUDA kernels; this module only
+checks tensor dtypes/shapes/devices and passes pointers.  PyTorch is used for
+device memory and streams.  There is no CPU fallback: if the library is
+missing, every call raises.
+
+Functions mirror the C names:
+    paged_attention_decode, paged_attention_workspace_bytes, reshape_and_cache,
+    copy_blocks, device_errors, BlockManager (bm_*), decode_step (host buffers
+    in, host result out).
+"""
+from ._native import (  # noqa: F401
+    BlockManager,
+    DecodeSession,
+    PagedKVError,
+    copy_blocks,
+    decode_step,
+    device_errors,
+    library_path,
+    load_library,
+    paged_attention_decode,
+    paged_attention_workspace_bytes,
+    reshape_and_cache,
+    DEVERR_BLOCK_ID,
+    DEVERR_CONTEXT_LEN,
+    DEVERR_SLOT,
+    DEVERR_TIMEOUT,
+)

@@ -1,0 +1,351 @@
+"""ctypes binding of libpagedkv.so (argument marshalling only).
+
+Each function checks its tensors (device, dtype, shape, contiguity), takes the
+current CUDA stream unless one is given, calls the C entry point of the same
+name and raises PagedKVError on a non-zero status.  Nothing here computes any
+part of the path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+_lock = threading.Lock()
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, EWORKSPACE, ENOMEM, ENOENT, ERANGE = 0, -1, -2, -3, -4, -5, -6, -7
+DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__("%s (status %d)" % (message, code))
+        self.code = code
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libpagedkv.so")
+
+
+def load_library():
+    """Loads libpagedkv.so; raises if it has not been built (there is no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise PagedKVError(ECUDA, "libpagedkv.so is missing: build it with "
+                               "`python -m paged_kv_cache_393_b200.build`; this package has no "
+                               "CPU fallback")
+        lib = ctypes.CDLL(path)
+        P, I, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+        sig = {
+            "pagedkv_last_error": ([], ctypes.c_char_p),
+            "pagedkv_device_errors": ([ctypes.POINTER(ctypes.c_uint), I], I),
+            "paged_attention_decode": ([P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
+            "paged_attention_workspace_bytes": ([I, I, I, I, I, I, I], Z),
+            "reshape_and_cache": ([P, P, P, P, P, I, I, I, I, I, P], I),
+            "copy_blocks": ([P, P, P, I, I, Z, I, P], I),
+            "bm_create": ([I, I, P], P),
+            "bm_destroy": ([P], None),
+            "bm_add_seq": ([P, I], I),
+            "bm_append_token": ([P, I, P], I),
+            "bm_append_tokens": ([P, P, I, P], I),
+            "bm_fork": ([P, I, I, P], I),
+            "bm_free_seq": ([P, I], I),
+            "bm_block_table": ([P, I, P, I], I),
+            "bm_seq_len": ([P, I], I),
+            "bm_build_batch": ([P, P, I, P, I, P], I),
+            "bm_take_copies": ([P, P, I], I),
+            "bm_refcount": ([P, I], I),
+            "bm_num_free": ([P], I),
+            "bm_free_list": ([P, P, I], I),
+            "bm_last_error": ([], ctypes.c_char_p),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+        return _lib
+
+
+def _check(status: int, what: str, err_fn: str = "pagedkv_last_error"):
+    if status < 0:
+        lib = load_library()
+        msg = getattr(lib, err_fn)().decode(errors="replace")
+        raise PagedKVError(status, "%s: %s" % (what, msg))
+    return status
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got shape %s" % (name, ndim, tuple(t.shape)))
+    return t.data_ptr()
+
+
+# ---- GPU operations ------------------------------------------------------------
+
+def paged_attention_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                    max_context_len, partition_size=0) -> int:
+    return int(load_library().paged_attention_workspace_bytes(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size))
+
+
+def paged_attention_decode(out, q, key_cache, value_cache, block_tables, context_lens, scale,
+                           max_context_len, partition_size=0, workspace=None, stream=None):
+    """out[B][H][D] = paged decode attention of q over the pools; see include/pagedkv.h."""
+    lib = load_library()
+    B, H, D = q.shape
+    N, Hk, bs, D2 = key_cache.shape
+    if D2 != D or tuple(value_cache.shape) != tuple(key_cache.shape) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shape mismatch: q %s, pools %s/%s, out %s" % (
+            tuple(q.shape), tuple(key_cache.shape), tuple(value_cache.shape), tuple(out.shape)))
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
+        raise ValueError("block_tables must be [B][max_blocks] and context_lens [B]")
+    ptrs = [_cuda(out, "out", torch.float16, 3), _cuda(q, "q", torch.float16, 3),
+            _cuda(key_cache, "key_cache", torch.float16, 4),
+            _cuda(value_cache, "value_cache", torch.float16, 4),
+            _cuda(block_tables, "block_tables", torch.int32, 2),
+            _cuda(context_lens, "context_lens", torch.int32, 1)]
+    need = paged_attention_workspace_bytes(B, H, Hk, D, bs, max_context_len, partition_size)
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _cuda(workspace, "workspace", workspace.dtype)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = lib.paged_attention_decode(*ptrs, float(scale), bs, Hk, B, H, D, block_tables.shape[1], N,
+                                    int(max_context_len), int(partition_size), ws_ptr, ws_bytes,
+                                    _stream(stream, q.device))
+    _check(st, "paged_attention_decode")
+    return out
+
+
+def reshape_and_cache(k, v, key_cache, value_cache, slot_mapping, stream=None):
+    """Writes k[t], v[t] ([T][Hk][D]) into slot slot_mapping[t] of the pools (bit-exact)."""
+    lib = load_library()
+    T, Hk, D = k.shape
+    N, Hk2, bs, D2 = key_cache.shape
+    if (Hk2, D2) != (Hk, D) or tuple(v.shape) != tuple(k.shape) or \
+            tuple(value_cache.shape) != tuple(key_cache.shape) or tuple(slot_mapping.shape) != (T,):
+        raise ValueError("shape mismatch")
+    st = lib.reshape_and_cache(_cuda(k, "k", torch.float16, 3), _cuda(v, "v", torch.float16, 3),
+                               _cuda(key_cache, "key_cache", torch.float16, 4),
+                               _cuda(value_cache, "value_cache", torch.float16, 4),
+                               _cuda(slot_mapping, "slot_mapping", torch.int64, 1),
+                               T, Hk, D, bs, N, _stream(stream, k.device))
+    _check(st, "reshape_and_cache")
+
+
+def copy_blocks(key_caches, value_caches, pairs, stream=None):
+    """Copies block src -> dst for every row (src, dst) of pairs ([n][2] int64, device), in
+    every layer's K and V pool."""
+    lib = load_library()
+    if len(key_caches) != len(value_caches) or not key_caches:
+        raise ValueError("need one K and one V pool per layer")
+    shape = tuple(key_caches[0].shape)
+    for t in list(key_caches) + list(value_caches):
+        if tuple(t.shape) != shape:
+            raise ValueError("every pool must have shape %s" % (shape,))
+        _cuda(t, "pool", torch.float16, 4)
+    n = 0 if pairs is None else pairs.shape[0]
+    if n == 0:
+        return
+    if pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [n][2]")
+    L = len(key_caches)
+    karr = (ctypes.c_void_p * L)(*[t.data_ptr() for t in key_caches])
+    varr = (ctypes.c_void_p * L)(*[t.data_ptr() for t in value_caches])
+    N = shape[0]
+    block_elems = shape[1] * shape[2] * shape[3]
+    st = lib.copy_blocks(karr, varr, _cuda(pairs, "pairs", torch.int64, 2), n, L, block_elems, N,
+                         _stream(stream, key_caches[0].device))
+    _check(st, "copy_blocks")
+
+
+def device_errors(clear: bool = True) -> int:
+    """Error bits the kernels raised on the current device (synchronizes the device)."""
+    flags = ctypes.c_uint(0)
+    _check(load_library().pagedkv_device_errors(ctypes.byref(flags), int(bool(clear))),
+           "pagedkv_device_errors")
+    return int(flags.value)
+
+
+class DecodeSession:
+    """A decode step driven from host buffers: the call a serving loop makes.
+
+    Holds device staging buffers for one batch shape.  ``step`` copies the
+    step's inputs from (pinned) host memory, runs copy_blocks for pending
+    copy-on-write pairs, reshape_and_cache for the new tokens and
+    paged_attention_decode, and copies the output back into a host tensor.
+    """
+
+    def __init__(self, key_cache, value_cache, num_seqs, num_heads, max_blocks, max_context_len,
+                 partition_size=0, max_pairs=0):
+        dev = key_cache.device
+        N, Hk, bs, D = key_cache.shape
+        self.key_cache, self.value_cache = key_cache, value_cache
+        self.max_context_len = int(max_context_len)
+        self.partition_size = partition_size
+        self.q = torch.empty((num_seqs, num_heads, D), dtype=torch.float16, device=dev)
+        self.k = torch.empty((num_seqs, Hk, D), dtype=torch.float16, device=dev)
+        self.v = torch.empty_like(self.k)
+        self.slots = torch.empty(num_seqs, dtype=torch.int64, device=dev)
+        self.tables = torch.empty((num_seqs, max_blocks), dtype=torch.int32, device=dev)
+        self.lens = torch.empty(num_seqs, dtype=torch.int32, device=dev)
+        self.out = torch.empty((num_seqs, num_heads, D), dtype=torch.float16, device=dev)
+        self.pairs = torch.empty((max(max_pairs, 1), 2), dtype=torch.int64, device=dev)
+        need = paged_attention_workspace_bytes(num_seqs, num_heads, Hk, D, bs, max_context_len,
+                                               partition_size)
+        self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+
+    def h2d_bytes(self, num_pairs=0) -> int:
+        ts = (self.q, self.k, self.v, self.slots, self.tables, self.lens)
+        return sum(t.numel() * t.element_size() for t in ts) + num_pairs * 16
+
+    def d2h_bytes(self) -> int:
+        return self.out.numel() * self.out.element_size()
+
+    def step(self, q, k, v, slots, tables, lens, out_host, pairs=None, stream=None):
+        s = torch.cuda.current_stream(self.q.device) if stream is None else stream
+        with torch.cuda.stream(s):
+            self.q.copy_(q, non_blocking=True)
+            self.k.copy_(k, non_blocking=True)
+            self.v.copy_(v, non_blocking=True)
+            self.slots.copy_(slots, non_blocking=True)
+            self.tables.copy_(tables, non_blocking=True)
+            self.lens.copy_(lens, non_blocking=True)
+            if pairs is not None and len(pairs):
+                n = pairs.shape[0]
+                self.pairs[:n].copy_(pairs, non_blocking=True)
+                copy_blocks([self.key_cache], [self.value_cache], self.pairs[:n], stream=s)
+            reshape_and_cache(self.k, self.v, self.key_cache, self.value_cache, self.slots, stream=s)
+            paged_attention_decode(self.out, self.q, self.key_cache, self.value_cache, self.tables,
+                                   self.lens, 1.0 / (self.q.shape[2] ** 0.5), self.max_context_len,
+                                   self.partition_size, self.workspace, stream=s)
+            out_host.copy_(self.out, non_blocking=True)
+        return out_host
+
+
+def decode_step(session: DecodeSession, *args, **kwargs):
+    """Functional alias of DecodeSession.step."""
+    return session.step(*args, **kwargs)
+
+
+# ---- host block manager --------------------------------------------------------
+
+def _np_ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+class BlockManager:
+    """Host block manager (bm_* in include/pagedkv.h).  add_seq / append_token return
+    None when the pool is exhausted; other failures raise PagedKVError."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self._lib = load_library()
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int32)
+            if order.shape != (num_blocks,):
+                raise ValueError("free_order must have num_blocks entries")
+        self._h = self._lib.bm_create(num_blocks, block_size,
+                                      None if order is None else _np_ptr(order))
+        if not self._h:
+            raise PagedKVError(EINVAL, "bm_create rejected its arguments")
+
+    def __del__(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h and self._lib is not None:
+            self._lib.bm_destroy(h)
+
+    def _chk(self, st, what):
+        return _check(st, what, "bm_last_error")
+
+    def add_seq(self, num_tokens: int):
+        st = self._lib.bm_add_seq(self._h, int(num_tokens))
+        if st == ENOMEM:
+            return None
+        return self._chk(st, "bm_add_seq")
+
+    def append_token(self, seq: int):
+        slot = ctypes.c_int64(0)
+        st = self._lib.bm_append_token(self._h, int(seq), ctypes.byref(slot))
+        if st == ENOMEM:
+            return None
+        self._chk(st, "bm_append_token")
+        return int(slot.value)
+
+    def append_tokens(self, seqs) -> np.ndarray:
+        """Appends one token to each sequence in order; returns the slots of those that
+        succeeded (fewer than len(seqs) when the pool ran out)."""
+        s = np.ascontiguousarray(seqs, dtype=np.int32)
+        out = np.empty(s.shape[0], np.int64)
+        n = self._chk(self._lib.bm_append_tokens(self._h, _np_ptr(s), s.shape[0], _np_ptr(out)),
+                      "bm_append_tokens")
+        return out[:n]
+
+    def fork(self, seq: int, n: int):
+        ids = np.empty(max(n, 1), np.int32)
+        self._chk(self._lib.bm_fork(self._h, int(seq), int(n), _np_ptr(ids)), "bm_fork")
+        return ids[:n].tolist()
+
+    def free_seq(self, seq: int):
+        self._chk(self._lib.bm_free_seq(self._h, int(seq)), "bm_free_seq")
+
+    def block_table(self, seq: int):
+        n = self._chk(self._lib.bm_block_table(self._h, int(seq), None, 0), "bm_block_table")
+        out = np.empty(max(n, 1), np.int32)
+        self._chk(self._lib.bm_block_table(self._h, int(seq), _np_ptr(out), n), "bm_block_table")
+        return out[:n].tolist()
+
+    def seq_len(self, seq: int) -> int:
+        return self._chk(self._lib.bm_seq_len(self._h, int(seq)), "bm_seq_len")
+
+    def build_batch(self, seqs, max_blocks: int):
+        s = np.ascontiguousarray(seqs, dtype=np.int32)
+        tables = np.empty((s.shape[0], max_blocks), np.int32)
+        lens = np.empty(s.shape[0], np.int32)
+        self._chk(self._lib.bm_build_batch(self._h, _np_ptr(s), s.shape[0], _np_ptr(tables),
+                                           int(max_blocks), _np_ptr(lens)), "bm_build_batch")
+        return tables, lens
+
+    def take_copies(self) -> np.ndarray:
+        n = self._chk(self._lib.bm_take_copies(self._h, None, 0), "bm_take_copies")
+        out = np.empty((max(n, 1), 2), np.int64)
+        n = self._chk(self._lib.bm_take_copies(self._h, _np_ptr(out), n), "bm_take_copies")
+        return out[:n]
+
+    def refcount(self, block: int) -> int:
+        return self._chk(self._lib.bm_refcount(self._h, int(block)), "bm_refcount")
+
+    def num_free(self) -> int:
+        return self._chk(self._lib.bm_num_free(self._h), "bm_num_free")
+
+    def free_list(self):
+        n = self._chk(self._lib.bm_free_list(self._h, None, 0), "bm_free_list")
+        out = np.empty(max(n, 1), np.int32)
+        self._chk(self._lib.bm_free_list(self._h, _np_ptr(out), n), "bm_free_list")
+        return out[:n].tolist()

@@ -1,0 +1,388 @@
+// C ABI of libpagedkv.so: argument checks, launch planning and dispatch.
+// Declarations and the contract of every entry point: include/pagedkv.h.
+#include "../../include/pagedkv.h"
+#include "kernels.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+#include <string>
+
+namespace pkv {
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(PAGEDKV_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- per-device error word -----------------------------------------------------
+
+__device__ unsigned int g_error_word;
+
+constexpr int MAX_DEVICES = 64;
+std::mutex g_err_mutex;
+unsigned* g_err_ptr[MAX_DEVICES];
+
+// Device address of the current device's error word (looked up once per device).
+int error_word(unsigned** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= MAX_DEVICES) return fail(PAGEDKV_ECUDA, "device id %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_err_mutex);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_error_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    g_err_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  *out = g_err_ptr[dev];
+  return PAGEDKV_OK;
+}
+
+// ---- tensor maps for the tensor-core kernel -------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// The pool [N][Hk][bs][D] viewed as a [N*Hk*bs][D] fp16 matrix; box = bs rows x
+// 64 columns (128 bytes, the 128-byte swizzle span).
+int encode_pool_map(CUtensorMap* map, const void* pool, int rows, int head_dim, int block_size) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(PAGEDKV_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)block_size};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(pool), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PAGEDKV_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return PAGEDKV_OK;
+}
+
+// ---- launch plan -------------------------------------------------------------------
+
+constexpr int NUM_SMS_HINT = 148;
+constexpr int AUTO_PARTITION = 512;
+constexpr size_t MAX_SMEM = 227 * 1024;
+
+// Optional overrides of the tuning choices (for sweeps); read once.
+struct Tuning {
+  int simt_kvc = 0, simt_stage_target = 0, mma_stages = 0;
+};
+const Tuning& tuning() {
+  static Tuning t = [] {
+    Tuning x;
+    if (const char* s = getenv("PAGEDKV_SIMT_KVC")) x.simt_kvc = atoi(s);
+    if (const char* s = getenv("PAGEDKV_SIMT_RING_BYTES")) x.simt_stage_target = atoi(s);
+    if (const char* s = getenv("PAGEDKV_MMA_STAGES")) x.mma_stages = atoi(s);
+    return x;
+  }();
+  return t;
+}
+
+struct Plan {
+  bool mma = false;
+  int hpc = 1, kvc = 1;      // CUDA-core kernel: query heads / kv heads per CTA
+  bool split = false;
+  int part_tokens = 0;
+  int num_parts = 1;
+  int stages = 2;
+  size_t smem = 0;
+  size_t ws_bytes = 0;
+};
+
+bool valid_block_size(int bs) { return bs == 4 || bs == 8 || bs == 16 || bs == 32 || bs == 64; }
+
+int largest_divisor_of(int n, const int* choices, int count) {
+  for (int i = 0; i < count; ++i)
+    if (n % choices[i] == 0) return choices[i];
+  return 1;
+}
+
+int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+              int block_size, int max_context_len, int partition_size) {
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+    return fail(PAGEDKV_EINVAL, "num_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                num_heads, num_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PAGEDKV_EUNSUPPORTED, "head_dim %d unsupported (64 or 128)", head_dim);
+  if (!valid_block_size(block_size))
+    return fail(PAGEDKV_EUNSUPPORTED, "block_size %d unsupported (4, 8, 16, 32 or 64)", block_size);
+  if (max_context_len <= 0) return fail(PAGEDKV_EINVAL, "max_context_len must be positive");
+  if (num_seqs < 0 || num_seqs > 65535)
+    return fail(PAGEDKV_EUNSUPPORTED, "num_seqs %d outside [0, 65535]", num_seqs);
+  const int G = num_heads / num_kv_heads;
+  Plan p;
+  p.mma = G >= 2 && G <= 8 && block_size >= 8;
+  const Tuning& tn = tuning();
+  if (!p.mma) {
+    if (G == 1) {
+      // widest contiguous kv-head group whose stage stays within 16 KB
+      const int choices[3] = {4, 2, 1};
+      p.kvc = 1;
+      for (int c : choices) {
+        if (num_heads % c == 0 && simt_stage_bytes(head_dim, block_size, c) <= 16384) {
+          p.kvc = c;
+          break;
+        }
+      }
+      if (tn.simt_kvc == 1 || tn.simt_kvc == 2 || tn.simt_kvc == 4) {
+        if (num_heads % tn.simt_kvc == 0) p.kvc = tn.simt_kvc;
+      }
+      p.hpc = p.kvc;
+    } else {
+      const int choices[4] = {8, 4, 2, 1};
+      p.hpc = largest_divisor_of(G, choices, 4);
+      p.kvc = 1;
+    }
+  }
+  // split-K: explicit, or automatic for long contexts / too few CTAs to fill the GPU
+  const int unit = p.mma ? 16 : block_size;
+  const int align = block_size > 16 ? block_size : 16;
+  if (partition_size > 0) {
+    if (partition_size % align != 0)
+      return fail(PAGEDKV_EINVAL, "partition_size %d must be a multiple of 16 and of block_size",
+                  partition_size);
+    p.split = true;
+    p.part_tokens = partition_size;
+  } else if (partition_size == 0) {
+    const long long ctas = p.mma ? (long long)num_seqs * num_kv_heads
+                                 : (long long)num_seqs * (num_heads / p.hpc);
+    const int auto_part = AUTO_PARTITION % align == 0 ? AUTO_PARTITION : align;
+    if (max_context_len > auto_part &&
+        (max_context_len > 4 * auto_part || ctas < 2LL * NUM_SMS_HINT)) {
+      p.split = true;
+      p.part_tokens = auto_part;
+    }
+  } else if (partition_size != -1) {
+    return fail(PAGEDKV_EINVAL, "partition_size %d invalid (-1, 0 or a positive size)",
+                partition_size);
+  }
+  (void)unit;
+  if (p.split) {
+    p.num_parts = (max_context_len + p.part_tokens - 1) / p.part_tokens;
+    if (p.num_parts > 65535) return fail(PAGEDKV_EUNSUPPORTED, "too many partitions");
+    p.ws_bytes = (size_t)num_seqs * num_heads * p.num_parts * (head_dim + 2) * sizeof(float);
+  } else {
+    p.part_tokens = ((max_context_len + block_size - 1) / block_size) * block_size;
+    p.num_parts = 1;
+  }
+  // ring depth
+  if (p.mma) {
+    const size_t stage = mma_stage_bytes(head_dim, block_size);
+    int st = tn.mma_stages > 0 ? tn.mma_stages : (int)(65536 / stage);
+    st = st < 2 ? 2 : (st > 16 ? 16 : st);
+    while (st > 2 && mma_smem_bytes(head_dim, block_size, st) > MAX_SMEM) --st;
+    p.stages = st;
+    p.smem = mma_smem_bytes(head_dim, block_size, st);
+  } else {
+    const size_t stage = simt_stage_bytes(head_dim, block_size, p.kvc);
+    const size_t target = tn.simt_stage_target > 0 ? (size_t)tn.simt_stage_target : 65536;
+    int st = (int)(target / stage);
+    st = st < 2 ? 2 : (st > 16 ? 16 : st);
+    while (st > 2 && simt_smem_bytes(head_dim, block_size, p.kvc, st) > MAX_SMEM) --st;
+    p.stages = st;
+    p.smem = simt_smem_bytes(head_dim, block_size, p.kvc, st);
+  }
+  if (p.smem > MAX_SMEM) return fail(PAGEDKV_EUNSUPPORTED, "shared memory plan too large");
+  *plan = p;
+  return PAGEDKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+const char* pagedkv_last_error(void) { return g_last_error.c_str(); }
+
+int pagedkv_device_errors(unsigned int* flags, int clear) {
+  if (!flags) return fail(PAGEDKV_EINVAL, "flags is NULL");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaMemcpyFromSymbol(flags, g_error_word, sizeof(unsigned));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+  if (clear) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(unsigned));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  }
+  return PAGEDKV_OK;
+}
+
+size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                       int block_size, int max_context_len, int partition_size) {
+  Plan plan;
+  if (make_plan(&plan, num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                partition_size) != PAGEDKV_OK)
+    return 0;
+  return plan.ws_bytes;
+}
+
+int paged_attention_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, float scale,
+                           int block_size, int num_kv_heads, int num_seqs, int num_heads,
+                           int head_dim, int max_blocks_per_seq, int num_blocks,
+                           int max_context_len, int partition_size, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (num_seqs == 0) return PAGEDKV_OK;
+  if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
+    return fail(PAGEDKV_EINVAL, "a required pointer is NULL");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache))
+    return fail(PAGEDKV_EINVAL, "out, q and the pools must be 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(PAGEDKV_EINVAL, "scale must be finite");
+  if (max_blocks_per_seq <= 0 || num_blocks <= 0)
+    return fail(PAGEDKV_EINVAL, "max_blocks_per_seq and num_blocks must be positive");
+  if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+    return fail(PAGEDKV_EINVAL, "max_context_len %d exceeds the table (%d blocks of %d)",
+                max_context_len, max_blocks_per_seq, block_size);
+  Plan plan;
+  int st = make_plan(&plan, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                     max_context_len, partition_size);
+  if (st != PAGEDKV_OK) return st;
+  if (plan.mma && (long long)num_blocks * num_kv_heads * block_size > 0x7fffffffLL)
+    return fail(PAGEDKV_EUNSUPPORTED, "pool of %lld rows exceeds the tensor-map range",
+                (long long)num_blocks * num_kv_heads * block_size);
+  if (plan.split) {
+    if (!workspace || workspace_bytes < plan.ws_bytes)
+      return fail(PAGEDKV_EWORKSPACE, "workspace of %zu bytes required, %zu given", plan.ws_bytes,
+                  workspace ? workspace_bytes : (size_t)0);
+    if (!aligned16(workspace)) return fail(PAGEDKV_EINVAL, "workspace must be 16-byte aligned");
+  }
+  unsigned* err = nullptr;
+  st = error_word(&err);
+  if (st != PAGEDKV_OK) return st;
+
+  DecodeParams p = {};
+  p.out = static_cast<__half*>(out);
+  p.q = static_cast<const __half*>(q);
+  p.k_cache = static_cast<const __half*>(key_cache);
+  p.v_cache = static_cast<const __half*>(value_cache);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  if (plan.split) {
+    p.ws_o = static_cast<float*>(workspace);
+    p.ws_ml = p.ws_o + (size_t)num_seqs * num_heads * plan.num_parts * head_dim;
+  }
+  p.err = err;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_seqs = num_seqs;
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.head_dim = head_dim;
+  p.block_size = block_size;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.max_context_len = max_context_len;
+  p.part_tokens = plan.part_tokens;
+  p.num_parts = plan.num_parts;
+  p.stages = plan.stages;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  cudaError_t e;
+  if (plan.mma) {
+    CUtensorMap km, vm;
+    const int rows = num_blocks * num_kv_heads * block_size;
+    st = encode_pool_map(&km, key_cache, rows, head_dim, block_size);
+    if (st != PAGEDKV_OK) return st;
+    st = encode_pool_map(&vm, value_cache, rows, head_dim, block_size);
+    if (st != PAGEDKV_OK) return st;
+    e = launch_mma_decode(p, km, vm, plan.split, s);
+  } else {
+    e = launch_simt_decode(p, plan.hpc, plan.kvc, plan.split, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  if (plan.split) {
+    e = launch_split_reduce(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
+  }
+  return PAGEDKV_OK;
+}
+
+int reshape_and_cache(const void* k, const void* v, void* key_cache, void* value_cache,
+                      const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                      int block_size, int num_blocks, void* stream) {
+  if (num_tokens == 0) return PAGEDKV_OK;
+  if (num_tokens < 0) return fail(PAGEDKV_EINVAL, "num_tokens must be >= 0");
+  if (!k || !v || !key_cache || !value_cache || !slot_mapping)
+    return fail(PAGEDKV_EINVAL, "a required pointer is NULL");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(key_cache) || !aligned16(value_cache))
+    return fail(PAGEDKV_EINVAL, "k, v and the pools must be 16-byte aligned");
+  if (num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 != 0 || block_size <= 0 || num_blocks <= 0)
+    return fail(PAGEDKV_EINVAL, "bad shape (kv heads %d, head_dim %d, block_size %d, blocks %d)",
+                num_kv_heads, head_dim, block_size, num_blocks);
+  unsigned* err = nullptr;
+  int st = error_word(&err);
+  if (st != PAGEDKV_OK) return st;
+  cudaError_t e = launch_reshape_and_cache(
+      static_cast<const __half*>(k), static_cast<const __half*>(v), static_cast<__half*>(key_cache),
+      static_cast<__half*>(value_cache), slot_mapping, num_tokens, num_kv_heads, head_dim,
+      block_size, num_blocks, err, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache launch");
+  return PAGEDKV_OK;
+}
+
+int copy_blocks(void* const* key_caches, void* const* value_caches, const int64_t* src_dst_pairs,
+                int num_pairs, int num_layers, size_t block_elems, int num_blocks, void* stream) {
+  if (num_pairs == 0) return PAGEDKV_OK;
+  if (num_pairs < 0 || num_pairs > 65535)
+    return fail(PAGEDKV_EINVAL, "num_pairs %d outside [0, 65535]", num_pairs);
+  if (num_layers <= 0 || num_layers > MAX_COPY_LAYERS)
+    return fail(PAGEDKV_EINVAL, "num_layers %d outside [1, %d]", num_layers, MAX_COPY_LAYERS);
+  if (!key_caches || !value_caches || !src_dst_pairs)
+    return fail(PAGEDKV_EINVAL, "a required pointer is NULL");
+  if (block_elems == 0 || block_elems % 8 != 0 || num_blocks <= 0)
+    return fail(PAGEDKV_EINVAL, "block_elems must be a positive multiple of 8");
+  for (int l = 0; l < num_layers; ++l) {
+    if (!key_caches[l] || !value_caches[l] || !aligned16(key_caches[l]) || !aligned16(value_caches[l]))
+      return fail(PAGEDKV_EINVAL, "layer %d pool pointer NULL or not 16-byte aligned", l);
+  }
+  unsigned* err = nullptr;
+  int st = error_word(&err);
+  if (st != PAGEDKV_OK) return st;
+  cudaError_t e = launch_copy_blocks(key_caches, value_caches, src_dst_pairs, num_pairs, num_layers,
+                                     block_elems, num_blocks, err, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "copy_blocks launch");
+  return PAGEDKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,365 @@
+// Paged decode attention on the CUDA cores (sm_100a), and the split-K merge.
+//
+// What it computes (per sequence b and query head h, kv head h / G):
+//   out[b][h] = softmax_i(scale * q[b][h] . K_b[i]) . V_b,   i < L_b,
+// with K_b[i], V_b[i] read from physical block block_tables[b][i / bs], row
+// i % bs -- the block-table gather of PagedAttention (lpnh.cn/news/1824136 §2.2
+// item 3, §3.2 step 4; 5688vip ch. 4 "PagedAttention：显存管理、分页机制、块大小选择",
+// section "分页机制：块表与物理块的组织方式").
+//
+// Design (one query token per head is ~1 flop per byte, so this is HBM-bound):
+//  * CTA = (sequence, group of HPC query heads, context partition).  The group
+//    reads KVC consecutive kv heads, which are adjacent inside every block, so
+//    each block contributes ONE contiguous KVC*bs*D fp16 tile of K and one of V.
+//  * A producer warp turns block-table entries into 1-D TMA bulk copies
+//    (cp.async.bulk, evict-first in L2) into a ring of shared-memory stages;
+//    each stage completes on an mbarrier with its byte count.  Table entries
+//    are fetched 32 at a time by the producer's lanes and broadcast by shuffle.
+//  * HPC consumer warps, one per query head, read the staged tile with 16-byte
+//    shared loads: D/8 lanes cover one K/V row, so a warp covers 32/(D/8) rows
+//    per instruction.  Scores are reduced over the D/8 lanes of a row, the
+//    online softmax runs in log2 units (scale*log2(e) folded into q) with fp32
+//    accumulation, and rows beyond the context are never multiplied (their
+//    slots may hold anything, NaN included).
+//  * With a split, each CTA covers one partition and stores (max, sum,
+//    unnormalised output); split_reduce_kernel merges the partitions.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <atomic>
+
+namespace pkv {
+namespace {
+
+__device__ __forceinline__ float dot8(const float (&q)[8], uint4 raw) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = unpack_half2(w[i]);
+    acc = fmaf(q[2 * i], f.x, acc);
+    acc = fmaf(q[2 * i + 1], f.y, acc);
+  }
+  return acc;
+}
+
+__device__ __forceinline__ void axpy8(float (&acc)[8], float a, uint4 raw) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = unpack_half2(w[i]);
+    acc[2 * i] = fmaf(a, f.x, acc[2 * i]);
+    acc[2 * i + 1] = fmaf(a, f.y, acc[2 * i + 1]);
+  }
+}
+
+template <int D, int BS, int HPC, int KVC, bool SPLIT>
+__global__ void __launch_bounds__((HPC + 1) * 32)
+    simt_decode_kernel(const DecodeParams p) {
+  constexpr int LPR = D / 8;          // lanes per K/V row (8 fp16 each)
+  constexpr int RPW = 32 / LPR;       // rows per warp-wide 16-byte load
+  constexpr int ITERS = BS / RPW;     // row groups per block
+  constexpr int TILE = KVC * BS * D;  // fp16 values of one K (or V) stage tile
+  constexpr uint32_t TILE_BYTES = TILE * 2;
+  static_assert(BS % RPW == 0, "a block must hold whole row groups");
+  static_assert(TILE_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int stages = p.stages;
+  __half* tiles = reinterpret_cast<__half*>(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)stages * 2 * TILE_BYTES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * stages);
+  // bars[s]: stage s filled (1 arrival + tx bytes); bars[stages + s]: stage s drained (HPC arrivals)
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int part = blockIdx.z;
+  const int h0 = blockIdx.x * HPC;
+  const int G = p.num_heads / p.num_kv_heads;
+  const int kv0 = h0 / G;
+  const bool reporter = threadIdx.x == 0 && blockIdx.x == 0 && part == 0;
+
+  int L = p.context_lens[b];
+  if (L > p.max_context_len) {
+    if (reporter) flag_error(p.err, ERR_CONTEXT_LEN);
+    L = p.max_context_len;
+  }
+  if (L <= 0) {
+    if (reporter) flag_error(p.err, ERR_CONTEXT_LEN);
+    if (!SPLIT && warp < HPC && lane < LPR) {
+      *reinterpret_cast<uint4*>(p.out + ((size_t)b * p.num_heads + h0 + warp) * D + lane * 8) =
+          make_uint4(0, 0, 0, 0);
+    }
+    return;  // a split launch leaves the zeros to the merge kernel
+  }
+  const int nblk = (L + BS - 1) / BS;
+  const int part_blocks = p.part_tokens / BS;
+  const int blk_begin = part * part_blocks;
+  const int n_local = min(nblk, blk_begin + part_blocks) - blk_begin;
+  if (n_local <= 0) return;  // partition beyond this context
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);
+      mbar_init(smem_u32(&bars[stages + s]), HPC);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == HPC) {
+    // ---------------- producer warp ----------------
+    const int32_t* row = p.block_tables + (size_t)b * p.max_blocks + blk_begin;
+    const uint64_t policy = l2_evict_first_policy();
+    const uint32_t ring = smem_u32(tiles);
+    int issued = 0;
+    for (int g0 = 0; g0 < n_local; g0 += 32) {
+      int id = 0;
+      if (g0 + lane < n_local) {
+        id = row[g0 + lane];
+        if (id < 0 || id >= p.num_blocks) {
+          flag_error(p.err, ERR_BLOCK_ID);
+          id = 0;
+        }
+      }
+      const int cnt = min(32, n_local - g0);
+      for (int k = 0; k < cnt; ++k) {
+        const int phys = __shfl_sync(0xffffffffu, id, k);
+        if (lane == 0 && !*abort_flag) {
+          const int i = g0 + k;
+          const int st = i % stages;
+          const int round = i / stages;
+          if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
+            *abort_flag = 1;
+            flag_error(p.err, ERR_TIMEOUT);
+          } else {
+            const size_t off = ((size_t)phys * p.num_kv_heads + kv0) * (size_t)(BS * D);
+            const uint32_t full = smem_u32(&bars[st]);
+            const uint32_t dst = ring + (uint32_t)st * 2 * TILE_BYTES;
+            mbar_arrive_expect_tx(full, 2 * TILE_BYTES);
+            bulk_load(dst, p.k_cache + off, TILE_BYTES, full, policy);
+            bulk_load(dst + TILE_BYTES, p.v_cache + off, TILE_BYTES, full, policy);
+            issued = i + 1;
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      // Only the last `stages` fills can still be in flight: let them land
+      // before this CTA's shared memory can be handed to another CTA.
+      for (int i = max(0, issued - stages); i < issued; ++i)
+        mbar_wait(smem_u32(&bars[i % stages]), (i / stages) & 1);
+    }
+    return;
+  }
+
+  // ---------------- consumer warps: one query head each ----------------
+  const int h = h0 + warp;
+  const int kvi = h / G - kv0;
+  const int sub = lane / LPR;       // row inside a row group
+  const int col = (lane % LPR) * 8; // first of this lane's 8 dims
+
+  float qf[8];
+  {
+    const uint4 raw = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.num_heads + h) * D + col);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = unpack_half2(w[i]);
+      qf[2 * i] = f.x * p.scale_log2;
+      qf[2 * i + 1] = f.y * p.scale_log2;
+    }
+  }
+
+  float m = -INFINITY;  // running max of the scores (log2 units)
+  float l = 0.f;        // running sum of 2^(s - m) over this lane's rows
+  float acc[8];
+#pragma unroll
+  for (int d = 0; d < 8; ++d) acc[d] = 0.f;
+
+  const int tok_begin = blk_begin * BS;
+  for (int i = 0; i < n_local; ++i) {
+    const int st = i % stages;
+    if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+    const bool ready = mbar_wait(smem_u32(&bars[st]), (i / stages) & 1);
+    if (!__all_sync(0xffffffffu, ready)) {
+      if (lane == 0) {
+        *abort_flag = 1;
+        flag_error(p.err, ERR_TIMEOUT);
+      }
+      break;
+    }
+    const __half* kt = tiles + (size_t)st * 2 * TILE + kvi * (BS * D);
+    const __half* vt = kt + TILE;
+    const int ntok = min(BS, L - (tok_begin + i * BS));
+
+    float s[ITERS];
+#pragma unroll
+    for (int j = 0; j < ITERS; ++j) {
+      const int t = j * RPW + sub;
+      float d = dot8(qf, *reinterpret_cast<const uint4*>(kt + t * D + col));
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      s[j] = t < ntok ? d : -INFINITY;
+    }
+    float mb = s[0];
+#pragma unroll
+    for (int j = 1; j < ITERS; ++j) mb = fmaxf(mb, s[j]);
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const float m_new = fmaxf(m, mb);  // finite: the block's first row is in the context
+    const float alpha = rescale_factor(m, m_new);
+    l *= alpha;
+#pragma unroll
+    for (int d = 0; d < 8; ++d) acc[d] *= alpha;
+#pragma unroll
+    for (int j = 0; j < ITERS; ++j) {
+      const int t = j * RPW + sub;
+      if (t < ntok) {
+        const float pj = exp2f(s[j] - m_new);
+        l += pj;
+        axpy8(acc, pj, *reinterpret_cast<const uint4*>(vt + t * D + col));
+      }
+    }
+    m = m_new;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars[stages + st]));
+  }
+
+  // Lanes with the same columns hold sums over different rows: add them up.
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1) {
+    l += __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+    for (int d = 0; d < 8; ++d) acc[d] += __shfl_xor_sync(0xffffffffu, acc[d], o);
+  }
+  if (sub == 0) {
+    const size_t bh = (size_t)b * p.num_heads + h;
+    if (!SPLIT) {
+      uint4 packed;
+      packed.x = pack_half2(acc[0] / l, acc[1] / l);
+      packed.y = pack_half2(acc[2] / l, acc[3] / l);
+      packed.z = pack_half2(acc[4] / l, acc[5] / l);
+      packed.w = pack_half2(acc[6] / l, acc[7] / l);
+      *reinterpret_cast<uint4*>(p.out + bh * D + col) = packed;
+    } else {
+      const size_t slot = bh * p.num_parts + part;
+      float4* dst = reinterpret_cast<float4*>(p.ws_o + slot * D + col);
+      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      if (lane == 0) {
+        p.ws_ml[slot * 2] = m;
+        p.ws_ml[slot * 2 + 1] = l;
+      }
+    }
+  }
+}
+
+// Merge of the partitions of one (sequence, head): with partition maxima m_i,
+// sums l_i and unnormalised outputs o_i, out = sum_i 2^(m_i - M) o_i /
+// sum_i 2^(m_i - M) l_i where M = max_i m_i.  One thread per dim.
+template <int D>
+__global__ void __launch_bounds__(D) split_reduce_kernel(const DecodeParams p) {
+  const int h = blockIdx.x;
+  const int b = blockIdx.y;
+  const int d = threadIdx.x;
+  int L = p.context_lens[b];
+  if (L > p.max_context_len) L = p.max_context_len;  // flagged by the first pass
+  __half* o = p.out + ((size_t)b * p.num_heads + h) * D;
+  if (L <= 0) {
+    o[d] = __float2half_rn(0.f);
+    return;
+  }
+  const int P = (L + p.part_tokens - 1) / p.part_tokens;
+  const size_t base = ((size_t)b * p.num_heads + h) * p.num_parts;
+  float M = -INFINITY;
+  for (int i = 0; i < P; ++i) M = fmaxf(M, p.ws_ml[(base + i) * 2]);
+  float num = 0.f, den = 0.f;
+  for (int i = 0; i < P; ++i) {
+    const float w = rescale_factor(p.ws_ml[(base + i) * 2], M);
+    den = fmaf(w, p.ws_ml[(base + i) * 2 + 1], den);
+    num = fmaf(w, p.ws_o[(base + i) * D + d], num);
+  }
+  o[d] = __float2half_rn(num / den);
+}
+
+constexpr int MAX_DEVICES = 64;
+
+// Raises a kernel's dynamic shared-memory limit once per device as needed.
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes, std::atomic<int>* granted) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+  if (granted[dev].load(std::memory_order_relaxed) >= (int)bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) granted[dev].store((int)bytes, std::memory_order_relaxed);
+  return e;
+}
+
+template <int D, int BS, int HPC, int KVC, bool SPLIT>
+cudaError_t launch_simt_instance(const DecodeParams& p, cudaStream_t stream) {
+  static std::atomic<int> granted[MAX_DEVICES];
+  auto kernel = simt_decode_kernel<D, BS, HPC, KVC, SPLIT>;
+  const size_t smem = simt_smem_bytes(D, BS, KVC, p.stages);
+  cudaError_t e = allow_smem(kernel, smem, granted);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(p.num_heads / HPC, p.num_seqs, SPLIT ? p.num_parts : 1);
+  kernel<<<grid, (HPC + 1) * 32, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t simt_stage_bytes(int head_dim, int block_size, int kvc) {
+  return 2ull * kvc * block_size * head_dim * sizeof(__half);
+}
+
+size_t simt_smem_bytes(int head_dim, int block_size, int kvc, int stages) {
+  return (size_t)stages * simt_stage_bytes(head_dim, block_size, kvc) +
+         2ull * stages * sizeof(uint64_t) + 16;
+}
+
+#define PKV_SIMT_CASE(D_, BS_, H_, K_)                                         \
+  if (p.head_dim == D_ && p.block_size == BS_ && hpc == H_ && kvc == K_)       \
+    return split ? launch_simt_instance<D_, BS_, H_, K_, true>(p, stream)      \
+                 : launch_simt_instance<D_, BS_, H_, K_, false>(p, stream);
+#define PKV_SIMT_BS(D_, H_, K_) \
+  PKV_SIMT_CASE(D_, 4, H_, K_)  \
+  PKV_SIMT_CASE(D_, 8, H_, K_)  \
+  PKV_SIMT_CASE(D_, 16, H_, K_) \
+  PKV_SIMT_CASE(D_, 32, H_, K_) \
+  PKV_SIMT_CASE(D_, 64, H_, K_)
+#define PKV_SIMT_GROUPS(D_) \
+  PKV_SIMT_BS(D_, 1, 1)     \
+  PKV_SIMT_BS(D_, 2, 2)     \
+  PKV_SIMT_BS(D_, 4, 4)     \
+  PKV_SIMT_BS(D_, 2, 1)     \
+  PKV_SIMT_BS(D_, 4, 1)     \
+  PKV_SIMT_BS(D_, 8, 1)
+
+cudaError_t launch_simt_decode(const DecodeParams& p, int hpc, int kvc, bool split,
+                               cudaStream_t stream) {
+  PKV_SIMT_GROUPS(64)
+  PKV_SIMT_GROUPS(128)
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_split_reduce(const DecodeParams& p, cudaStream_t stream) {
+  const dim3 grid(p.num_heads, p.num_seqs);
+  if (p.head_dim == 64) {
+    split_reduce_kernel<64><<<grid, 64, 0, stream>>>(p);
+  } else if (p.head_dim == 128) {
+    split_reduce_kernel<128><<<grid, 128, 0, stream>>>(p);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pkv

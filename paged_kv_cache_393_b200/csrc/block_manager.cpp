@@ -1,0 +1,265 @@
+// Host block manager of the paged KV cache: free list, reference counts,
+// on-demand growth, fork, copy-on-write and release.  Contract: include/pagedkv.h.
+//
+// Sources of the rules (all restated, none copied):
+//  * a free list from which allocation takes the LAST entry, refcount 1 on
+//    allocation, growth by one block when the sequence has none or its last
+//    block is full, failure on an empty pool: the PagedKVManager concept model
+//    (n1n.ai "PagedAttention 对比传统 KV 缓存", section "实现逻辑代码示例") and
+//    lpnh.cn/news/2758356 §3.1-§3.2;
+//  * release decrements every block and returns those at 0 (lpnh.cn/news/2758356
+//    §3.2; lpnh.cn/news/1824136 §3.2 step 6);
+//  * sharing on fork and copy-on-write of a shared, not yet full block, with a
+//    shared full block needing no copy (lpnh.cn/news/2758356 §4.2);
+//  * counts updated under a lock (lpnh.cn/news/2758356 §4.3 warns that
+//    unsynchronised counts free shared blocks early).
+#include "../../include/pagedkv.h"
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+#include <unordered_map>
+#include <utility>
+#include <vector>
+
+struct pagedkv_block_manager {
+  struct Seq {
+    std::vector<int32_t> table;
+    int64_t len = 0;
+  };
+  int num_blocks = 0;
+  int block_size = 0;
+  std::vector<int32_t> free_list;   // allocation pops the back
+  std::vector<int32_t> refcount;    // per physical block
+  std::unordered_map<int, Seq> seqs;
+  std::vector<std::pair<int64_t, int64_t>> copies;  // queued (src, dst)
+  int next_id = 0;
+  std::mutex mu;
+};
+
+namespace {
+
+thread_local std::string g_bm_error;
+
+int bm_fail(int code, const char* msg, long long a = 0) {
+  char buf[256];
+  snprintf(buf, sizeof(buf), msg, a);
+  g_bm_error = buf;
+  return code;
+}
+
+int32_t pop_free(pagedkv_block_manager* m) {
+  const int32_t blk = m->free_list.back();
+  m->free_list.pop_back();
+  m->refcount[blk] = 1;
+  return blk;
+}
+
+// Append one token to s; on success *slot holds its flat slot.  Changes nothing
+// when the pool is empty.
+int append_one(pagedkv_block_manager* m, pagedkv_block_manager::Seq& s, int64_t* slot) {
+  const int bs = m->block_size;
+  const int64_t pos = s.len;
+  if (pos % bs == 0) {
+    // no block yet, or the last block is full: a fresh block (no copy needed,
+    // even when the full last block is shared)
+    if (m->free_list.empty()) return bm_fail(PAGEDKV_ENOMEM, "block pool exhausted");
+    s.table.push_back(pop_free(m));
+  } else {
+    const int32_t last = s.table.back();
+    if (m->refcount[last] > 1) {
+      // shared and not full: copy on write
+      if (m->free_list.empty()) return bm_fail(PAGEDKV_ENOMEM, "block pool exhausted (copy on write)");
+      const int32_t fresh = pop_free(m);
+      m->copies.emplace_back(last, fresh);
+      m->refcount[last] -= 1;
+      s.table.back() = fresh;
+    }
+  }
+  *slot = (int64_t)s.table[pos / bs] * bs + pos % bs;
+  s.len = pos + 1;
+  return PAGEDKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pagedkv_block_manager* bm_create(int num_blocks, int block_size, const int32_t* free_order) {
+  if (num_blocks <= 0 || block_size <= 0) return nullptr;
+  pagedkv_block_manager* m = new (std::nothrow) pagedkv_block_manager();
+  if (!m) return nullptr;
+  m->num_blocks = num_blocks;
+  m->block_size = block_size;
+  m->refcount.assign(num_blocks, 0);
+  m->free_list.resize(num_blocks);
+  if (free_order) {
+    std::vector<char> seen(num_blocks, 0);
+    for (int i = 0; i < num_blocks; ++i) {
+      const int32_t b = free_order[i];
+      if (b < 0 || b >= num_blocks || seen[b]) {
+        delete m;
+        return nullptr;  // not a permutation
+      }
+      seen[b] = 1;
+      m->free_list[i] = b;
+    }
+  } else {
+    for (int i = 0; i < num_blocks; ++i) m->free_list[i] = i;
+  }
+  return m;
+}
+
+void bm_destroy(pagedkv_block_manager* m) { delete m; }
+
+int bm_add_seq(pagedkv_block_manager* m, int num_tokens) {
+  if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
+  if (num_tokens < 0) return bm_fail(PAGEDKV_EINVAL, "num_tokens %lld < 0", num_tokens);
+  std::lock_guard<std::mutex> lock(m->mu);
+  const int64_t need = ((int64_t)num_tokens + m->block_size - 1) / m->block_size;
+  if (need > (int64_t)m->free_list.size())
+    return bm_fail(PAGEDKV_ENOMEM, "pool cannot hold %lld more blocks", need);
+  pagedkv_block_manager::Seq s;
+  s.table.reserve(need);
+  for (int64_t i = 0; i < need; ++i) s.table.push_back(pop_free(m));
+  s.len = num_tokens;
+  const int id = m->next_id++;
+  m->seqs.emplace(id, std::move(s));
+  return id;
+}
+
+int bm_append_token(pagedkv_block_manager* m, int seq, int64_t* slot_out) {
+  if (!m || !slot_out) return bm_fail(PAGEDKV_EINVAL, "NULL argument");
+  std::lock_guard<std::mutex> lock(m->mu);
+  auto it = m->seqs.find(seq);
+  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  return append_one(m, it->second, slot_out);
+}
+
+int bm_append_tokens(pagedkv_block_manager* m, const int32_t* seqs, int n, int64_t* slots_out) {
+  if (!m || (n > 0 && (!seqs || !slots_out)) || n < 0) return bm_fail(PAGEDKV_EINVAL, "bad arguments");
+  std::lock_guard<std::mutex> lock(m->mu);
+  for (int i = 0; i < n; ++i) {
+    auto it = m->seqs.find(seqs[i]);
+    if (it == m->seqs.end()) {
+      bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seqs[i]);
+      return i;
+    }
+    if (append_one(m, it->second, &slots_out[i]) != PAGEDKV_OK) return i;
+  }
+  return n;
+}
+
+int bm_fork(pagedkv_block_manager* m, int seq, int n, int32_t* ids_out) {
+  if (!m || n < 0 || (n > 0 && !ids_out)) return bm_fail(PAGEDKV_EINVAL, "bad arguments");
+  std::lock_guard<std::mutex> lock(m->mu);
+  auto it = m->seqs.find(seq);
+  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  const pagedkv_block_manager::Seq parent = it->second;
+  for (int c = 0; c < n; ++c) {
+    for (int32_t b : parent.table) m->refcount[b] += 1;
+    const int id = m->next_id++;
+    m->seqs.emplace(id, parent);
+    ids_out[c] = id;
+  }
+  return PAGEDKV_OK;
+}
+
+int bm_free_seq(pagedkv_block_manager* m, int seq) {
+  if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
+  std::lock_guard<std::mutex> lock(m->mu);
+  auto it = m->seqs.find(seq);
+  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  for (int32_t b : it->second.table) {
+    if (--m->refcount[b] == 0) m->free_list.push_back(b);
+  }
+  m->seqs.erase(it);
+  return PAGEDKV_OK;
+}
+
+int bm_block_table(pagedkv_block_manager* m, int seq, int32_t* out, int cap) {
+  if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
+  std::lock_guard<std::mutex> lock(m->mu);
+  auto it = m->seqs.find(seq);
+  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  const int n = (int)it->second.table.size();
+  if (!out) return n;
+  if (cap < n) return bm_fail(PAGEDKV_ERANGE, "table of %lld entries does not fit", n);
+  if (n) memcpy(out, it->second.table.data(), n * sizeof(int32_t));
+  return n;
+}
+
+int bm_seq_len(pagedkv_block_manager* m, int seq) {
+  if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
+  std::lock_guard<std::mutex> lock(m->mu);
+  auto it = m->seqs.find(seq);
+  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  return (int)it->second.len;
+}
+
+int bm_build_batch(pagedkv_block_manager* m, const int32_t* seqs, int n, int32_t* block_tables,
+                   int max_blocks, int32_t* context_lens) {
+  if (!m || n < 0 || max_blocks <= 0 || (n > 0 && (!seqs || !block_tables || !context_lens)))
+    return bm_fail(PAGEDKV_EINVAL, "bad arguments");
+  std::lock_guard<std::mutex> lock(m->mu);
+  for (int i = 0; i < n; ++i) {
+    auto it = m->seqs.find(seqs[i]);
+    if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seqs[i]);
+    if ((int)it->second.table.size() > max_blocks)
+      return bm_fail(PAGEDKV_ERANGE, "sequence %lld has more blocks than max_blocks", seqs[i]);
+  }
+  for (int i = 0; i < n; ++i) {
+    const auto& s = m->seqs.find(seqs[i])->second;
+    int32_t* row = block_tables + (size_t)i * max_blocks;
+    const int nb = (int)s.table.size();
+    for (int j = 0; j < nb; ++j) row[j] = s.table[j];
+    for (int j = nb; j < max_blocks; ++j) row[j] = -1;
+    context_lens[i] = (int32_t)s.len;
+  }
+  return PAGEDKV_OK;
+}
+
+int bm_take_copies(pagedkv_block_manager* m, int64_t* pairs, int cap) {
+  if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
+  std::lock_guard<std::mutex> lock(m->mu);
+  const int n = (int)m->copies.size();
+  if (!pairs) return n;
+  if (cap < n) return bm_fail(PAGEDKV_ERANGE, "%lld pairs do not fit", n);
+  for (int i = 0; i < n; ++i) {
+    pairs[2 * i] = m->copies[i].first;
+    pairs[2 * i + 1] = m->copies[i].second;
+  }
+  m->copies.clear();
+  return n;
+}
+
+int bm_refcount(pagedkv_block_manager* m, int block) {
+  if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
+  std::lock_guard<std::mutex> lock(m->mu);
+  if (block < 0 || block >= m->num_blocks) return bm_fail(PAGEDKV_EINVAL, "block %lld out of range", block);
+  return m->refcount[block];
+}
+
+int bm_num_free(pagedkv_block_manager* m) {
+  if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
+  std::lock_guard<std::mutex> lock(m->mu);
+  return (int)m->free_list.size();
+}
+
+int bm_free_list(pagedkv_block_manager* m, int32_t* out, int cap) {
+  if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
+  std::lock_guard<std::mutex> lock(m->mu);
+  const int n = (int)m->free_list.size();
+  if (!out) return n;
+  if (cap < n) return bm_fail(PAGEDKV_ERANGE, "free list of %lld does not fit", n);
+  if (n) memcpy(out, m->free_list.data(), n * sizeof(int32_t));
+  return n;
+}
+
+// Message of the calling thread's last failed bm_* call.
+const char* bm_last_error(void) { return g_bm_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pkv {
+
+// Arguments of one paged decode-attention launch (both passes of split-K).
+struct DecodeParams {
+  __half* out;                 // [B][H][D]
+  const __half* q;             // [B][H][D]
+  const __half* k_cache;       // [N][Hk][bs][D]
+  const __half* v_cache;       // [N][Hk][bs][D]
+  const int32_t* block_tables; // [B][max_blocks]
+  const int32_t* context_lens; // [B]
+  float* ws_o;                 // split only: [B][H][num_parts][D] unnormalised partial outputs
+  float* ws_ml;                // split only: [B][H][num_parts][2] (running max in log2 units, sum)
+  unsigned* err;               // per-device error word
+  float scale_log2;            // scale * log2(e): scores are kept in log2 units
+  int num_seqs, num_heads, num_kv_heads, head_dim, block_size;
+  int max_blocks, num_blocks, max_context_len;
+  int part_tokens;             // tokens per partition (a multiple of 16 and of bs)
+  int num_parts;               // partitions per sequence in the grid
+  int stages;                  // depth of the shared-memory ring
+};
+
+// Consumer warps of the grouped-query (tensor-core) kernel; plus one producer warp.
+constexpr int MMA_CONSUMER_WARPS = 4;
+
+// Shared-memory bytes of one ring stage / the whole launch.
+size_t simt_stage_bytes(int head_dim, int block_size, int kvc);
+size_t simt_smem_bytes(int head_dim, int block_size, int kvc, int stages);
+size_t mma_stage_bytes(int head_dim, int block_size);
+size_t mma_smem_bytes(int head_dim, int block_size, int stages);
+
+// CUDA-core kernel: CTA = (b, group of hpc query heads, partition); the group
+// reads kvc consecutive kv heads.  Returns cudaErrorInvalidValue for an
+// uncompiled (head_dim, block_size, hpc, kvc) combination.
+cudaError_t launch_simt_decode(const DecodeParams& p, int hpc, int kvc, bool split,
+                               cudaStream_t stream);
+
+// Tensor-core kernel for query groups of 2..8 heads: CTA = (b, kv head, partition).
+cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& k_map,
+                              const CUtensorMap& v_map, bool split, cudaStream_t stream);
+
+// Merges the partitions of a split launch into `out`.
+cudaError_t launch_split_reduce(const DecodeParams& p, cudaStream_t stream);
+
+// Slot-mapping scatter of new K/V rows into the pools.
+cudaError_t launch_reshape_and_cache(const __half* k, const __half* v, __half* key_cache,
+                                     __half* value_cache, const int64_t* slot_mapping,
+                                     int num_tokens, int num_kv_heads, int head_dim,
+                                     int block_size, int num_blocks, unsigned* err,
+                                     cudaStream_t stream);
+
+constexpr int MAX_COPY_LAYERS = 128;
+
+// Copy-on-write block copies over every layer's K and V pool.
+cudaError_t launch_copy_blocks(void* const* key_caches, void* const* value_caches,
+                               const int64_t* pairs, int num_pairs, int num_layers,
+                               size_t block_elems, int num_blocks, unsigned* err,
+                               cudaStream_t stream);
+
+}  // namespace pkv

@@ -1,0 +1,116 @@
+"""The C ABI: the library loads, exports every symbol the headers declare, and
+rejects bad arguments on the host before touching a GPU (no compute call here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+import paged_kv_cache_393_b200 as pkv
+from paged_kv_cache_393_b200 import _native as nat
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_393_b200 import build
+    build.build()
+    return nat.load_library()
+
+
+def _declared_functions():
+    """Every function the headers declare (each declaration starts with PAGEDKV_API)."""
+    names = set()
+    for path in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(path, encoding="utf-8").read(), flags=re.S)
+        for m in re.finditer(r"^PAGEDKV_API\s+[^;(]*?\b([A-Za-z_][A-Za-z0-9_]*)\s*\(", text, re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert {"paged_attention_decode", "reshape_and_cache", "copy_blocks", "bm_create",
+            "bm_append_token", "pagedkv_last_error"} <= names
+    for name in sorted(names):
+        assert hasattr(lib, name), name
+
+
+def test_exports_are_limited_to_the_abi(lib):
+    # the library is built with hidden visibility except for the extern "C" entry points
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", nat.library_path()], capture_output=True,
+                         text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert _declared_functions() <= exported
+
+
+FAKE = 1 << 20      # 16-byte aligned addresses never dereferenced: rejected before any launch
+
+
+def _decode(lib, **over):
+    a = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, scale=0.125, bs=16, hk=4, b=2,
+             h=8, d=128, maxblk=8, n=64, maxlen=100, part=0, ws=None, wsb=0)
+    a.update(over)
+    return lib.paged_attention_decode(a["out"], a["q"], a["kc"], a["vc"], a["bt"], a["cl"],
+                                      a["scale"], a["bs"], a["hk"], a["b"], a["h"], a["d"],
+                                      a["maxblk"], a["n"], a["maxlen"], a["part"], a["ws"],
+                                      a["wsb"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), nat.EINVAL),
+    (dict(out=FAKE + 8), nat.EINVAL),                 # misaligned
+    (dict(d=96), nat.EUNSUPPORTED),
+    (dict(bs=12, maxlen=90), nat.EUNSUPPORTED),
+    (dict(h=6), nat.EINVAL),                          # not a multiple of the kv heads
+    (dict(maxlen=200), nat.EINVAL),                   # beyond 8 blocks of 16
+    (dict(maxlen=0), nat.EINVAL),
+    (dict(part=24), nat.EINVAL),                      # not a multiple of 16
+    (dict(part=-2), nat.EINVAL),
+    (dict(part=32), nat.EWORKSPACE),                  # split without a workspace
+    (dict(scale=float("nan")), nat.EINVAL),
+    (dict(b=70000), nat.EUNSUPPORTED),
+])
+def test_decode_rejects_bad_arguments_on_the_host(lib, over, code):
+    assert _decode(lib, **over) == code
+    assert lib.pagedkv_last_error().decode()
+
+
+def test_empty_batch_is_a_no_op(lib):
+    assert _decode(lib, b=0, q=None) == nat.OK
+
+
+def test_workspace_bytes(lib):
+    # single pass: no workspace
+    assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, 0) == 0
+    assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, -1) == 0
+    # explicit split: B * H * P * (D + 2) floats
+    assert pkv.paged_attention_workspace_bytes(4, 8, 2, 64, 16, 1000, 256) == 4 * 8 * 4 * 66 * 4
+    # long GQA contexts split automatically into 512-token partitions
+    assert pkv.paged_attention_workspace_bytes(128, 64, 8, 128, 16, 16384, 0) == \
+        128 * 64 * 32 * 130 * 4
+    assert pkv.paged_attention_workspace_bytes(1, 8, 3, 64, 16, 100, 0) == 0     # rejected shape
+
+
+def test_cache_ops_reject_bad_arguments_on_the_host(lib):
+    assert lib.reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 64, 16, 8, None) == nat.OK
+    assert lib.reshape_and_cache(None, FAKE, FAKE, FAKE, FAKE, 3, 4, 64, 16, 8, None) == nat.EINVAL
+    assert lib.reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 3, 4, 60, 16, 8, None) == nat.EINVAL
+    assert lib.reshape_and_cache(FAKE + 4, FAKE, FAKE, FAKE, FAKE, 3, 4, 64, 16, 8, None) == nat.EINVAL
+    arr = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    assert lib.copy_blocks(arr, arr, FAKE, 0, 2, 1024, 8, None) == nat.OK
+    assert lib.copy_blocks(arr, arr, FAKE, 3, 0, 1024, 8, None) == nat.EINVAL
+    assert lib.copy_blocks(arr, arr, FAKE, 3, 129, 1024, 8, None) == nat.EINVAL
+    assert lib.copy_blocks(arr, arr, FAKE, 3, 2, 1020, 8, None) == nat.EINVAL
+    bad = (ctypes.c_void_p * 2)(FAKE, FAKE + 2)
+    assert lib.copy_blocks(bad, arr, FAKE, 3, 2, 1024, 8, None) == nat.EINVAL
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(nat, "_lib", None)
+    monkeypatch.setattr(nat, "library_path", lambda: str(tmp_path / "libpagedkv.so"))
+    with pytest.raises(nat.PagedKVError, match="no CPU fallback"):
+        nat.load_library()

@@ -1,0 +1,364 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Cache writes and block copies must match bit for bit (compared as raw fp16 bit
+patterns, NaN sentinels included); attention outputs must satisfy
+|gpu - oracle| <= 2e-3 + 1e-2 |oracle| element by element.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from oracle_side import OracleBatch, assert_attention_close, compact_pools
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu tests")
+    from paged_kv_cache_393_b200 import build
+    build.build()
+    import paged_kv_cache_393_b200 as m
+    m.device_errors(clear=True)
+    yield m
+    torch.cuda.empty_cache()
+
+
+def _fixed(name, H, Hk, D, bs, lens, seed=2000, slack=16):
+    N = sum(-(-L // bs) for L in lens) + slack
+    return wl.Workload(name, len(lens), H, Hk, D, bs, N, seed, "fixed", fixed_lens=tuple(lens))
+
+
+def _bits(t):
+    return t.detach().cpu().numpy().view(np.uint16)
+
+
+def _run_and_compare(pkv, w, partition_size=0, sample=None, check_pool=True):
+    from paged_kv_cache_393_b200.batch import PagedBatch
+    gb = PagedBatch(w, DEV)
+    ob = OracleBatch(w, sample)
+    # the product block manager and the oracle's model agree exactly
+    assert [gb.bm.block_table(s) for s in gb.seqs] == ob.tables
+    assert np.array_equal(gb.slots_host, ob.new_slots)
+    # one decode step: scatter the new token, then attend
+    pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
+    pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                               gb.context_lens, w.scale, gb.max_context_len, partition_size)
+    torch.cuda.synchronize()
+    assert pkv.device_errors() == 0
+    if check_pool:
+        idx = torch.tensor(ob.blocks, dtype=torch.long, device=DEV)
+        assert np.array_equal(_bits(gb.key_cache[idx]), ob.key_cache.view(np.uint16))
+        assert np.array_equal(_bits(gb.value_cache[idx]), ob.value_cache.view(np.uint16))
+    got = gb.out.cpu().numpy().astype(np.float64)[ob.sample]
+    err = assert_attention_close(got, ob.attention())
+    del gb
+    torch.cuda.empty_cache()
+    return err
+
+
+# ---- small cases: every kernel variant, ragged tails, several tiles ----------------
+
+SMALL = [
+    # (workload, partition_size)
+    (wl.get("tiny"), 0),                                                    # 4=4 heads, D64, bs4
+    (_fixed("mha128_bs16", 8, 8, 128, 16, [1, 15, 16, 17, 100, 257, 700]), 0),
+    (_fixed("mha128_bs16_split", 8, 8, 128, 16, [1, 15, 16, 17, 100, 257, 700]), 32),
+    (_fixed("mha64_bs8", 4, 4, 64, 8, [3, 8, 9, 64, 65, 333]), 0),
+    (_fixed("mha64_bs32_split", 4, 4, 64, 32, [5, 31, 32, 33, 600]), 64),
+    (_fixed("mha128_bs64", 4, 4, 128, 64, [1, 63, 64, 65, 500]), 0),
+    (_fixed("mha128_bs4", 6, 6, 128, 4, [2, 4, 5, 77]), 0),
+    (_fixed("gqa8_d128_bs16", 16, 2, 128, 16, [1, 16, 17, 300, 1030]), 0),
+    (_fixed("gqa8_d128_bs16_split", 16, 2, 128, 16, [1, 16, 17, 300, 1030]), 64),
+    (_fixed("gqa4_d64_bs8", 8, 2, 64, 8, [3, 8, 9, 33, 200]), 0),
+    (_fixed("gqa4_d64_bs8_split", 8, 2, 64, 8, [3, 8, 9, 33, 200]), 16),
+    (_fixed("gqa2_d128_bs32", 4, 2, 128, 32, [1, 31, 32, 33, 410]), 0),
+    (_fixed("gqa2_d128_bs64_split", 4, 2, 128, 64, [1, 63, 64, 65, 410]), 128),
+    (_fixed("gqa3_d64_bs16", 6, 2, 64, 16, [7, 40, 129]), 0),
+    (_fixed("gqa8_bs4_cuda_cores", 16, 2, 64, 4, [1, 4, 5, 90]), 0),
+    (_fixed("gqa16_cuda_cores", 32, 2, 64, 16, [2, 17, 250]), 0),
+    (_fixed("gqa16_cuda_cores_split", 32, 2, 64, 16, [2, 17, 250]), 32),
+]
+
+
+@pytest.mark.parametrize("w,part", SMALL, ids=[c[0].name for c in SMALL])
+def test_small_cases(pkv, w, part):
+    _run_and_compare(pkv, w, partition_size=part)
+
+
+def test_single_pass_and_split_agree(pkv):
+    w = _fixed("agree", 8, 2, 128, 16, [100, 1000, 2049])
+    from paged_kv_cache_393_b200.batch import PagedBatch
+    gb = PagedBatch(w, DEV)
+    outs = []
+    for part in (-1, 512, 64):
+        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                                   gb.context_lens, w.scale, gb.max_context_len, part)
+        outs.append(gb.out.float().cpu().numpy())
+    assert np.abs(outs[0] - outs[1]).max() < 2e-3 and np.abs(outs[0] - outs[2]).max() < 2e-3
+
+
+def test_deterministic(pkv):
+    w = _fixed("det", 8, 8, 128, 16, [33, 400])
+    from paged_kv_cache_393_b200.batch import PagedBatch
+    gb = PagedBatch(w, DEV)
+    res = []
+    for _ in range(3):
+        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                                   gb.context_lens, w.scale, gb.max_context_len)
+        res.append(_bits(gb.out))
+    assert np.array_equal(res[0], res[1]) and np.array_equal(res[0], res[2])
+
+
+def test_block_table_figure_on_the_gpu(pkv):
+    # the pages' example: 12 tokens at block_size 4 in physical blocks 7, 3, 1
+    D, bs, N = 64, 4, 10
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal((12, 1, D)).astype(np.float16)
+    v = rng.standard_normal((12, 1, D)).astype(np.float16)
+    q = rng.standard_normal((1, 1, D)).astype(np.float16)
+    table = [7, 3, 1]
+    slots = np.array([table[i // bs] * bs + i % bs for i in range(12)], np.int64)
+    kc_h, vc_h = oracle.reshape_and_cache(wl.sentinel_pool(N, 1, bs, D), wl.sentinel_pool(N, 1, bs, D),
+                                          k, v, slots, bs)
+    ref = oracle.paged_attention(q, kc_h, vc_h, [table], [12], 0.125, bs, 1)
+    from paged_kv_cache_393_b200.batch import sentinel_pools
+    kc, vc = sentinel_pools(N, 1, bs, D, DEV)
+    pkv.reshape_and_cache(torch.from_numpy(k).to(DEV), torch.from_numpy(v).to(DEV), kc, vc,
+                          torch.from_numpy(slots).to(DEV))
+    out = torch.empty((1, 1, D), dtype=torch.float16, device=DEV)
+    pkv.paged_attention_decode(out, torch.from_numpy(q).to(DEV), kc, vc,
+                               torch.tensor([table], dtype=torch.int32, device=DEV),
+                               torch.tensor([12], dtype=torch.int32, device=DEV), 0.125, 12)
+    assert np.array_equal(_bits(kc), kc_h.view(np.uint16))
+    assert_attention_close(out.cpu().numpy(), ref)
+
+
+def test_context_of_one_is_exactly_v(pkv):
+    w = _fixed("len1", 8, 2, 128, 16, [1, 1, 1])
+    from paged_kv_cache_393_b200.batch import PagedBatch
+    gb = PagedBatch(w, DEV)
+    pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
+    pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                               gb.context_lens, w.scale, 1)
+    out = _bits(gb.out)
+    vnew = gb.v_new_host.view(np.uint16)
+    for h in range(8):
+        assert np.array_equal(out[:, h], vnew[:, h // 4])
+
+
+# ---- full-size workloads, sampled ---------------------------------------------------
+
+def test_llama7b_full_size(pkv):
+    w = wl.get("llama7b")
+    lens = wl.context_lens(w)
+    sample = sorted({0, 1, int(np.argmax(lens)), int(np.argmin(lens)), 100, 255})
+    _run_and_compare(pkv, w, sample=sample)
+
+
+@pytest.mark.parametrize("bs", wl.SWEEP_BLOCK_SIZES)
+def test_block_size_sweep_full_size(pkv, bs):
+    _run_and_compare(pkv, wl.bs_sweep(bs), sample=[0, 77, 255])
+
+
+def test_gqa_full_size(pkv):
+    w = wl.get("gqa")
+    lens = wl.context_lens(w)
+    sample = sorted({0, int(np.argmax(lens)), int(np.argmin(lens)), 64, 127})
+    _run_and_compare(pkv, w, partition_size=w.partition_size, sample=sample)
+
+
+def test_gqa_full_size_automatic_split(pkv):
+    w = wl.get("gqa")
+    lens = wl.context_lens(w)
+    _run_and_compare(pkv, w, partition_size=0, sample=[int(np.argmax(lens)), 3], check_pool=False)
+
+
+# ---- copy-on-write workload ---------------------------------------------------------
+
+def test_cow_workload(pkv):
+    from paged_kv_cache_393_b200.batch import CowBatch
+    w = wl.get("cow")
+    Hk, D, bs, N = w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks
+    gb = CowBatch(w, DEV)
+    model = oracle.BlockManagerModel(N, bs, free_order=wl.free_order(N, w.seed))
+    samples, prompt_of, prompt_tail = [], {}, {}
+    for p in range(w.prompts):
+        s = model.add_seq(w.prompt_len)
+        prompt_tail[p] = model.block_table(s)[-1]
+        for x in [s] + model.fork(s, w.samples - 1):
+            samples.append(x)
+            prompt_of[x] = p
+    assert samples == gb.samples
+    prompt_kv = [wl.sequence_kv(w.seed, p, w.prompt_len, Hk, D) for p in range(w.prompts)]
+
+    # step 0: seven copies per prompt (the last sharer writes in place), then the new tokens
+    host = gb.prepare_step()
+    ref_slots = [model.append_token(s) for s in samples]
+    ref_pairs = model.take_copies()
+    assert host["slots"].tolist() == ref_slots
+    assert host["pairs"].tolist() == [list(x) for x in ref_pairs]
+    assert len(ref_pairs) == w.prompts * (w.samples - 1)
+    assert {a for a, _ in ref_pairs} == set(prompt_tail.values())
+    gb.run_cache_updates(host)
+    torch.cuda.synchronize()
+    assert pkv.device_errors() == 0
+
+    # expected tail blocks: prompt tails written, copied by the oracle, then the step's rows
+    blocks = sorted(set(prompt_tail.values()) | {b for _, b in ref_pairs})
+    relabel = {b: i for i, b in enumerate(blocks)}
+    first = (w.prompt_len // bs) * bs
+    kc = wl.sentinel_pool(len(blocks), Hk, bs, D)
+    vc = wl.sentinel_pool(len(blocks), Hk, bs, D)
+    kc, vc = oracle.reshape_and_cache(
+        kc, vc, np.concatenate([kv[0][first:] for kv in prompt_kv]),
+        np.concatenate([kv[1][first:] for kv in prompt_kv]),
+        np.concatenate([relabel[prompt_tail[p]] * bs + np.arange(w.prompt_len - first)
+                        for p in range(w.prompts)]), bs)
+    kcs, vcs = oracle.copy_blocks([kc], [vc], [(relabel[a], relabel[b]) for a, b in ref_pairs])
+    new_slots = [relabel[s // bs] * bs + s % bs for s in ref_slots]
+    kc, vc = oracle.reshape_and_cache(kcs[0], vcs[0], host["k"], host["v"], new_slots, bs)
+    idx = torch.tensor(blocks, dtype=torch.long, device=DEV)
+    assert np.array_equal(_bits(gb.key_cache[idx]), kc.view(np.uint16))
+    assert np.array_equal(_bits(gb.value_cache[idx]), vc.view(np.uint16))
+    # after the copies each prompt tail is referenced by one sample only
+    assert all(model.refcount[b] == 1 for b in prompt_tail.values())
+
+    new_kv = {0: (host["k"], host["v"])}
+    chosen = [0, 7, 8, 100, 255]
+
+    def check_attention(host, steps_done):
+        tables = torch.from_numpy(host["tables"]).to(DEV)
+        lens = torch.from_numpy(host["lens"]).to(DEV)
+        q = torch.from_numpy(host["q"]).to(DEV)
+        out = torch.empty_like(q)
+        pkv.paged_attention_decode(out, q, gb.key_cache, gb.value_cache, tables, lens, w.scale,
+                                   gb.max_context_len)
+        entries = []
+        for i in chosen:
+            s = samples[i]
+            k0, v0 = prompt_kv[prompt_of[s]]
+            kn = np.stack([new_kv[j][0][i] for j in range(steps_done)])
+            vn = np.stack([new_kv[j][1][i] for j in range(steps_done)])
+            entries.append((model.block_table(s), np.concatenate([k0, kn]),
+                            np.concatenate([v0, vn])))
+        kc_o, vc_o, t_o, l_o, _ = compact_pools(entries, bs, Hk, D)
+        assert l_o.tolist() == host["lens"][chosen].tolist()
+        ref = oracle.paged_attention(host["q"][chosen], kc_o, vc_o, t_o, l_o, w.scale, bs, Hk,
+                                     nthreads=8)
+        assert_attention_close(out.cpu().numpy()[chosen], ref)
+
+    check_attention(host, 1)
+    for step in range(1, w.decode_steps):
+        host = gb.prepare_step()
+        ref_slots = [model.append_token(s) for s in samples]
+        assert host["slots"].tolist() == ref_slots
+        assert host["pairs"].tolist() == [list(x) for x in model.take_copies()]
+        gb.run_cache_updates(host)
+        new_kv[step] = (host["k"], host["v"])
+    torch.cuda.synchronize()
+    assert pkv.device_errors() == 0
+    assert (host["lens"] == w.prompt_len + w.decode_steps).all()
+    check_attention(host, w.decode_steps)
+
+
+# ---- edge cases and device-side checks ----------------------------------------------
+
+def _tiny_batch():
+    from paged_kv_cache_393_b200.batch import PagedBatch
+    return PagedBatch(_fixed("edge", 4, 4, 64, 16, [5, 40, 17]), DEV)
+
+
+def test_empty_batch_is_a_no_op(pkv):
+    gb = _tiny_batch()
+    before = _bits(gb.out)
+    pkv.paged_attention_decode(gb.out[:0], gb.q[:0], gb.key_cache, gb.value_cache,
+                               gb.block_tables[:0], gb.context_lens[:0], 0.125, 40)
+    pkv.reshape_and_cache(gb.k_new[:0], gb.v_new[:0], gb.key_cache, gb.value_cache, gb.slots[:0])
+    torch.cuda.synchronize()
+    assert np.array_equal(before, _bits(gb.out))
+    assert pkv.device_errors() == 0
+
+
+def test_zero_context_length_gives_zeros_and_a_flag(pkv):
+    gb = _tiny_batch()
+    for part in (-1, 16):
+        lens = gb.context_lens.clone()
+        lens[1] = 0
+        gb.out.fill_(1.0)
+        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                                   lens, 0.125, gb.max_context_len, part)
+        flags = pkv.device_errors()
+        assert flags & pkv.DEVERR_CONTEXT_LEN
+        assert (gb.out[1] == 0).all()
+        assert torch.isfinite(gb.out).all()
+
+
+def test_bad_block_id_is_flagged_not_faulted(pkv):
+    gb = _tiny_batch()
+    tables = gb.block_tables.clone()
+    tables[1, 1] = gb.w.num_blocks + 5
+    tables[2, 0] = -3
+    pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, tables,
+                               gb.context_lens, 0.125, gb.max_context_len)
+    assert pkv.device_errors() & pkv.DEVERR_BLOCK_ID
+    # the mma kernel's producer checks the same way
+    from paged_kv_cache_393_b200.batch import PagedBatch
+    g2 = PagedBatch(_fixed("edge_gqa", 8, 2, 64, 16, [20, 40]), DEV)
+    t2 = g2.block_tables.clone()
+    t2[0, 1] = 1 << 30
+    pkv.paged_attention_decode(g2.out, g2.q, g2.key_cache, g2.value_cache, t2, g2.context_lens,
+                               0.125, g2.max_context_len)
+    assert pkv.device_errors() & pkv.DEVERR_BLOCK_ID
+
+
+def test_context_beyond_max_is_clamped_and_flagged(pkv):
+    gb = _tiny_batch()
+    lens = gb.context_lens.clone()
+    lens[0] = 10_000
+    pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                               lens, 0.125, gb.max_context_len)
+    assert pkv.device_errors() & pkv.DEVERR_CONTEXT_LEN
+
+
+def test_bad_slot_is_flagged_and_skipped(pkv):
+    gb = _tiny_batch()
+    before = _bits(gb.key_cache)
+    slots = torch.tensor([-1, gb.w.num_blocks * 16 + 3, -1], dtype=torch.int64, device=DEV)
+    pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, slots)
+    assert pkv.device_errors() & pkv.DEVERR_SLOT
+    assert np.array_equal(before, _bits(gb.key_cache))
+
+
+def test_copy_blocks_multi_layer_and_bad_ids(pkv):
+    rng = np.random.default_rng(3)
+    N, Hk, bs, D = 12, 2, 16, 64
+    layers_k = [rng.standard_normal((N, Hk, bs, D)).astype(np.float16) for _ in range(3)]
+    layers_v = [rng.standard_normal((N, Hk, bs, D)).astype(np.float16) for _ in range(3)]
+    pairs = [(1, 7), (2, 9), (4, 0)]
+    ek, ev = oracle.copy_blocks(layers_k, layers_v, pairs)
+    dk = [torch.from_numpy(x).to(DEV) for x in layers_k]
+    dv = [torch.from_numpy(x).to(DEV) for x in layers_v]
+    pkv.copy_blocks(dk, dv, torch.tensor(pairs, dtype=torch.int64, device=DEV))
+    torch.cuda.synchronize()
+    for i in range(3):
+        assert np.array_equal(_bits(dk[i]), ek[i].view(np.uint16))
+        assert np.array_equal(_bits(dv[i]), ev[i].view(np.uint16))
+    assert pkv.device_errors() == 0
+    before = _bits(dk[0])
+    pkv.copy_blocks(dk, dv, torch.tensor([(3, N), (-1, 2)], dtype=torch.int64, device=DEV))
+    assert pkv.device_errors() & pkv.DEVERR_BLOCK_ID
+    assert np.array_equal(before, _bits(dk[0]))
+
+
+def test_max_context_at_the_table_limit(pkv):
+    # the longest context the table allows, split and unsplit
+    w = _fixed("maxctx", 2, 2, 128, 16, [4096], slack=0)
+    for part in (-1, 512):
+        _run_and_compare(pkv, w, partition_size=part)

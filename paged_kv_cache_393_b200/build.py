@@ -6,6 +6,7 @@ from __future__ import annotations
 
 import argparse
 import concurrent.futures as cf
+import hashlib
 import os
 import subprocess
 import sys
@@ -43,7 +44,24 @@ def _compile(src: str, ptxas_verbose: bool) -> str:
     return obj
 
 
+def source_digest() -> str:
+    """Hash of every source, header and flag that goes into the library."""
+    h = hashlib.sha256(" ".join(FLAGS).encode())
+    for path in [os.path.join(CSRC, s) for s in SOURCES] + HEADERS:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
 def build(force: bool = False, ptxas_verbose: bool = False, verbose: bool = False) -> str:
+    digest = source_digest()
+    stamp = LIB + ".sha256"
+    if not force and not ptxas_verbose and os.path.exists(LIB) and os.path.exists(stamp):
+        with open(stamp) as f:
+            if f.read().strip() == digest:
+                if verbose:
+                    print("up to date:", LIB)
+                return LIB
     os.makedirs(BUILD, exist_ok=True)
     hdr_time = _newest(HEADERS)
     todo = []
@@ -63,6 +81,8 @@ def build(force: bool = False, ptxas_verbose: bool = False, verbose: bool = Fals
         if res.returncode != 0:
             raise RuntimeError("link failed:\n%s%s" % (res.stdout, res.stderr))
         os.replace(tmp, LIB)
+    with open(stamp, "w") as f:
+        f.write(digest + "\n")
     if verbose:
         print("built", LIB, "(recompiled: %s)" % (", ".join(todo) or "nothing"))
     return LIB

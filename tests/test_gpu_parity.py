@@ -96,11 +96,13 @@ def test_single_pass_and_split_agree(pkv):
     w = _fixed("agree", 8, 2, 128, 16, [100, 1000, 2049])
     from paged_kv_cache_393_b200.batch import PagedBatch
     gb = PagedBatch(w, DEV)
+    pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
     outs = []
     for part in (-1, 512, 64):
         pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
                                    gb.context_lens, w.scale, gb.max_context_len, part)
         outs.append(gb.out.float().cpu().numpy())
+    assert np.isfinite(outs[0]).all()
     assert np.abs(outs[0] - outs[1]).max() < 2e-3 and np.abs(outs[0] - outs[2]).max() < 2e-3
 
 
@@ -108,11 +110,13 @@ def test_deterministic(pkv):
     w = _fixed("det", 8, 8, 128, 16, [33, 400])
     from paged_kv_cache_393_b200.batch import PagedBatch
     gb = PagedBatch(w, DEV)
+    pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
     res = []
     for _ in range(3):
         pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
                                    gb.context_lens, w.scale, gb.max_context_len)
         res.append(_bits(gb.out))
+    assert np.isfinite(gb.out.float().cpu().numpy()).all()
     assert np.array_equal(res[0], res[1]) and np.array_equal(res[0], res[2])
 
 
@@ -272,7 +276,10 @@ def test_cow_workload(pkv):
 
 def _tiny_batch():
     from paged_kv_cache_393_b200.batch import PagedBatch
-    return PagedBatch(_fixed("edge", 4, 4, 64, 16, [5, 40, 17]), DEV)
+    import paged_kv_cache_393_b200 as m
+    gb = PagedBatch(_fixed("edge", 4, 4, 64, 16, [5, 40, 17]), DEV)
+    m.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
+    return gb
 
 
 def test_empty_batch_is_a_no_op(pkv):

@@ -130,6 +130,40 @@ PAGEDKV_API size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, 
                                        int head_dim, int block_size, int max_context_len,
                                        int partition_size);
 
+/* ---- allocation-free decode ------------------------------------------------------
+ *
+ * The pages have no counterpart of this call; it serves callers that cannot
+ * allocate device memory for a workspace: an engine that reserved nearly all
+ * of HBM for its block pool at start-up, a plugin inside a runtime that owns
+ * the device allocator, a latency-bound loop that cannot afford cudaMalloc /
+ * cudaFree (they may synchronize the device).
+ *
+ * Same arguments, result and errors as paged_attention_decode, minus the
+ * workspace: split-K scratch comes from one array compiled into the library,
+ * PAGEDKV_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory that every GPU
+ * loading the library keeps until the process exits.  It allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library call).
+ *  - A call whose split needs more scratch (see paged_attention_workspace_bytes)
+ *    returns PAGEDKV_EWORKSPACE and enqueues nothing.
+ *  - The first call on a device that needs scratch looks up the array's device
+ *    address (cudaGetSymbolAddress); make that first call before any stream
+ *    capture on that device.
+ *  - All calls on a device share the array and leave their partial results in
+ *    it; calls that can overlap on the GPU (other streams, other threads) race.
+ *    Nothing needs to start at zero.
+ */
+#define PAGEDKV_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+PAGEDKV_API int paged_attention_decode_noalloc(void *out, const void *q,
+                                               const void *key_cache, const void *value_cache,
+                                               const int32_t *block_tables,
+                                               const int32_t *context_lens, float scale,
+                                               int block_size, int num_kv_heads, int num_seqs,
+                                               int num_heads, int head_dim,
+                                               int max_blocks_per_seq, int num_blocks,
+                                               int max_context_len, int partition_size,
+                                               void *stream);
+
 /* ---- reshape_and_cache -------------------------------------------------------
  *
  * For every token t < num_tokens with slot s = slot_mapping[t] >= 0:

@@ -227,6 +227,10 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
 }
 
 }  // namespace
+
+// Records a failure for pagedkv_last_error() from another translation unit.
+int record_error(int code, const char* message) { return fail(code, "%s", message); }
+
 }  // namespace pkv
 
 using namespace pkv;

@@ -80,14 +80,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// The pool [N][Hk][bs][D] viewed as a [N*Hk*bs][D] fp16 matrix; box = bs rows x
-// 64 columns (128 bytes, the 128-byte swizzle span).
+// The pool [N][Hk][bs][D] viewed as a [N*Hk*bs][D] fp16 matrix; box = min(bs, 16)
+// rows x 64 columns (128 bytes, the 128-byte swizzle span).
 int encode_pool_map(CUtensorMap* map, const void* pool, int rows, int head_dim, int block_size) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(PAGEDKV_ECUDA, "cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)block_size};
+  const cuuint32_t box[2] = {64, (cuuint32_t)(block_size < 16 ? block_size : 16)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(pool), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -204,17 +204,19 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     p.part_tokens = ((max_context_len + block_size - 1) / block_size) * block_size;
     p.num_parts = 1;
   }
-  // ring depth
+  // ring depth: few stages and many CTAs per SM stream best (measured)
   if (p.mma) {
-    const size_t stage = mma_stage_bytes(head_dim, block_size);
-    int st = tn.mma_stages > 0 ? tn.mma_stages : (int)(65536 / stage);
-    st = st < 2 ? 2 : (st > 16 ? 16 : st);
-    while (st > 2 && mma_smem_bytes(head_dim, block_size, st) > MAX_SMEM) --st;
+    // a multiple of the consumer warps, so every warp owns the same number of stages
+    int st = tn.mma_stages > 0 ? tn.mma_stages : 4;
+    st = ((st + MMA_CONSUMER_WARPS - 1) / MMA_CONSUMER_WARPS) * MMA_CONSUMER_WARPS;
+    st = st > 16 ? 16 : st;
+    while (st > MMA_CONSUMER_WARPS && mma_smem_bytes(head_dim, block_size, st) > MAX_SMEM)
+      st -= MMA_CONSUMER_WARPS;
     p.stages = st;
     p.smem = mma_smem_bytes(head_dim, block_size, st);
   } else {
     const size_t stage = simt_stage_bytes(head_dim, block_size, p.kvc);
-    const size_t target = tn.simt_stage_target > 0 ? (size_t)tn.simt_stage_target : 65536;
+    const size_t target = tn.simt_stage_target > 0 ? (size_t)tn.simt_stage_target : 32768;
     int st = (int)(target / stage);
     st = st < 2 ? 2 : (st > 16 ? 16 : st);
     while (st > 2 && simt_smem_bytes(head_dim, block_size, p.kvc, st) > MAX_SMEM) --st;

@@ -9,18 +9,21 @@
 //
 // Design (one query token per head is ~1 flop per byte, so this is HBM-bound):
 //  * CTA = (sequence, group of HPC query heads, context partition).  The group
-//    reads KVC consecutive kv heads, which are adjacent inside every block, so
-//    each block contributes ONE contiguous KVC*bs*D fp16 tile of K and one of V.
+//    reads KVC consecutive kv heads, which are adjacent inside every block.
 //  * A producer warp turns block-table entries into 1-D TMA bulk copies
-//    (cp.async.bulk, evict-first in L2) into a ring of shared-memory stages;
-//    each stage completes on an mbarrier with its byte count.  Table entries
-//    are fetched 32 at a time by the producer's lanes and broadcast by shuffle.
+//    (cp.async.bulk, evict-first in L2) into a ring of shared-memory stages of
+//    16 tokens each, whatever the block size: a stage is one block's KVC heads
+//    (bs 16, one contiguous copy), 16 rows of each head of one block (bs 32/64),
+//    or the KVC heads of 16/bs consecutive blocks (bs 4/8).  Each stage
+//    completes on an mbarrier with its byte count.  Table entries are read 32 at
+//    a time by the producer's lanes and staged in shared memory.
 //  * HPC consumer warps, one per query head, read the staged tile with 16-byte
 //    shared loads: D/8 lanes cover one K/V row, so a warp covers 32/(D/8) rows
 //    per instruction.  Scores are reduced over the D/8 lanes of a row, the
 //    online softmax runs in log2 units (scale*log2(e) folded into q) with fp32
 //    accumulation, and rows beyond the context are never multiplied (their
-//    slots may hold anything, NaN included).
+//    slots may hold anything, NaN included).  Every consumer warp reads every
+//    stage in order, so no warp can run a phase ahead of a stage's barrier.
 //  * With a split, each CTA covers one partition and stores (max, sum,
 //    unnormalised output); split_reduce_kernel merges the partitions.
 #include "common.cuh"
@@ -56,18 +59,26 @@ __device__ __forceinline__ void axpy8(float (&acc)[8], float a, uint4 raw) {
 template <int D, int BS, int HPC, int KVC, bool SPLIT>
 __global__ void __launch_bounds__((HPC + 1) * 32)
     simt_decode_kernel(const DecodeParams p) {
-  constexpr int LPR = D / 8;          // lanes per K/V row (8 fp16 each)
-  constexpr int RPW = 32 / LPR;       // rows per warp-wide 16-byte load
-  constexpr int ITERS = BS / RPW;     // row groups per block
-  constexpr int TILE = KVC * BS * D;  // fp16 values of one K (or V) stage tile
+  constexpr int CHUNK = 16;                    // tokens per ring stage
+  constexpr int CB = BS < CHUNK ? BS : CHUNK;  // rows per sub-tile: a whole block, or 16 rows of one
+  constexpr int NB = CHUNK / CB;               // sub-tiles (blocks) per stage
+  constexpr int LPR = D / 8;                   // lanes per K/V row (8 fp16 each)
+  constexpr int RPW = 32 / LPR;                // rows per warp-wide 16-byte load
+  constexpr int ITERS = CHUNK / RPW;           // row groups per stage
+  constexpr int TILE = KVC * CHUNK * D;        // fp16 values of one K (or V) stage tile
   constexpr uint32_t TILE_BYTES = TILE * 2;
-  static_assert(BS % RPW == 0, "a block must hold whole row groups");
-  static_assert(TILE_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
+  constexpr uint32_t SUB_BYTES = KVC * CB * D * 2;  // one sub-tile: KVC heads x CB rows
+  static_assert(CHUNK % RPW == 0 && CHUNK % CB == 0, "a stage must hold whole row groups");
+  static_assert(32 % NB == 0, "stages must not straddle a window of 32 table entries");
+  // A stage tile is laid out [NB sub-tiles][KVC heads][CB rows][D]: for bs <= 16
+  // a sub-tile is one block's KVC adjacent heads (one contiguous copy), for
+  // bs > 16 it is 16 rows of each of the KVC heads of one block.
 
   extern __shared__ __align__(128) unsigned char smem[];
   const int stages = p.stages;
   __half* tiles = reinterpret_cast<__half*>(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)stages * 2 * TILE_BYTES);
+  int* s_ids = reinterpret_cast<int*>(smem + (size_t)stages * 2 * TILE_BYTES);  // [32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_ids + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * stages);
   // bars[s]: stage s filled (1 arrival + tx bytes); bars[stages + s]: stage s drained (HPC arrivals)
 
@@ -93,11 +104,12 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
     }
     return;  // a split launch leaves the zeros to the merge kernel
   }
-  const int nblk = (L + BS - 1) / BS;
-  const int part_blocks = p.part_tokens / BS;
-  const int blk_begin = part * part_blocks;
-  const int n_local = min(nblk, blk_begin + part_blocks) - blk_begin;
-  if (n_local <= 0) return;  // partition beyond this context
+  const int tok0 = part * p.part_tokens;            // first token of this partition
+  const int ntok = min(L, tok0 + p.part_tokens) - tok0;
+  if (ntok <= 0) return;                            // partition beyond this context
+  const int nchunks = (ntok + CHUNK - 1) / CHUNK;
+  const int blk0 = tok0 / BS;
+  const int nblk = (ntok + BS - 1) / BS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -111,47 +123,73 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
 
   if (warp == HPC) {
     // ---------------- producer warp ----------------
-    const int32_t* row = p.block_tables + (size_t)b * p.max_blocks + blk_begin;
+    const int32_t* row = p.block_tables + (size_t)b * p.max_blocks + blk0;
     const uint64_t policy = l2_evict_first_policy();
     const uint32_t ring = smem_u32(tiles);
     int issued = 0;
-    for (int g0 = 0; g0 < n_local; g0 += 32) {
-      int id = 0;
-      if (g0 + lane < n_local) {
-        id = row[g0 + lane];
+    // table entries are read 32 at a time by the lanes and staged in shared memory
+    for (int w0 = 0; w0 < nblk; w0 += 32) {
+      if (w0 + lane < nblk) {
+        int id = row[w0 + lane];
         if (id < 0 || id >= p.num_blocks) {
           flag_error(p.err, ERR_BLOCK_ID);
           id = 0;
         }
+        s_ids[lane] = id;
       }
-      const int cnt = min(32, n_local - g0);
-      for (int k = 0; k < cnt; ++k) {
-        const int phys = __shfl_sync(0xffffffffu, id, k);
-        if (lane == 0 && !*abort_flag) {
-          const int i = g0 + k;
-          const int st = i % stages;
-          const int round = i / stages;
+      __syncwarp();
+      if (lane == 0) {
+        const int c_end = min(nchunks, (w0 + 32) * BS / CHUNK);
+        for (int c = w0 * BS / CHUNK; c < c_end && !*abort_flag; ++c) {
+          const int st = c % stages;
+          const int round = c / stages;
           if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
             *abort_flag = 1;
             flag_error(p.err, ERR_TIMEOUT);
-          } else {
-            const size_t off = ((size_t)phys * p.num_kv_heads + kv0) * (size_t)(BS * D);
-            const uint32_t full = smem_u32(&bars[st]);
-            const uint32_t dst = ring + (uint32_t)st * 2 * TILE_BYTES;
-            mbar_arrive_expect_tx(full, 2 * TILE_BYTES);
-            bulk_load(dst, p.k_cache + off, TILE_BYTES, full, policy);
-            bulk_load(dst + TILE_BYTES, p.v_cache + off, TILE_BYTES, full, policy);
-            issued = i + 1;
+            break;
           }
+          const uint32_t full = smem_u32(&bars[st]);
+          const uint32_t kdst = ring + (uint32_t)st * 2 * TILE_BYTES;
+          const uint32_t vdst = kdst + TILE_BYTES;
+          if (BS >= CHUNK) {
+            const int tok = c * CHUNK;
+            const int phys = s_ids[tok / BS - w0];
+            const int r0 = tok % BS;
+            mbar_arrive_expect_tx(full, 2 * TILE_BYTES);
+            if (BS == CHUNK) {  // the KVC heads of one block are one contiguous tile
+              const size_t off = ((size_t)phys * p.num_kv_heads + kv0) * (size_t)(BS * D);
+              bulk_load(kdst, p.k_cache + off, TILE_BYTES, full, policy);
+              bulk_load(vdst, p.v_cache + off, TILE_BYTES, full, policy);
+            } else {
+#pragma unroll
+              for (int h = 0; h < KVC; ++h) {
+                const size_t off =
+                    (((size_t)phys * p.num_kv_heads + kv0 + h) * BS + r0) * (size_t)D;
+                bulk_load(kdst + h * CHUNK * D * 2, p.k_cache + off, CHUNK * D * 2, full, policy);
+                bulk_load(vdst + h * CHUNK * D * 2, p.v_cache + off, CHUNK * D * 2, full, policy);
+              }
+            }
+          } else {
+            const int first = c * NB;                // first block of the stage
+            const int nb = min(NB, nblk - first);
+            mbar_arrive_expect_tx(full, 2u * nb * SUB_BYTES);
+            for (int k = 0; k < nb; ++k) {
+              const size_t off =
+                  ((size_t)s_ids[first + k - w0] * p.num_kv_heads + kv0) * (size_t)(BS * D);
+              bulk_load(kdst + k * SUB_BYTES, p.k_cache + off, SUB_BYTES, full, policy);
+              bulk_load(vdst + k * SUB_BYTES, p.v_cache + off, SUB_BYTES, full, policy);
+            }
+          }
+          issued = c + 1;
         }
-        __syncwarp();
       }
+      __syncwarp();  // s_ids is rewritten for the next window
     }
     if (lane == 0 && *abort_flag) {
       // Only the last `stages` fills can still be in flight: let them land
       // before this CTA's shared memory can be handed to another CTA.
-      for (int i = max(0, issued - stages); i < issued; ++i)
-        mbar_wait(smem_u32(&bars[i % stages]), (i / stages) & 1);
+      for (int c = max(0, issued - stages); c < issued; ++c)
+        mbar_wait(smem_u32(&bars[c % stages]), (c / stages) & 1);
     }
     return;
   }
@@ -180,11 +218,10 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
 #pragma unroll
   for (int d = 0; d < 8; ++d) acc[d] = 0.f;
 
-  const int tok_begin = blk_begin * BS;
-  for (int i = 0; i < n_local; ++i) {
-    const int st = i % stages;
+  for (int c = 0; c < nchunks; ++c) {
+    const int st = c % stages;
     if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
-    const bool ready = mbar_wait(smem_u32(&bars[st]), (i / stages) & 1);
+    const bool ready = mbar_wait(smem_u32(&bars[st]), (c / stages) & 1);
     if (!__all_sync(0xffffffffu, ready)) {
       if (lane == 0) {
         *abort_flag = 1;
@@ -192,25 +229,26 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
       }
       break;
     }
-    const __half* kt = tiles + (size_t)st * 2 * TILE + kvi * (BS * D);
+    const __half* kt = tiles + (size_t)st * 2 * TILE;
     const __half* vt = kt + TILE;
-    const int ntok = min(BS, L - (tok_begin + i * BS));
+    const int nvalid = min(CHUNK, ntok - c * CHUNK);
 
     float s[ITERS];
 #pragma unroll
     for (int j = 0; j < ITERS; ++j) {
       const int t = j * RPW + sub;
-      float d = dot8(qf, *reinterpret_cast<const uint4*>(kt + t * D + col));
+      const int r = (((t / CB) * KVC + kvi) * CB + t % CB) * D + col;
+      float d = dot8(qf, *reinterpret_cast<const uint4*>(kt + r));
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-      s[j] = t < ntok ? d : -INFINITY;
+      s[j] = t < nvalid ? d : -INFINITY;
     }
     float mb = s[0];
 #pragma unroll
     for (int j = 1; j < ITERS; ++j) mb = fmaxf(mb, s[j]);
 #pragma unroll
     for (int o = LPR; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-    const float m_new = fmaxf(m, mb);  // finite: the block's first row is in the context
+    const float m_new = fmaxf(m, mb);  // finite: the stage's first row is in the context
     const float alpha = rescale_factor(m, m_new);
     l *= alpha;
 #pragma unroll
@@ -218,10 +256,11 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
 #pragma unroll
     for (int j = 0; j < ITERS; ++j) {
       const int t = j * RPW + sub;
-      if (t < ntok) {
+      if (t < nvalid) {
         const float pj = exp2f(s[j] - m_new);
         l += pj;
-        axpy8(acc, pj, *reinterpret_cast<const uint4*>(vt + t * D + col));
+        const int r = (((t / CB) * KVC + kvi) * CB + t % CB) * D + col;
+        axpy8(acc, pj, *reinterpret_cast<const uint4*>(vt + r));
       }
     }
     m = m_new;
@@ -317,11 +356,12 @@ cudaError_t launch_simt_instance(const DecodeParams& p, cudaStream_t stream) {
 }  // namespace
 
 size_t simt_stage_bytes(int head_dim, int block_size, int kvc) {
-  return 2ull * kvc * block_size * head_dim * sizeof(__half);
+  (void)block_size;  // a stage is 16 tokens whatever the block size
+  return 2ull * kvc * 16 * head_dim * sizeof(__half);
 }
 
 size_t simt_smem_bytes(int head_dim, int block_size, int kvc, int stages) {
-  return (size_t)stages * simt_stage_bytes(head_dim, block_size, kvc) +
+  return (size_t)stages * simt_stage_bytes(head_dim, block_size, kvc) + 32 * sizeof(int) +
          2ull * stages * sizeof(uint64_t) + 16;
 }
 

@@ -84,6 +84,12 @@ SMALL = [
     (_fixed("gqa8_bs4_cuda_cores", 16, 2, 64, 4, [1, 4, 5, 90]), 0),
     (_fixed("gqa16_cuda_cores", 32, 2, 64, 16, [2, 17, 250]), 0),
     (_fixed("gqa16_cuda_cores_split", 32, 2, 64, 16, [2, 17, 250]), 32),
+    # long single passes: every stage of the ring is refilled many times
+    (_fixed("gqa8_d128_bs64_long", 16, 2, 128, 64, [700, 1500]), -1),
+    (_fixed("gqa4_d128_bs32_long", 8, 2, 128, 32, [999, 1800]), -1),
+    (_fixed("gqa8_d64_bs8_long", 16, 2, 64, 8, [1500, 33]), -1),
+    (_fixed("mha128_bs64_long", 4, 4, 128, 64, [1000, 1777]), -1),
+    (_fixed("mha64_bs32_long", 8, 8, 64, 32, [1300, 7]), -1),
 ]
 
 

@@ -17,6 +17,8 @@ Workloads (shapes of the pages' Llama-2-7B / 70B-like decode batches):
 * ``cow``       32 prompts of 1000 tokens, each forked into 8 samples (256
                 sequences), then 200 decode steps; 32 = 32 heads, head_dim 128,
                 block_size 16, pool of 32768 blocks.
+* ``llama7b_small`` / ``gqa_small``  32- and 16-sequence cuts of those batches
+                (pools of about 1 GB) for profiler captures.
 * ``gqa``       128 sequences, 64 query heads over 8 kv heads, head_dim 128,
                 block_size 16, context lengths round(LogNormal(ln 1024, 1))
                 clipped to [64, 16384], split into 512-token partitions,
@@ -78,6 +80,12 @@ WORKLOADS = {
     "tiny": Workload("tiny", 3, 4, 4, 64, 4, 64, 1001, "fixed", fixed_lens=(12, 50, 1)),
     "llama7b": Workload("llama7b", 256, 32, 32, 128, 16, 32768, 1002, "uniform",
                         len_lo=500, len_hi=1524),
+    # a 32-sequence cut of llama7b (0.5 GB of K/V, pools of 1 GB) for profiler captures
+    "llama7b_small": Workload("llama7b_small", 32, 32, 32, 128, 16, 4096, 1002, "uniform",
+                              len_lo=500, len_hi=1524),
+    "gqa_small": Workload("gqa_small", 16, 64, 8, 128, 16, 16384, 1005, "lognormal",
+                          lognormal_median=1024.0, lognormal_sigma=1.0, len_lo=64, len_hi=16384,
+                          partition_size=512),
     "cow": Workload("cow", 256, 32, 32, 128, 16, 32768, 1004, "cow",
                     prompts=32, prompt_len=1000, samples=8, decode_steps=200),
     "gqa": Workload("gqa", 128, 64, 8, 128, 16, 131072, 1005, "lognormal",

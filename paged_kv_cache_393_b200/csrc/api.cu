@@ -105,6 +105,7 @@ constexpr size_t MAX_SMEM = 227 * 1024;
 // Optional overrides of the tuning choices (for sweeps); read once.
 struct Tuning {
   int simt_kvc = 0, simt_stage_target = 0, mma_stages = 0;
+  bool no_persistent = false;
 };
 const Tuning& tuning() {
   static Tuning t = [] {
@@ -112,6 +113,7 @@ const Tuning& tuning() {
     if (const char* s = getenv("PAGEDKV_SIMT_KVC")) x.simt_kvc = atoi(s);
     if (const char* s = getenv("PAGEDKV_SIMT_RING_BYTES")) x.simt_stage_target = atoi(s);
     if (const char* s = getenv("PAGEDKV_MMA_STAGES")) x.mma_stages = atoi(s);
+    if (const char* s = getenv("PAGEDKV_NO_PERSISTENT")) x.no_persistent = atoi(s) != 0;
     return x;
   }();
   return t;
@@ -119,6 +121,7 @@ const Tuning& tuning() {
 
 struct Plan {
   bool mma = false;
+  bool persistent = false;   // tensor-core split-K with a ticket-fed persistent grid
   int hpc = 1, kvc = 1;      // CUDA-core kernel: query heads / kv heads per CTA
   bool split = false;
   int part_tokens = 0;
@@ -198,8 +201,12 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
   (void)unit;
   if (p.split) {
     p.num_parts = (max_context_len + p.part_tokens - 1) / p.part_tokens;
-    if (p.num_parts > 65535) return fail(PAGEDKV_EUNSUPPORTED, "too many partitions");
+    if (p.num_parts > MAX_PARTITIONS)
+      return fail(PAGEDKV_EUNSUPPORTED, "%d partitions exceed %d: use a larger partition_size",
+                  p.num_parts, MAX_PARTITIONS);
     p.ws_bytes = (size_t)num_seqs * num_heads * p.num_parts * (head_dim + 2) * sizeof(float);
+    p.persistent = p.mma && num_seqs <= PERSISTENT_MAX_SEQS && !tn.no_persistent;
+    if (p.persistent) p.ws_bytes = ((p.ws_bytes + 15) / 16) * 16 + 16;  // + the ticket word
   } else {
     p.part_tokens = ((max_context_len + block_size - 1) / block_size) * block_size;
     p.num_parts = 1;
@@ -210,10 +217,13 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     int st = tn.mma_stages > 0 ? tn.mma_stages : 4;
     st = ((st + MMA_CONSUMER_WARPS - 1) / MMA_CONSUMER_WARPS) * MMA_CONSUMER_WARPS;
     st = st > 16 ? 16 : st;
-    while (st > MMA_CONSUMER_WARPS && mma_smem_bytes(head_dim, block_size, st) > MAX_SMEM)
-      st -= MMA_CONSUMER_WARPS;
+    auto smem_of = [&](int n) {
+      return p.persistent ? mma_persistent_smem_bytes(head_dim, n, num_seqs)
+                          : mma_smem_bytes(head_dim, block_size, n);
+    };
+    while (st > MMA_CONSUMER_WARPS && smem_of(st) > MAX_SMEM) st -= MMA_CONSUMER_WARPS;
     p.stages = st;
-    p.smem = mma_smem_bytes(head_dim, block_size, st);
+    p.smem = smem_of(st);
   } else {
     const size_t stage = simt_stage_bytes(head_dim, block_size, p.kvc);
     const size_t target = tn.simt_stage_target > 0 ? (size_t)tn.simt_stage_target : 32768;
@@ -332,7 +342,15 @@ int paged_attention_decode(void* out, const void* q, const void* key_cache, cons
     if (st != PAGEDKV_OK) return st;
     st = encode_pool_map(&vm, value_cache, rows, head_dim, block_size);
     if (st != PAGEDKV_OK) return st;
-    e = launch_mma_decode(p, km, vm, plan.split, s);
+    if (plan.persistent) {
+      const size_t parts_bytes =
+          (size_t)num_seqs * num_heads * plan.num_parts * (head_dim + 2) * sizeof(float);
+      unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
+                                                             ((parts_bytes + 15) / 16) * 16);
+      e = launch_mma_decode_persistent(p, km, vm, ticket, s);
+    } else {
+      e = launch_mma_decode(p, km, vm, plan.split, s);
+    }
   } else {
     e = launch_simt_decode(p, plan.hpc, plan.kvc, plan.split, s);
   }

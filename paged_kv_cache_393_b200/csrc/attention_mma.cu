@@ -24,9 +24,18 @@
 // order; a warp therefore never waits on a barrier phase that a slower warp
 // has not reached yet (parity waits cannot tell phase k from phase k+2).
 // Four consumer warps, each with its own online softmax, merge through shared
-// memory at the end, reusing the drained ring.  Rows past the context are
-// masked out of the scores, and the matching V rows are zeroed in shared
-// memory before PV (0 * NaN would poison the sum).
+// memory.  Rows past the context are masked out of the scores, and the
+// matching V rows are zeroed in shared memory before PV (0 * NaN would poison
+// the sum).
+//
+// Two schedules share this code:
+//  * mma_decode_kernel: one CTA per (sequence, kv head, partition);
+//  * mma_decode_persistent_kernel (split-K): a few CTAs per SM take work items
+//    (sequence, kv head, partition) from a ticket counter -- every full
+//    partition first, then the partial last partitions -- and the producer
+//    streams chunks across item boundaries without draining the ring.  The
+//    items' query tiles travel through a small queue (bulk copies) with their
+//    descriptors, and each finished item is merged while the next streams in.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -36,6 +45,8 @@ namespace pkv {
 namespace {
 
 constexpr int NW = MMA_CONSUMER_WARPS;
+constexpr int CHUNK = 16;  // tokens per ring stage
+constexpr int IQ = 1;      // item-queue depth of the persistent kernel
 
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -56,36 +67,294 @@ __device__ __forceinline__ bool named_barrier_or(int id, int threads, bool pred)
 }
 
 // Shared-memory address of the 16-byte unit holding column `colh` (fp16 index)
-// of token row `tok` in a stage tile laid out as [D/64 slices][CHUNK rows][128 B]
+// of token row `tok` in a stage tile laid out as [D/64 slices][16 rows][128 B]
 // with the 128-byte swizzle (unit index XOR row mod 8).
-template <int CHUNK>
 __device__ __forceinline__ uint32_t swz_addr(uint32_t tile, int tok, int colh) {
   const int sl = colh >> 6;
   const int unit = (colh & 63) >> 3;
   return tile + sl * (CHUNK * 128) + tok * 128 + ((unit ^ (tok & 7)) << 4);
 }
 
+template <int D>
+struct StageGeom {
+  static constexpr int NSL = D / 64;                           // 64-column slices
+  static constexpr uint32_t SLICE_BYTES = CHUNK * 128;
+  static constexpr uint32_t TILE_BYTES = NSL * SLICE_BYTES;    // K (or V) of one stage
+  static constexpr int MT = D / 16;                            // 16-wide slices of D
+  static constexpr int OSTRIDE = D + 4;                        // padded merge rows
+  static constexpr uint32_t MERGE_BYTES = NW * 8 * (2 + OSTRIDE) * 4;
+};
+
+// ---- producer side ---------------------------------------------------------------
+
+// Issues the TMA copies of chunk c (16 tokens) of an item whose table window
+// (entries w0 .. w0+31 of the item's blocks) is staged in s_ids.
+template <int D, int BS>
+__device__ __forceinline__ void issue_stage(uint32_t kdst, uint32_t full, const int* s_ids, int w0,
+                                            int c, int nblk, int kvh, int num_kv_heads,
+                                            const CUtensorMap* km, const CUtensorMap* vm,
+                                            uint64_t policy) {
+  using Geo = StageGeom<D>;
+  constexpr int CB = BS < CHUNK ? BS : CHUNK;  // rows per TMA box
+  constexpr int NB = CHUNK / CB;               // boxes per stage and slice
+  constexpr uint32_t BOX_BYTES = CB * 128;
+  const uint32_t vdst = kdst + Geo::TILE_BYTES;
+  const int first = c * NB;  // first block of the stage (bs 8)
+  const int nb = BS >= CHUNK ? 1 : min(NB, nblk - first);
+  mbar_arrive_expect_tx(full, 2u * nb * Geo::NSL * BOX_BYTES);
+  for (int k = 0; k < nb; ++k) {
+    int y;
+    if (BS >= CHUNK) {
+      const int tok = c * CHUNK;
+      y = (s_ids[tok / BS - w0] * num_kv_heads + kvh) * BS + tok % BS;
+    } else {
+      y = (s_ids[first + k - w0] * num_kv_heads + kvh) * BS;
+    }
+#pragma unroll
+    for (int sl = 0; sl < Geo::NSL; ++sl) {
+      const uint32_t off = sl * Geo::SLICE_BYTES + k * BOX_BYTES;
+      tensor_load_2d(kdst + off, km, sl * 64, y, full, policy);
+      tensor_load_2d(vdst + off, vm, sl * 64, y, full, policy);
+    }
+  }
+}
+
+// Streams the nchunks chunks of one item (its table row starts at `row`) into
+// the ring, the item's first chunk having global chunk index gc0.  Run by the
+// whole producer warp; lane 0 issues.  Returns false (warp-uniform) when it
+// gave up; *issued_end is one past the last global chunk issued.
+template <int D, int BS>
+__device__ bool produce_item(const int32_t* row, int nblk, int nchunks, int gc0, int kvh,
+                             const DecodeParams& p, int* s_ids, uint64_t* bars, int stages,
+                             uint32_t ring, const CUtensorMap* km, const CUtensorMap* vm,
+                             uint64_t policy, volatile int* abort_flag, int lane, int* issued_end) {
+  using Geo = StageGeom<D>;
+  bool ok = true;
+  for (int w0 = 0; w0 < nblk; w0 += 32) {
+    if (w0 + lane < nblk) {
+      int id = row[w0 + lane];
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(p.err, ERR_BLOCK_ID);
+        id = 0;
+      }
+      s_ids[lane] = id;
+    }
+    __syncwarp();
+    if (lane == 0 && ok) {
+      const int c_end = min(nchunks, (w0 + 32) * BS / CHUNK);
+      for (int c = w0 * BS / CHUNK; c < c_end; ++c) {
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        const int gc = gc0 + c;
+        const int st = gc % stages;
+        const int round = gc / stages;
+        if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
+          *abort_flag = 1;
+          flag_error(p.err, ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+        issue_stage<D, BS>(ring + (uint32_t)st * 2 * Geo::TILE_BYTES, smem_u32(&bars[st]), s_ids,
+                           w0, c, nblk, kvh, p.num_kv_heads, km, vm, policy);
+        *issued_end = gc + 1;
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+    __syncwarp();  // s_ids is rewritten for the next window
+  }
+  return ok;
+}
+
+// After an abort only the last `stages` fills can still be in flight: let them
+// land before this CTA's shared memory can be handed to another CTA.
+__device__ __forceinline__ void drain_ring(uint64_t* bars, int stages, int issued_end) {
+  for (int c = max(0, issued_end - stages); c < issued_end; ++c)
+    mbar_wait(smem_u32(&bars[c % stages]), (c / stages) & 1);
+}
+
+// ---- consumer side ---------------------------------------------------------------
+
+template <int D>
+struct Acc {
+  float m0, m1;  // running max of heads 2t, 2t+1 (log2 units)
+  float l0, l1;  // this lane's part of the running sums
+  float o[D / 16][4];
+  __device__ __forceinline__ void reset() {
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  }
+};
+
+// One 16-token stage: QK^T, masked online softmax, PV.  valid = rows of the
+// stage inside the context (1..16).
+template <int D>
+__device__ __forceinline__ void consume_stage(Acc<D>& a, uint32_t kt, int valid,
+                                              const uint32_t (&qb)[D / 16][2], float scale_log2,
+                                              int lane) {
+  using Geo = StageGeom<D>;
+  const uint32_t vt = kt + Geo::TILE_BYTES;
+  const int g = lane >> 2;
+  const int mat = lane >> 3;  // ldmatrix: which 8x8 matrix this lane addresses
+  const int r8 = lane & 7;    // ... and which of its rows
+
+  // ---- S^T = K . Q^T ----
+  float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int ks = 0; ks < Geo::MT; ++ks) {
+    const int tok = r8 + ((mat & 1) << 3);
+    const int colh = ks * 16 + ((mat >> 1) << 3);
+    uint32_t a0, a1, a2, a3;
+    ldmatrix_x4(swz_addr(kt, tok, colh), a0, a1, a2, a3);
+    mma_16816(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+  }
+  const float s0 = g < valid ? sc[0] * scale_log2 : -INFINITY;
+  const float s1 = g < valid ? sc[1] * scale_log2 : -INFINITY;
+  const float s2 = g + 8 < valid ? sc[2] * scale_log2 : -INFINITY;
+  const float s3 = g + 8 < valid ? sc[3] * scale_log2 : -INFINITY;
+  float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+  }
+  const float mn0 = fmaxf(a.m0, mx0), mn1 = fmaxf(a.m1, mx1);  // finite: row 0 is valid
+  const float al0 = rescale_factor(a.m0, mn0), al1 = rescale_factor(a.m1, mn1);
+  a.m0 = mn0;
+  a.m1 = mn1;
+  const uint32_t p01 = pack_half2(exp2f(s0 - mn0), exp2f(s1 - mn1));  // token g
+  const uint32_t p23 = pack_half2(exp2f(s2 - mn0), exp2f(s3 - mn1));  // token g + 8
+  const float2 f01 = unpack_half2(p01), f23 = unpack_half2(p23);
+  a.l0 = fmaf(a.l0, al0, f01.x + f23.x);
+  a.l1 = fmaf(a.l1, al1, f01.y + f23.y);
+#pragma unroll
+  for (int mt = 0; mt < Geo::MT; ++mt) {
+    a.o[mt][0] *= al0;
+    a.o[mt][1] *= al1;
+    a.o[mt][2] *= al0;
+    a.o[mt][3] *= al1;
+  }
+  // P^T fragments: {P[token 2t][head g], P[token 2t+1][head g]} (+8 for pb1)
+  const uint32_t pb0 = movmatrix_trans(p01);
+  const uint32_t pb1 = movmatrix_trans(p23);
+  const bool partial = valid < CHUNK;
+  if (partial) {
+    // Zero the V rows past the context (whole 128-byte rows, so the swizzle
+    // does not matter).
+    const int rows = CHUNK - valid;
+    for (int idx = lane; idx < rows * Geo::NSL * 8; idx += 32) {
+      const int r = valid + idx / (Geo::NSL * 8);
+      const int rem = idx % (Geo::NSL * 8);
+      const uint32_t addr = vt + (rem >> 3) * Geo::SLICE_BYTES + r * 128 + ((rem & 7) << 4);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+    }
+    __syncwarp();
+  }
+  // ---- O^T += V^T . P^T ----
+#pragma unroll
+  for (int mt = 0; mt < Geo::MT; ++mt) {
+    const int tok = r8 + ((mat >> 1) << 3);
+    const int colh = mt * 16 + ((mat & 1) << 3);
+    uint32_t a0, a1, a2, a3;
+    ldmatrix_x4_trans(swz_addr(vt, tok, colh), a0, a1, a2, a3);
+    mma_16816(a.o[mt], a0, a1, a2, a3, pb0, pb1);
+  }
+  if (partial) fence_proxy_async_smem();  // generic writes before the next TMA fill
+}
+
+// B operand of S^T = K . Q^T from a [rows = heads][D] fp16 query tile in
+// global or shared memory (generic pointer): Q[head g][16 dims of step ks],
+// zero for g >= G.
+template <int D>
+__device__ __forceinline__ void load_q_fragments(uint32_t (&qb)[D / 16][2], const __half* q_tile,
+                                                 int G, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const __half* qrow = q_tile + (size_t)g * D;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    qb[ks][0] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
+    qb[ks][1] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t + 8) : 0u;
+  }
+}
+
+// Each warp's state into the merge buffers (after the per-head sums are reduced).
+template <int D>
+__device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, float* s_o, int warp,
+                                            int lane) {
+  using Geo = StageGeom<D>;
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    a.l0 += __shfl_xor_sync(0xffffffffu, a.l0, off);
+    a.l1 += __shfl_xor_sync(0xffffffffu, a.l1, off);
+  }
+  if (g == 0) {
+    s_m[warp * 8 + 2 * t] = a.m0;
+    s_m[warp * 8 + 2 * t + 1] = a.m1;
+    s_l[warp * 8 + 2 * t] = a.l0;
+    s_l[warp * 8 + 2 * t + 1] = a.l1;
+  }
+  float* so = s_o + warp * 8 * Geo::OSTRIDE;
+#pragma unroll
+  for (int mt = 0; mt < Geo::MT; ++mt) {
+    so[(2 * t) * Geo::OSTRIDE + mt * 16 + g] = a.o[mt][0];
+    so[(2 * t + 1) * Geo::OSTRIDE + mt * 16 + g] = a.o[mt][1];
+    so[(2 * t) * Geo::OSTRIDE + mt * 16 + g + 8] = a.o[mt][2];
+    so[(2 * t + 1) * Geo::OSTRIDE + mt * 16 + g + 8] = a.o[mt][3];
+  }
+}
+
+// Merges the four warps' states of item (b, kvh, part) and stores the result:
+// the fp16 output when the item is the whole context, else the partition's
+// (max, sum, unnormalised output) for the merge kernel.
+template <int D>
+__device__ __forceinline__ void store_item(const float* s_m, const float* s_l, const float* s_o,
+                                           const DecodeParams& p, int b, int kvh, int part, int G,
+                                           bool whole) {
+  using Geo = StageGeom<D>;
+  for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+    const int head = idx / D;
+    const int d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * 8 + head]);
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float a = rescale_factor(s_m[w * 8 + head], M);
+      num = fmaf(a, s_o[(w * 8 + head) * Geo::OSTRIDE + d], num);
+      den = fmaf(a, s_l[w * 8 + head], den);
+    }
+    const size_t bh = (size_t)b * p.num_heads + kvh * G + head;
+    if (whole) {
+      p.out[bh * D + d] = __float2half_rn(num / den);
+    } else {
+      const size_t slot = bh * p.num_parts + part;
+      p.ws_o[slot * D + d] = num;
+      if (d == 0) {
+        p.ws_ml[slot * 2] = M;
+        p.ws_ml[slot * 2 + 1] = den;
+      }
+    }
+  }
+}
+
+// ---- one CTA per (sequence, kv head, partition) ---------------------------------
+
 template <int D, int BS, bool SPLIT>
 __global__ void __launch_bounds__((NW + 1) * 32)
     mma_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                       const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
-  constexpr int CHUNK = 16;                    // tokens per stage
-  constexpr int CB = BS < CHUNK ? BS : CHUNK;  // rows per TMA box
-  constexpr int NB = CHUNK / CB;               // boxes (blocks) per stage and slice
-  constexpr int NSL = D / 64;                  // 64-column slices (128 bytes)
-  constexpr uint32_t SLICE_BYTES = CHUNK * 128;
-  constexpr uint32_t TILE_BYTES = NSL * SLICE_BYTES;  // K (or V) of one stage
-  constexpr uint32_t BOX_BYTES = CB * 128;
-  constexpr int MT = D / 16;                   // 16-wide slices of D
-  constexpr int OSTRIDE = D + 4;               // padded merge rows (fewer bank conflicts)
-  static_assert(32 % NB == 0, "stages must not straddle a window of 32 table entries");
-
+  using Geo = StageGeom<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int stages = p.stages;
   const uint32_t ring = smem_u32(smem);  // [stages][K tile | V tile], 1024-aligned
-  int* s_ids = reinterpret_cast<int*>(smem + (size_t)stages * 2 * TILE_BYTES);  // [32]
+  int* s_ids = reinterpret_cast<int*>(smem + (size_t)stages * 2 * Geo::TILE_BYTES);  // [32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_ids + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * stages);
   // merge buffers, placed over the ring once every stage has been consumed
@@ -118,7 +387,6 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   const int ntok = min(L, tok0 + p.part_tokens) - tok0;
   if (ntok <= 0) return;
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
-  const int blk0 = tok0 / BS;
   const int nblk = (ntok + BS - 1) / BS;
 
   if (threadIdx.x == 0) {
@@ -137,85 +405,20 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       prefetch_tensor_map(&k_map);
       prefetch_tensor_map(&v_map);
     }
-    const int32_t* row = p.block_tables + (size_t)b * p.max_blocks + blk0;
-    const uint64_t policy = l2_evict_first_policy();
-    int issued = 0;
-    for (int w0 = 0; w0 < nblk; w0 += 32) {
-      if (w0 + lane < nblk) {
-        int id = row[w0 + lane];
-        if (id < 0 || id >= p.num_blocks) {
-          flag_error(p.err, ERR_BLOCK_ID);
-          id = 0;
-        }
-        s_ids[lane] = id;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        const int c_end = min(nchunks, (w0 + 32) * BS / CHUNK);
-        for (int c = w0 * BS / CHUNK; c < c_end && !*abort_flag; ++c) {
-          const int st = c % stages;
-          const int round = c / stages;
-          if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
-            *abort_flag = 1;
-            flag_error(p.err, ERR_TIMEOUT);
-            break;
-          }
-          const uint32_t full = smem_u32(&bars[st]);
-          const uint32_t kdst = ring + (uint32_t)st * 2 * TILE_BYTES;
-          const uint32_t vdst = kdst + TILE_BYTES;
-          const int first = c * NB;  // first block of the stage (bs 8), or unused
-          const int nb = BS >= CHUNK ? 1 : min(NB, nblk - first);
-          mbar_arrive_expect_tx(full, 2u * nb * NSL * BOX_BYTES);
-          for (int k = 0; k < nb; ++k) {
-            int y;
-            if (BS >= CHUNK) {
-              const int tok = c * CHUNK;
-              y = (s_ids[tok / BS - w0] * p.num_kv_heads + kvh) * BS + tok % BS;
-            } else {
-              y = (s_ids[first + k - w0] * p.num_kv_heads + kvh) * BS;
-            }
-#pragma unroll
-            for (int sl = 0; sl < NSL; ++sl) {
-              const uint32_t off = sl * SLICE_BYTES + k * BOX_BYTES;
-              tensor_load_2d(kdst + off, &k_map, sl * 64, y, full, policy);
-              tensor_load_2d(vdst + off, &v_map, sl * 64, y, full, policy);
-            }
-          }
-          issued = c + 1;
-        }
-      }
-      __syncwarp();
-    }
-    if (lane == 0 && *abort_flag) {
-      for (int c = max(0, issued - stages); c < issued; ++c)
-        mbar_wait(smem_u32(&bars[c % stages]), (c / stages) & 1);
-    }
+    const int32_t* row = p.block_tables + (size_t)b * p.max_blocks + tok0 / BS;
+    int issued_end = 0;
+    produce_item<D, BS>(row, nblk, nchunks, 0, kvh, p, s_ids, bars, stages, ring, &k_map, &v_map,
+                        l2_evict_first_policy(), abort_flag, lane, &issued_end);
+    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued_end);
     return;
   }
 
   // ---------------- consumer warps ----------------
-  const int g = lane >> 2;  // fragment row group
-  const int t = lane & 3;   // fragment column pair
-  // B operand of S^T = K . Q^T: Q[head g][16 dims of step ks], zero for g >= G.
-  uint32_t qb[MT][2];
-  {
-    const __half* qrow = p.q + ((size_t)b * p.num_heads + kvh * G + g) * D;
-#pragma unroll
-    for (int ks = 0; ks < MT; ++ks) {
-      qb[ks][0] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
-      qb[ks][1] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t + 8) : 0u;
-    }
-  }
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2t, 2t+1 (log2 units)
-  float l0 = 0.f, l1 = 0.f;              // this lane's part of the running sums
-  float o[MT][4];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-
-  const int mat = lane >> 3;  // ldmatrix: which 8x8 matrix this lane addresses
-  const int r8 = lane & 7;    // ... and which of its rows
-  bool gave_up = false;       // this warp stopped before consuming all its stages
-
+  uint32_t qb[Geo::MT][2];
+  load_q_fragments<D>(qb, p.q + ((size_t)b * p.num_heads + kvh * G) * D, G, lane);
+  Acc<D> a;
+  a.reset();
+  bool gave_up = false;  // this warp stopped before consuming all its stages
   for (int c = 0; c < nchunks; ++c) {
     const int st = c % stages;
     if (st % NW != warp) continue;  // this stage belongs to another warp
@@ -232,129 +435,273 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       gave_up = true;
       break;
     }
-    const uint32_t kt = ring + (uint32_t)st * 2 * TILE_BYTES;
-    const uint32_t vt = kt + TILE_BYTES;
-    const int valid = min(CHUNK, ntok - c * CHUNK);  // rows of this stage inside the context
-
-    // ---- S^T = K . Q^T for 16 tokens ----
-    float sc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < MT; ++ks) {
-      const int tok = r8 + ((mat & 1) << 3);
-      const int colh = ks * 16 + ((mat >> 1) << 3);
-      uint32_t a0, a1, a2, a3;
-      ldmatrix_x4(swz_addr<CHUNK>(kt, tok, colh), a0, a1, a2, a3);
-      mma_16816(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-    }
-    const float s0 = g < valid ? sc[0] * p.scale_log2 : -INFINITY;
-    const float s1 = g < valid ? sc[1] * p.scale_log2 : -INFINITY;
-    const float s2 = g + 8 < valid ? sc[2] * p.scale_log2 : -INFINITY;
-    const float s3 = g + 8 < valid ? sc[3] * p.scale_log2 : -INFINITY;
-    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: row 0 is valid
-    const float al0 = rescale_factor(m0, mn0), al1 = rescale_factor(m1, mn1);
-    m0 = mn0;
-    m1 = mn1;
-    const uint32_t p01 = pack_half2(exp2f(s0 - mn0), exp2f(s1 - mn1));  // token g
-    const uint32_t p23 = pack_half2(exp2f(s2 - mn0), exp2f(s3 - mn1));  // token g + 8
-    const float2 f01 = unpack_half2(p01), f23 = unpack_half2(p23);
-    l0 = fmaf(l0, al0, f01.x + f23.x);
-    l1 = fmaf(l1, al1, f01.y + f23.y);
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      o[mt][0] *= al0;
-      o[mt][1] *= al1;
-      o[mt][2] *= al0;
-      o[mt][3] *= al1;
-    }
-    // P^T fragments: {P[token 2t][head g], P[token 2t+1][head g]} (+8 for pb1)
-    const uint32_t pb0 = movmatrix_trans(p01);
-    const uint32_t pb1 = movmatrix_trans(p23);
-    const bool partial = valid < CHUNK;
-    if (partial) {
-      // Zero the V rows past the context (whole 128-byte rows, so the swizzle
-      // does not matter).
-      const int rows = CHUNK - valid;
-      for (int idx = lane; idx < rows * NSL * 8; idx += 32) {
-        const int r = valid + idx / (NSL * 8);
-        const int rem = idx % (NSL * 8);
-        const uint32_t addr = vt + (rem >> 3) * SLICE_BYTES + r * 128 + ((rem & 7) << 4);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
-      }
-      __syncwarp();
-    }
-    // ---- O^T += V^T . P^T ----
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int tok = r8 + ((mat >> 1) << 3);
-      const int colh = mt * 16 + ((mat & 1) << 3);
-      uint32_t a0, a1, a2, a3;
-      ldmatrix_x4_trans(swz_addr<CHUNK>(vt, tok, colh), a0, a1, a2, a3);
-      mma_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
-    }
-    if (partial) fence_proxy_async_smem();  // generic writes before the next TMA fill
+    consume_stage<D>(a, ring + (uint32_t)st * 2 * Geo::TILE_BYTES, min(CHUNK, ntok - c * CHUNK),
+                     qb, p.scale_log2, lane);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&bars[stages + st]));
   }
 
-  // ---- merge the four warps' partial softmax states ----
-#pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-  }
   // When every warp consumed all its stages, every copy has landed and the ring
   // can hold the merge buffers.  Otherwise copies may still be landing: give up
   // (the error word already says the output is invalid).
   if (named_barrier_or(1, NW * 32, gave_up)) return;
-  if (g == 0) {
-    s_m[warp * 8 + 2 * t] = m0;
-    s_m[warp * 8 + 2 * t + 1] = m1;
-    s_l[warp * 8 + 2 * t] = l0;
-    s_l[warp * 8 + 2 * t + 1] = l1;
-  }
-  float* so = s_o + warp * 8 * OSTRIDE;
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
-    so[(2 * t) * OSTRIDE + mt * 16 + g] = o[mt][0];
-    so[(2 * t + 1) * OSTRIDE + mt * 16 + g] = o[mt][1];
-    so[(2 * t) * OSTRIDE + mt * 16 + g + 8] = o[mt][2];
-    so[(2 * t + 1) * OSTRIDE + mt * 16 + g + 8] = o[mt][3];
-  }
+  // the merge kernel (if any) may be scheduled once every CTA got here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  write_state<D>(a, s_m, s_l, s_o, warp, lane);
   named_barrier_sync(1, NW * 32);
-  for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
-    const int head = idx / D;
-    const int d = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * 8 + head]);
-    float num = 0.f, den = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float a = rescale_factor(s_m[w * 8 + head], M);
-      num = fmaf(a, s_o[(w * 8 + head) * OSTRIDE + d], num);
-      den = fmaf(a, s_l[w * 8 + head], den);
+  store_item<D>(s_m, s_l, s_o, p, b, kvh, part, G, !SPLIT || L <= p.part_tokens);
+}
+
+// ---- persistent split-K kernel ---------------------------------------------------
+
+struct PersistentArgs {
+  unsigned int* ticket;  // zeroed before the launch
+};
+
+// Work item of ticket t: every full partition (part_tokens tokens) comes first,
+// in (sequence, partition) order, then the partial last partitions in sequence
+// order; kv head fastest.  pref_f[b] / pref_p[b] count the full / partial
+// partitions of sequences before b.  Returns (b, kvh, part, tokens).
+__device__ __forceinline__ int4 item_of_ticket(int t, int num_kv_heads, int num_seqs,
+                                               int part_tokens, const int* pref_f,
+                                               const int* pref_p, const int* lens) {
+  const int kvh = t % num_kv_heads;
+  int u = t / num_kv_heads;
+  const int total_f = pref_f[num_seqs];
+  const int* pref = pref_f;
+  if (u >= total_f) {
+    u -= total_f;
+    pref = pref_p;
+  }
+  // largest b with pref[b] <= u (pref is non-decreasing, pref[0] = 0)
+  int lo = 0, hi = num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pref[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  const int b = lo;
+  if (pref == pref_f) return make_int4(b, kvh, u - pref_f[b], part_tokens);
+  const int L = lens[b];
+  return make_int4(b, kvh, L / part_tokens, L % part_tokens);
+}
+
+template <int D, int BS>
+__global__ void __launch_bounds__((NW + 1) * 32)
+    mma_decode_persistent_kernel(const __grid_constant__ CUtensorMap k_map,
+                                 const __grid_constant__ CUtensorMap v_map, const DecodeParams p,
+                                 const PersistentArgs pa) {
+  using Geo = StageGeom<D>;
+  constexpr uint32_t QTILE_BYTES = 8 * D * 2;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int stages = p.stages;
+  const int B = p.num_seqs;
+  const uint32_t ring = smem_u32(smem);
+  unsigned char* cur = smem + (size_t)stages * 2 * Geo::TILE_BYTES;
+  __half* s_q = reinterpret_cast<__half*>(cur);  // [IQ][8][D]
+  cur += IQ * QTILE_BYTES;
+  float* s_m = reinterpret_cast<float*>(cur);    // [NW][8]
+  float* s_l = s_m + NW * 8;                     // [NW][8]
+  float* s_o = s_l + NW * 8;                     // [NW][8][OSTRIDE]
+  cur += Geo::MERGE_BYTES;
+  int4* s_item = reinterpret_cast<int4*>(cur);   // [IQ]
+  cur += IQ * sizeof(int4);
+  int* s_lens = reinterpret_cast<int*>(cur);     // [B]
+  int* pref_f = s_lens + B;                      // [B + 1]
+  int* pref_p = pref_f + B + 1;                  // [B + 1]
+  int* s_ids = pref_p + B + 1;                   // [32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(s_ids + 32) + 7) & ~uintptr_t(7));
+  uint64_t* ifull = bars + 2 * stages;           // [IQ]: item descriptor + query tile landed
+  uint64_t* iempty = ifull + IQ;                 // [IQ]: NW consumer warps done with the slot
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(iempty + IQ);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = p.num_heads / p.num_kv_heads;
+  const int pt = p.part_tokens;
+
+  // per-sequence partition counts, then their prefix sums (warp 0)
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    int L = p.context_lens[b];
+    if (L > p.max_context_len || L <= 0) {
+      if (blockIdx.x == 0) flag_error(p.err, ERR_CONTEXT_LEN);
+      L = L <= 0 ? 0 : p.max_context_len;
     }
-    const size_t bh = (size_t)b * p.num_heads + kvh * G + head;
-    if (!SPLIT) {
-      p.out[bh * D + d] = __float2half_rn(num / den);
-    } else {
-      const size_t slot = bh * p.num_parts + part;
-      p.ws_o[slot * D + d] = num;
-      if (d == 0) {
-        p.ws_ml[slot * 2] = M;
-        p.ws_ml[slot * 2 + 1] = den;
+    s_lens[b] = L;
+    pref_f[b + 1] = L / pt;
+    pref_p[b + 1] = (L % pt) != 0 ? 1 : 0;
+  }
+  if (threadIdx.x == 0) {
+    pref_f[0] = 0;
+    pref_p[0] = 0;
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);
+      mbar_init(smem_u32(&bars[stages + s]), 1);
+    }
+    for (int s = 0; s < IQ; ++s) {
+      mbar_init(smem_u32(&ifull[s]), 1);
+      mbar_init(smem_u32(&iempty[s]), NW);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry_f = 0, carry_p = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int b = b0 + lane;
+      int vf = b < B ? pref_f[b + 1] : 0;
+      int vp = b < B ? pref_p[b + 1] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int xf = __shfl_up_sync(0xffffffffu, vf, o);
+        const int xp = __shfl_up_sync(0xffffffffu, vp, o);
+        if (lane >= o) {
+          vf += xf;
+          vp += xp;
+        }
       }
+      if (b < B) {
+        pref_f[b + 1] = vf + carry_f;
+        pref_p[b + 1] = vp + carry_p;
+      }
+      carry_f += __shfl_sync(0xffffffffu, vf, 31);
+      carry_p += __shfl_sync(0xffffffffu, vp, 31);
     }
   }
+  __syncthreads();
+  const int total = p.num_kv_heads * (pref_f[B] + pref_p[B]);
+
+  if (warp == NW) {
+    // ---------------- producer warp ----------------
+    if (lane == 0) {
+      prefetch_tensor_map(&k_map);
+      prefetch_tensor_map(&v_map);
+    }
+    const uint64_t policy = l2_evict_first_policy();
+    int gc = 0;          // global index of the next chunk
+    int issued_end = 0;  // one past the last chunk issued
+    // tickets are taken one item ahead, so the atomic's latency hides behind
+    // the current item's copies
+    int t_next = lane == 0 ? (int)atomicAdd(pa.ticket, 1u) : 0;
+    for (int it = 0;; ++it) {
+      int t = __shfl_sync(0xffffffffu, t_next, 0);
+      if (lane == 0 && t < total) t_next = (int)atomicAdd(pa.ticket, 1u);
+      const bool done = t >= total || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
+      const int4 d = done ? make_int4(0, 0, 0, 0)
+                          : item_of_ticket(t, p.num_kv_heads, B, pt, pref_f, pref_p, s_lens);
+      const int qs = it % IQ;
+      bool ok = true;
+      if (lane == 0) {
+        if (it >= IQ && !mbar_wait(smem_u32(&iempty[qs]), ((it / IQ) - 1) & 1)) {
+          *abort_flag = 1;
+          flag_error(p.err, ERR_TIMEOUT);
+          ok = false;
+        }
+        if (ok) {
+          s_item[qs] = d;
+          const uint32_t full = smem_u32(&ifull[qs]);
+          if (!done) {
+            mbar_arrive_expect_tx(full, (uint32_t)(G * D * 2));
+            bulk_load(smem_u32(s_q) + qs * QTILE_BYTES,
+                      p.q + ((size_t)d.x * p.num_heads + d.y * G) * D, (uint32_t)(G * D * 2), full,
+                      policy);
+          } else {
+            mbar_arrive(full);  // the end marker (tokens = 0)
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+      if (done || !ok) break;
+      const int tok0 = d.z * pt;
+      const int nchunks = (d.w + CHUNK - 1) / CHUNK;
+      const int nblk = (d.w + BS - 1) / BS;
+      const int32_t* row = p.block_tables + (size_t)d.x * p.max_blocks + tok0 / BS;
+      if (!produce_item<D, BS>(row, nblk, nchunks, gc, d.y, p, s_ids, bars, stages, ring, &k_map,
+                               &v_map, policy, abort_flag, lane, &issued_end))
+        break;
+      gc += nchunks;
+    }
+    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued_end);
+    return;
+  }
+
+  // ---------------- consumer warps ----------------
+  int gc = 0;
+  for (int it = 0;; ++it) {
+    const int qs = it % IQ;
+    bool stop = false, gave_up = false;
+    int4 d = make_int4(0, 0, 0, 0);
+    const bool ready = mbar_wait(smem_u32(&ifull[qs]), (it / IQ) & 1);
+    if (!__all_sync(0xffffffffu, ready)) {
+      if (lane == 0) {
+        *abort_flag = 1;
+        flag_error(p.err, ERR_TIMEOUT);
+      }
+      stop = true;
+    } else {
+      d = s_item[qs];
+      stop = d.w == 0;
+    }
+    Acc<D> a;
+    a.reset();
+    if (!stop) {
+      uint32_t qb[Geo::MT][2];
+      load_q_fragments<D>(qb, s_q + qs * (8 * D), G, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&iempty[qs]));  // descriptor and query tile consumed
+      const int nchunks = (d.w + CHUNK - 1) / CHUNK;
+      for (int j = 0; j < nchunks && !gave_up; ++j) {
+        const int c = gc + j;
+        const int st = c % stages;
+        if (st % NW != warp) continue;
+        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {
+          gave_up = true;
+          break;
+        }
+        const bool ok = mbar_wait(smem_u32(&bars[st]), (c / stages) & 1);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            flag_error(p.err, ERR_TIMEOUT);
+          }
+          gave_up = true;
+          break;
+        }
+        consume_stage<D>(a, ring + (uint32_t)st * 2 * Geo::TILE_BYTES,
+                         min(CHUNK, d.w - j * CHUNK), qb, p.scale_log2, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars[stages + st]));
+      }
+      gc += nchunks;
+    }
+    // All four warps decide together: the end of the work, or an abort anywhere.
+    if (named_barrier_or(1, NW * 32, stop || gave_up)) break;
+    write_state<D>(a, s_m, s_l, s_o, warp, lane);
+    named_barrier_sync(1, NW * 32);
+    store_item<D>(s_m, s_l, s_o, p, d.x, d.y, d.z, G, s_lens[d.x] <= pt);
+  }
+  // the merge kernel may be scheduled once every CTA got here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 constexpr int MAX_DEVICES = 64;
+
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes, std::atomic<int>* granted) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+  if (granted[dev].load(std::memory_order_relaxed) >= (int)bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) granted[dev].store((int)bytes, std::memory_order_relaxed);
+  return e;
+}
 
 template <int D, int BS, bool SPLIT>
 cudaError_t launch_mma_instance(const DecodeParams& p, const CUtensorMap& km,
@@ -362,19 +709,47 @@ cudaError_t launch_mma_instance(const DecodeParams& p, const CUtensorMap& km,
   static std::atomic<int> granted[MAX_DEVICES];
   auto kernel = mma_decode_kernel<D, BS, SPLIT>;
   const size_t smem = mma_smem_bytes(D, BS, p.stages);
-  if (smem > 48 * 1024) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
-    if (granted[dev].load(std::memory_order_relaxed) < (int)smem) {
-      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      granted[dev].store((int)smem, std::memory_order_relaxed);
-    }
-  }
+  cudaError_t e = allow_smem(kernel, smem, granted);
+  if (e != cudaSuccess) return e;
   const dim3 grid(p.num_kv_heads, p.num_seqs, SPLIT ? p.num_parts : 1);
   kernel<<<grid, (NW + 1) * 32, smem, stream>>>(km, vm, p);
+  return cudaGetLastError();
+}
+
+template <int D, int BS>
+cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap& km,
+                                       const CUtensorMap& vm, unsigned int* ticket,
+                                       cudaStream_t stream) {
+  static std::atomic<int> granted[MAX_DEVICES];
+  static std::atomic<int> blocks_per_sm[MAX_DEVICES];
+  static std::atomic<int> blocks_smem[MAX_DEVICES];
+  auto kernel = mma_decode_persistent_kernel<D, BS>;
+  const size_t smem = mma_persistent_smem_bytes(D, p.stages, p.num_seqs);
+  cudaError_t e = allow_smem(kernel, smem, granted);
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+  if (blocks_smem[dev].load(std::memory_order_relaxed) != (int)smem) {
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, (NW + 1) * 32, smem);
+    if (e != cudaSuccess) return e;
+    blocks_per_sm[dev].store(n < 1 ? 1 : n, std::memory_order_relaxed);
+    blocks_smem[dev].store((int)smem, std::memory_order_relaxed);
+  }
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  // no more CTAs than work items can exist
+  const long long items = (long long)p.num_kv_heads * p.num_seqs * p.num_parts;
+  long long ctas = (long long)sms * blocks_per_sm[dev].load(std::memory_order_relaxed);
+  if (ctas > items) ctas = items;
+  e = cudaMemsetAsync(ticket, 0, sizeof(unsigned int), stream);
+  if (e != cudaSuccess) return e;
+  PersistentArgs pa;
+  pa.ticket = ticket;
+  kernel<<<(unsigned)ctas, (NW + 1) * 32, smem, stream>>>(km, vm, p, pa);
   return cudaGetLastError();
 }
 
@@ -382,16 +757,19 @@ cudaError_t launch_mma_instance(const DecodeParams& p, const CUtensorMap& km,
 
 size_t mma_stage_bytes(int head_dim, int block_size) {
   (void)block_size;  // a stage is 16 tokens whatever the block size
-  return 2ull * 16 * head_dim * sizeof(__half);
-}
-
-size_t mma_merge_bytes(int head_dim) {
-  return (size_t)NW * 8 * (2 + head_dim + 4) * sizeof(float);
+  return 2ull * CHUNK * head_dim * sizeof(__half);
 }
 
 size_t mma_smem_bytes(int head_dim, int block_size, int stages) {
   return 1024 /* alignment slack */ + (size_t)stages * mma_stage_bytes(head_dim, block_size) +
          32 * sizeof(int) + 2ull * stages * sizeof(uint64_t) + 16;
+}
+
+size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs) {
+  const size_t merge = (size_t)NW * 8 * (2 + head_dim + 4) * sizeof(float);
+  return 1024 + (size_t)stages * mma_stage_bytes(head_dim, 16) + IQ * 8ull * head_dim * 2 + merge +
+         IQ * sizeof(int4) + (3ull * num_seqs + 2 + 32) * sizeof(int) + 8 +
+         (2ull * stages + 2 * IQ) * sizeof(uint64_t) + 16;
 }
 
 #define PKV_MMA_CASE(D_, BS_)                                                  \
@@ -409,6 +787,24 @@ cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& km, cons
   PKV_MMA_CASE(128, 16)
   PKV_MMA_CASE(128, 32)
   PKV_MMA_CASE(128, 64)
+  return cudaErrorInvalidValue;
+}
+
+#define PKV_MMA_PERSISTENT_CASE(D_, BS_)        \
+  if (p.head_dim == D_ && p.block_size == BS_) \
+    return launch_persistent_instance<D_, BS_>(p, km, vm, ticket, stream);
+
+cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& km,
+                                         const CUtensorMap& vm, unsigned int* ticket,
+                                         cudaStream_t stream) {
+  PKV_MMA_PERSISTENT_CASE(64, 8)
+  PKV_MMA_PERSISTENT_CASE(64, 16)
+  PKV_MMA_PERSISTENT_CASE(64, 32)
+  PKV_MMA_PERSISTENT_CASE(64, 64)
+  PKV_MMA_PERSISTENT_CASE(128, 8)
+  PKV_MMA_PERSISTENT_CASE(128, 16)
+  PKV_MMA_PERSISTENT_CASE(128, 32)
+  PKV_MMA_PERSISTENT_CASE(128, 64)
   return cudaErrorInvalidValue;
 }
 

@@ -1,4 +1,4 @@
-// Paged decode attention on the CUDA cores (sm_100a), and the split-K merge.
+// Paged decode attention on the CUDA cores (sm_100a).
 //
 // What it computes (per sequence b and query head h, kv head h / G):
 //   out[b][h] = softmax_i(scale * q[b][h] . K_b[i]) . V_b,   i < L_b,
@@ -25,7 +25,8 @@
 //    slots may hold anything, NaN included).  Every consumer warp reads every
 //    stage in order, so no warp can run a phase ahead of a stage's barrier.
 //  * With a split, each CTA covers one partition and stores (max, sum,
-//    unnormalised output); split_reduce_kernel merges the partitions.
+//    unnormalised output) for split_merge_kernel; a context that fits in one
+//    partition is finished here and written directly.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -275,9 +276,11 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
 #pragma unroll
     for (int d = 0; d < 8; ++d) acc[d] += __shfl_xor_sync(0xffffffffu, acc[d], o);
   }
+  // the merge kernel (if any) may be scheduled once every CTA got here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (sub == 0) {
     const size_t bh = (size_t)b * p.num_heads + h;
-    if (!SPLIT) {
+    if (!SPLIT || L <= p.part_tokens) {
       uint4 packed;
       packed.x = pack_half2(acc[0] / l, acc[1] / l);
       packed.y = pack_half2(acc[2] / l, acc[3] / l);
@@ -295,34 +298,6 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
       }
     }
   }
-}
-
-// Merge of the partitions of one (sequence, head): with partition maxima m_i,
-// sums l_i and unnormalised outputs o_i, out = sum_i 2^(m_i - M) o_i /
-// sum_i 2^(m_i - M) l_i where M = max_i m_i.  One thread per dim.
-template <int D>
-__global__ void __launch_bounds__(D) split_reduce_kernel(const DecodeParams p) {
-  const int h = blockIdx.x;
-  const int b = blockIdx.y;
-  const int d = threadIdx.x;
-  int L = p.context_lens[b];
-  if (L > p.max_context_len) L = p.max_context_len;  // flagged by the first pass
-  __half* o = p.out + ((size_t)b * p.num_heads + h) * D;
-  if (L <= 0) {
-    o[d] = __float2half_rn(0.f);
-    return;
-  }
-  const int P = (L + p.part_tokens - 1) / p.part_tokens;
-  const size_t base = ((size_t)b * p.num_heads + h) * p.num_parts;
-  float M = -INFINITY;
-  for (int i = 0; i < P; ++i) M = fmaxf(M, p.ws_ml[(base + i) * 2]);
-  float num = 0.f, den = 0.f;
-  for (int i = 0; i < P; ++i) {
-    const float w = rescale_factor(p.ws_ml[(base + i) * 2], M);
-    den = fmaf(w, p.ws_ml[(base + i) * 2 + 1], den);
-    num = fmaf(w, p.ws_o[(base + i) * D + d], num);
-  }
-  o[d] = __float2half_rn(num / den);
 }
 
 constexpr int MAX_DEVICES = 64;
@@ -388,18 +363,6 @@ cudaError_t launch_simt_decode(const DecodeParams& p, int hpc, int kvc, bool spl
   PKV_SIMT_GROUPS(64)
   PKV_SIMT_GROUPS(128)
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_split_reduce(const DecodeParams& p, cudaStream_t stream) {
-  const dim3 grid(p.num_heads, p.num_seqs);
-  if (p.head_dim == 64) {
-    split_reduce_kernel<64><<<grid, 64, 0, stream>>>(p);
-  } else if (p.head_dim == 128) {
-    split_reduce_kernel<128><<<grid, 128, 0, stream>>>(p);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
 }
 
 }  // namespace pkv

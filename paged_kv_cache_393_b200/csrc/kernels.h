@@ -47,8 +47,19 @@ cudaError_t launch_simt_decode(const DecodeParams& p, int hpc, int kvc, bool spl
 cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& k_map,
                               const CUtensorMap& v_map, bool split, cudaStream_t stream);
 
-// Merges the partitions of a split launch into `out`.
+// Persistent split-K tensor-core kernel: a few CTAs per SM take (b, kv head,
+// partition) work items from `ticket` (a workspace word it zeroes first).
+cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& k_map,
+                                         const CUtensorMap& v_map, unsigned int* ticket,
+                                         cudaStream_t stream);
+size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs);
+constexpr int PERSISTENT_MAX_SEQS = 1024;
+
+// Merges the partitions of a split launch into `out` (a programmatic dependent
+// launch after the partition pass on the same stream).
 cudaError_t launch_split_reduce(const DecodeParams& p, cudaStream_t stream);
+size_t split_merge_smem_bytes(int num_parts);
+constexpr int MAX_PARTITIONS = 4096;
 
 // Slot-mapping scatter of new K/V rows into the pools.
 cudaError_t launch_reshape_and_cache(const __half* k, const __half* v, __half* key_cache,

@@ -73,6 +73,7 @@ def _decode(lib, **over):
     (dict(part=32), nat.EWORKSPACE),                  # split without a workspace
     (dict(scale=float("nan")), nat.EINVAL),
     (dict(b=70000), nat.EUNSUPPORTED),
+    (dict(part=16, maxlen=100000, maxblk=6250), nat.EUNSUPPORTED),   # > 4096 partitions
 ])
 def test_decode_rejects_bad_arguments_on_the_host(lib, over, code):
     assert _decode(lib, **over) == code
@@ -87,11 +88,16 @@ def test_workspace_bytes(lib):
     # single pass: no workspace
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, 0) == 0
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, -1) == 0
-    # explicit split: B * H * P * (D + 2) floats
-    assert pkv.paged_attention_workspace_bytes(4, 8, 2, 64, 16, 1000, 256) == 4 * 8 * 4 * 66 * 4
+    # explicit split: B * H * P * (D + 2) floats (CUDA-core kernel, MHA)
+    assert pkv.paged_attention_workspace_bytes(4, 8, 8, 64, 16, 1000, 256) == 4 * 8 * 4 * 66 * 4
+    # tensor-core split-K runs persistent CTAs fed by a ticket word: 16 more bytes
+    assert pkv.paged_attention_workspace_bytes(4, 8, 2, 64, 16, 1000, 256) == 4 * 8 * 4 * 66 * 4 + 16
     # long GQA contexts split automatically into 512-token partitions
     assert pkv.paged_attention_workspace_bytes(128, 64, 8, 128, 16, 16384, 0) == \
-        128 * 64 * 32 * 130 * 4
+        128 * 64 * 32 * 130 * 4 + 16
+    # beyond 1024 sequences the tensor-core split runs one CTA per item: no ticket
+    assert pkv.paged_attention_workspace_bytes(1100, 16, 2, 64, 16, 1000, 512) == \
+        1100 * 16 * 2 * 66 * 4
     assert pkv.paged_attention_workspace_bytes(1, 8, 3, 64, 16, 100, 0) == 0     # rejected shape
 
 

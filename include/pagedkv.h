@@ -109,9 +109,11 @@ PAGEDKV_API int pagedkv_device_errors(unsigned int *flags, int clear);
  *                  and of block_size), computed in parallel and merged by a
  *                  second kernel.
  *   workspace      device scratch of at least paged_attention_workspace_bytes(...)
- *                  bytes (16-byte aligned) when the call splits; may be NULL when
- *                  that function returns 0.  Its contents need no initialization
- *                  and are garbage afterwards.
+ *                  bytes (16-byte aligned): the split-K partial results, and for
+ *                  grouped queries (2..8 query heads per kv head) a work counter;
+ *                  may be NULL when that function returns 0.  Its contents need no
+ *                  initialization and are garbage afterwards; calls that may run
+ *                  at the same time need separate workspaces.
  *
  * num_seqs == 0 is a no-op.  Errors: EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
  */
@@ -124,8 +126,9 @@ PAGEDKV_API int paged_attention_decode(void *out, const void *q,
                            int partition_size, void *workspace, size_t workspace_bytes,
                            void *stream);
 
-/* Workspace bytes paged_attention_decode needs for these arguments (0 when the
- * call runs as a single pass).  Returns 0 for arguments it would reject too. */
+/* Workspace bytes paged_attention_decode needs for these arguments (0 when it
+ * needs none: a single pass over one kv head per query head).  Returns 0 for
+ * arguments it would reject too. */
 PAGEDKV_API size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
                                        int head_dim, int block_size, int max_context_len,
                                        int partition_size);
@@ -139,11 +142,11 @@ PAGEDKV_API size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, 
  * cudaFree (they may synchronize the device).
  *
  * Same arguments, result and errors as paged_attention_decode, minus the
- * workspace: split-K scratch comes from one array compiled into the library,
+ * workspace: its scratch comes from one array compiled into the library,
  * PAGEDKV_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory that every GPU
  * loading the library keeps until the process exits.  It allocates nothing
  * (no cudaMalloc, cudaFree or allocating library call).
- *  - A call whose split needs more scratch (see paged_attention_workspace_bytes)
+ *  - A call that needs more scratch (see paged_attention_workspace_bytes)
  *    returns PAGEDKV_EWORKSPACE and enqueues nothing.
  *  - The first call on a device that needs scratch looks up the array's device
  *    address (cudaGetSymbolAddress); make that first call before any stream

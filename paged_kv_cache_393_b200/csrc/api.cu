@@ -205,12 +205,13 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
       return fail(PAGEDKV_EUNSUPPORTED, "%d partitions exceed %d: use a larger partition_size",
                   p.num_parts, MAX_PARTITIONS);
     p.ws_bytes = (size_t)num_seqs * num_heads * p.num_parts * (head_dim + 2) * sizeof(float);
-    p.persistent = p.mma && num_seqs <= PERSISTENT_MAX_SEQS && !tn.no_persistent;
-    if (p.persistent) p.ws_bytes = ((p.ws_bytes + 15) / 16) * 16 + 16;  // + the ticket word
   } else {
     p.part_tokens = ((max_context_len + block_size - 1) / block_size) * block_size;
     p.num_parts = 1;
   }
+  // the tensor-core path runs persistent CTAs fed by a ticket word in the workspace
+  p.persistent = p.mma && num_seqs <= PERSISTENT_MAX_SEQS && !tn.no_persistent;
+  if (p.persistent) p.ws_bytes = ((p.ws_bytes + 15) / 16) * 16 + 16;
   // ring depth: few stages and many CTAs per SM stream best (measured)
   if (p.mma) {
     // a multiple of the consumer warps, so every warp owns the same number of stages
@@ -298,7 +299,7 @@ int paged_attention_decode(void* out, const void* q, const void* key_cache, cons
   if (plan.mma && (long long)num_blocks * num_kv_heads * block_size > 0x7fffffffLL)
     return fail(PAGEDKV_EUNSUPPORTED, "pool of %lld rows exceeds the tensor-map range",
                 (long long)num_blocks * num_kv_heads * block_size);
-  if (plan.split) {
+  if (plan.ws_bytes > 0) {
     if (!workspace || workspace_bytes < plan.ws_bytes)
       return fail(PAGEDKV_EWORKSPACE, "workspace of %zu bytes required, %zu given", plan.ws_bytes,
                   workspace ? workspace_bytes : (size_t)0);
@@ -344,10 +345,11 @@ int paged_attention_decode(void* out, const void* q, const void* key_cache, cons
     if (st != PAGEDKV_OK) return st;
     if (plan.persistent) {
       const size_t parts_bytes =
-          (size_t)num_seqs * num_heads * plan.num_parts * (head_dim + 2) * sizeof(float);
+          plan.split ? (size_t)num_seqs * num_heads * plan.num_parts * (head_dim + 2) * sizeof(float)
+                     : 0;
       unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
                                                              ((parts_bytes + 15) / 16) * 16);
-      e = launch_mma_decode_persistent(p, km, vm, ticket, s);
+      e = launch_mma_decode_persistent(p, km, vm, ticket, plan.split, s);
     } else {
       e = launch_mma_decode(p, km, vm, plan.split, s);
     }

@@ -20,19 +20,22 @@
 // 16 tokens: 16 rows of one block (bs >= 16) or two whole blocks (bs 8).
 // ldmatrix reads the swizzled tiles without bank conflicts (K plain for the A
 // operand of QK^T, V transposed for the A operand of PV).  Each stage has ONE
-// owner warp, (stage index) mod 4, which consumes every fill of that stage in
+// owner warp, (stage index) mod (consumer warps), which consumes every fill of that stage in
 // order; a warp therefore never waits on a barrier phase that a slower warp
 // has not reached yet (parity waits cannot tell phase k from phase k+2).
-// Four consumer warps, each with its own online softmax, merge through shared
+// The consumer warps (two: small CTAs, more of them per SM, measured best),
+// each with its own online softmax, merge through shared
 // memory.  Rows past the context are masked out of the scores, and the
 // matching V rows are zeroed in shared memory before PV (0 * NaN would poison
 // the sum).
 //
 // Two schedules share this code:
 //  * mma_decode_kernel: one CTA per (sequence, kv head, partition);
-//  * mma_decode_persistent_kernel (split-K): a few CTAs per SM take work items
+//  * mma_decode_persistent_kernel (up to 1024 sequences, split or not): a few
+//    CTAs per SM take work items
 //    (sequence, kv head, partition) from a ticket counter -- every full
-//    partition first, then the partial last partitions -- and the producer
+//    partition first, then the partial last partitions longest first -- and
+//    the producer
 //    streams chunks across item boundaries without draining the ring.  The
 //    items' query tiles travel through a small queue (bulk copies) with their
 //    descriptors, and each finished item is merged while the next streams in.
@@ -46,7 +49,7 @@ namespace {
 
 constexpr int NW = MMA_CONSUMER_WARPS;
 constexpr int CHUNK = 16;  // tokens per ring stage
-constexpr int IQ = 1;      // item-queue depth of the persistent kernel
+constexpr int IQ = 1;      // item-queue depth of the persistent kernel (a deeper queue costs occupancy)
 
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -307,7 +310,7 @@ __device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, f
   }
 }
 
-// Merges the four warps' states of item (b, kvh, part) and stores the result:
+// Merges the consumer warps' states of item (b, kvh, part) and stores the result:
 // the fp16 output when the item is the whole context, else the partition's
 // (max, sum, unnormalised output) for the merge kernel.
 template <int D>
@@ -456,35 +459,38 @@ __global__ void __launch_bounds__((NW + 1) * 32)
 
 struct PersistentArgs {
   unsigned int* ticket;  // zeroed before the launch
+  int write_zeros;       // no merge kernel follows: write the zero outputs of empty contexts
 };
 
 // Work item of ticket t: every full partition (part_tokens tokens) comes first,
-// in (sequence, partition) order, then the partial last partitions in sequence
-// order; kv head fastest.  pref_f[b] / pref_p[b] count the full / partial
-// partitions of sequences before b.  Returns (b, kvh, part, tokens).
+// in (sequence, partition) order, then the partial last partitions, longest
+// first (sequences sorted by their last partition's 16-token chunk count,
+// descending, ties by sequence index), so the items left at the end of the
+// launch are the shortest; kv head fastest.  pref_f[b] counts the full
+// partitions of the sequences before b; by_tail lists the sequences with a
+// partial partition in that order.  Returns (b, kvh, part, tokens).
 __device__ __forceinline__ int4 item_of_ticket(int t, int num_kv_heads, int num_seqs,
                                                int part_tokens, const int* pref_f,
-                                               const int* pref_p, const int* lens) {
+                                               const int* by_tail, const int* lens) {
   const int kvh = t % num_kv_heads;
   int u = t / num_kv_heads;
   const int total_f = pref_f[num_seqs];
-  const int* pref = pref_f;
   if (u >= total_f) {
-    u -= total_f;
-    pref = pref_p;
+    const int b = by_tail[u - total_f];
+    const int L = lens[b];
+    return make_int4(b, kvh, L / part_tokens, L % part_tokens);
   }
-  // largest b with pref[b] <= u (pref is non-decreasing, pref[0] = 0)
+  // largest b with pref_f[b] <= u (non-decreasing, pref_f[0] = 0)
   int lo = 0, hi = num_seqs - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (pref[mid] <= u) lo = mid;
+    if (pref_f[mid] <= u) lo = mid;
     else hi = mid - 1;
   }
-  const int b = lo;
-  if (pref == pref_f) return make_int4(b, kvh, u - pref_f[b], part_tokens);
-  const int L = lens[b];
-  return make_int4(b, kvh, L / part_tokens, L % part_tokens);
+  return make_int4(lo, kvh, u - pref_f[lo], part_tokens);
 }
+
+constexpr int TAIL_KEYS = 256;  // chunk-count keys of the partial-partition sort
 
 template <int D, int BS>
 __global__ void __launch_bounds__((NW + 1) * 32)
@@ -510,8 +516,10 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   cur += IQ * sizeof(int4);
   int* s_lens = reinterpret_cast<int*>(cur);     // [B]
   int* pref_f = s_lens + B;                      // [B + 1]
-  int* pref_p = pref_f + B + 1;                  // [B + 1]
-  int* s_ids = pref_p + B + 1;                   // [32]
+  int* by_tail = pref_f + B + 1;                 // [B]: sequences with a partial partition
+  int* tail_run = by_tail + B;                   // [TAIL_KEYS]: counts, then insert positions
+  int* s_num_tail = tail_run + TAIL_KEYS;        // [1]: sequences with a partial partition
+  int* s_ids = s_num_tail + 1;                   // [32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(s_ids + 32) + 7) & ~uintptr_t(7));
   uint64_t* ifull = bars + 2 * stages;           // [IQ]: item descriptor + query tile landed
@@ -523,7 +531,9 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   const int G = p.num_heads / p.num_kv_heads;
   const int pt = p.part_tokens;
 
-  // per-sequence partition counts, then their prefix sums (warp 0)
+  // per-sequence partition counts; the partial tails' chunk-count keys
+  for (int k = threadIdx.x; k < TAIL_KEYS; k += blockDim.x) tail_run[k] = 0;
+  __syncthreads();
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     int L = p.context_lens[b];
     if (L > p.max_context_len || L <= 0) {
@@ -531,12 +541,16 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       L = L <= 0 ? 0 : p.max_context_len;
     }
     s_lens[b] = L;
+    if (L == 0 && pa.write_zeros && blockIdx.x == 0) {
+      for (int i = 0; i < p.num_heads * D; ++i)
+        p.out[(size_t)b * p.num_heads * D + i] = __float2half_rn(0.f);
+    }
     pref_f[b + 1] = L / pt;
-    pref_p[b + 1] = (L % pt) != 0 ? 1 : 0;
+    const int tail = L % pt;
+    if (tail) atomicAdd(&tail_run[min(TAIL_KEYS - 1, (tail + CHUNK - 1) / CHUNK)], 1);
   }
   if (threadIdx.x == 0) {
     pref_f[0] = 0;
-    pref_p[0] = 0;
     for (int s = 0; s < stages; ++s) {
       mbar_init(smem_u32(&bars[s]), 1);
       mbar_init(smem_u32(&bars[stages + s]), 1);
@@ -550,30 +564,52 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   }
   __syncthreads();
   if (warp == 0) {
-    int carry_f = 0, carry_p = 0;
+    // inclusive prefix of the full-partition counts
+    int carry = 0;
     for (int b0 = 0; b0 < B; b0 += 32) {
       const int b = b0 + lane;
-      int vf = b < B ? pref_f[b + 1] : 0;
-      int vp = b < B ? pref_p[b + 1] : 0;
+      int v = b < B ? pref_f[b + 1] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int xf = __shfl_up_sync(0xffffffffu, vf, o);
-        const int xp = __shfl_up_sync(0xffffffffu, vp, o);
-        if (lane >= o) {
-          vf += xf;
-          vp += xp;
-        }
+        const int x = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += x;
       }
-      if (b < B) {
-        pref_f[b + 1] = vf + carry_f;
-        pref_p[b + 1] = vp + carry_p;
+      if (b < B) pref_f[b + 1] = v + carry;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    // first position of every key in descending key order
+    carry = 0;
+    for (int k0 = TAIL_KEYS - 32; k0 >= 0; k0 -= 32) {
+      const int k = k0 + 31 - lane;  // lane 0 takes the largest key of the group
+      const int c = tail_run[k];
+      int v = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += x;
       }
-      carry_f += __shfl_sync(0xffffffffu, vf, 31);
-      carry_p += __shfl_sync(0xffffffffu, vp, 31);
+      tail_run[k] = carry + v - c;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) *s_num_tail = carry;
+    __syncwarp();
+    // stable placement: sequences in index order within each key
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int b = b0 + lane;
+      const int tail = b < B ? s_lens[b] % pt : 0;
+      const int key = tail ? min(TAIL_KEYS - 1, (tail + CHUNK - 1) / CHUNK) : -1 - lane;
+      const unsigned same = __match_any_sync(0xffffffffu, key);
+      if (tail) {
+        const int rank = __popc(same & ((1u << lane) - 1));
+        by_tail[tail_run[key] + rank] = b;
+      }
+      __syncwarp();
+      if (tail && (same & ((1u << lane) - 1)) == 0) tail_run[key] += __popc(same);
+      __syncwarp();
     }
   }
   __syncthreads();
-  const int total = p.num_kv_heads * (pref_f[B] + pref_p[B]);
+  const int total = p.num_kv_heads * (pref_f[B] + *s_num_tail);
 
   if (warp == NW) {
     // ---------------- producer warp ----------------
@@ -584,15 +620,19 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     const uint64_t policy = l2_evict_first_policy();
     int gc = 0;          // global index of the next chunk
     int issued_end = 0;  // one past the last chunk issued
-    // tickets are taken one item ahead, so the atomic's latency hides behind
-    // the current item's copies
-    int t_next = lane == 0 ? (int)atomicAdd(pa.ticket, 1u) : 0;
+    // A ticket is taken when the previous item has been issued: taking them
+    // earlier reserves work a CTA cannot start yet and unbalances the end.
+    auto next_item = [&](int4* item) {
+      const int t = __shfl_sync(0xffffffffu, lane == 0 ? (int)atomicAdd(pa.ticket, 1u) : 0, 0);
+      *item = t < total ? item_of_ticket(t, p.num_kv_heads, B, pt, pref_f, by_tail, s_lens)
+                        : make_int4(0, 0, 0, 0);
+      return t < total;
+    };
+    int4 d;
+    bool have = next_item(&d);
     for (int it = 0;; ++it) {
-      int t = __shfl_sync(0xffffffffu, t_next, 0);
-      if (lane == 0 && t < total) t_next = (int)atomicAdd(pa.ticket, 1u);
-      const bool done = t >= total || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
-      const int4 d = done ? make_int4(0, 0, 0, 0)
-                          : item_of_ticket(t, p.num_kv_heads, B, pt, pref_f, pref_p, s_lens);
+      const bool done = !have || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
+      if (done) d = make_int4(0, 0, 0, 0);
       const int qs = it % IQ;
       bool ok = true;
       if (lane == 0) {
@@ -616,14 +656,14 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       }
       ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
       if (done || !ok) break;
-      const int tok0 = d.z * pt;
       const int nchunks = (d.w + CHUNK - 1) / CHUNK;
       const int nblk = (d.w + BS - 1) / BS;
-      const int32_t* row = p.block_tables + (size_t)d.x * p.max_blocks + tok0 / BS;
+      const int32_t* row = p.block_tables + (size_t)d.x * p.max_blocks + d.z * pt / BS;
       if (!produce_item<D, BS>(row, nblk, nchunks, gc, d.y, p, s_ids, bars, stages, ring, &k_map,
                                &v_map, policy, abort_flag, lane, &issued_end))
         break;
       gc += nchunks;
+      have = next_item(&d);
     }
     if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued_end);
     return;
@@ -678,7 +718,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       }
       gc += nchunks;
     }
-    // All four warps decide together: the end of the work, or an abort anywhere.
+    // All consumer warps decide together: the end of the work, or an abort anywhere.
     if (named_barrier_or(1, NW * 32, stop || gave_up)) break;
     write_state<D>(a, s_m, s_l, s_o, warp, lane);
     named_barrier_sync(1, NW * 32);
@@ -718,7 +758,7 @@ cudaError_t launch_mma_instance(const DecodeParams& p, const CUtensorMap& km,
 
 template <int D, int BS>
 cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap& km,
-                                       const CUtensorMap& vm, unsigned int* ticket,
+                                       const CUtensorMap& vm, unsigned int* ticket, bool split,
                                        cudaStream_t stream) {
   static std::atomic<int> granted[MAX_DEVICES];
   static std::atomic<int> blocks_per_sm[MAX_DEVICES];
@@ -749,6 +789,7 @@ cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap&
   if (e != cudaSuccess) return e;
   PersistentArgs pa;
   pa.ticket = ticket;
+  pa.write_zeros = split ? 0 : 1;
   kernel<<<(unsigned)ctas, (NW + 1) * 32, smem, stream>>>(km, vm, p, pa);
   return cudaGetLastError();
 }
@@ -768,7 +809,7 @@ size_t mma_smem_bytes(int head_dim, int block_size, int stages) {
 size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs) {
   const size_t merge = (size_t)NW * 8 * (2 + head_dim + 4) * sizeof(float);
   return 1024 + (size_t)stages * mma_stage_bytes(head_dim, 16) + IQ * 8ull * head_dim * 2 + merge +
-         IQ * sizeof(int4) + (3ull * num_seqs + 2 + 32) * sizeof(int) + 8 +
+         IQ * sizeof(int4) + (3ull * num_seqs + 1 + TAIL_KEYS + 1 + 32) * sizeof(int) + 8 +
          (2ull * stages + 2 * IQ) * sizeof(uint64_t) + 16;
 }
 
@@ -792,10 +833,10 @@ cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& km, cons
 
 #define PKV_MMA_PERSISTENT_CASE(D_, BS_)        \
   if (p.head_dim == D_ && p.block_size == BS_) \
-    return launch_persistent_instance<D_, BS_>(p, km, vm, ticket, stream);
+    return launch_persistent_instance<D_, BS_>(p, km, vm, ticket, split, stream);
 
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& km,
-                                         const CUtensorMap& vm, unsigned int* ticket,
+                                         const CUtensorMap& vm, unsigned int* ticket, bool split,
                                          cudaStream_t stream) {
   PKV_MMA_PERSISTENT_CASE(64, 8)
   PKV_MMA_PERSISTENT_CASE(64, 16)

@@ -29,7 +29,7 @@ struct DecodeParams {
 };
 
 // Consumer warps of the grouped-query (tensor-core) kernel; plus one producer warp.
-constexpr int MMA_CONSUMER_WARPS = 4;
+constexpr int MMA_CONSUMER_WARPS = 2;
 
 // Shared-memory bytes of one ring stage / the whole launch.
 size_t simt_stage_bytes(int head_dim, int block_size, int kvc);
@@ -47,11 +47,12 @@ cudaError_t launch_simt_decode(const DecodeParams& p, int hpc, int kvc, bool spl
 cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& k_map,
                               const CUtensorMap& v_map, bool split, cudaStream_t stream);
 
-// Persistent split-K tensor-core kernel: a few CTAs per SM take (b, kv head,
-// partition) work items from `ticket` (a workspace word it zeroes first).
+// Persistent tensor-core kernel: a few CTAs per SM take (b, kv head, partition)
+// work items from `ticket` (a workspace word it zeroes first).  Without a
+// split every item is a whole context.
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& k_map,
                                          const CUtensorMap& v_map, unsigned int* ticket,
-                                         cudaStream_t stream);
+                                         bool split, cudaStream_t stream);
 size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs);
 constexpr int PERSISTENT_MAX_SEQS = 1024;
 

@@ -6,9 +6,10 @@
 // inside a host runtime that owns the device allocator may have no way to ask
 // for memory at all; and a decode loop with a tight latency budget cannot
 // afford cudaMalloc/cudaFree, which may synchronize the whole device.  For
-// them this entry point takes the split-K scratch (the partial maxima, sums and
-// outputs merged by the second kernel) from one fixed array compiled into the
-// library instead of from a caller's buffer.
+// them this entry point takes its scratch -- the split-K partial maxima, sums
+// and outputs merged by the second kernel, and the work counter of the
+// grouped-query kernel -- from one fixed array compiled into the library
+// instead of from a caller's buffer.
 //
 // The array lives in device memory of every GPU that loads the library, for
 // the life of the process, and holds PAGEDKV_NOALLOC_SCRATCH_BYTES.  Calls
@@ -16,7 +17,8 @@
 // leaves its partial results behind: calls that may run on the GPU at the same
 // time (different streams, or different host threads) corrupt each other's
 // results, so serialize them.  Nothing in it needs to start at zero: every
-// partial result a call reads was written earlier in that same call.
+// partial result a call reads was written earlier in that same call, and the
+// work counter is cleared on the stream before each launch that uses it.
 #include "../../include/pagedkv.h"
 
 #include <cuda_runtime.h>
@@ -76,7 +78,7 @@ extern "C" int paged_attention_decode_noalloc(
                                                       block_size, max_context_len, partition_size);
   if (need > kScratchBytes)
     return report(PAGEDKV_EWORKSPACE,
-                  "this call needs %zu bytes of split-K scratch but the built-in scratch holds "
+                  "this call needs %zu bytes of scratch but the built-in scratch holds "
                   "%zu; use longer partitions or fewer sequences per call, or "
                   "paged_attention_decode with a workspace of your own",
                   need, kScratchBytes);

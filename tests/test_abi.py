@@ -95,6 +95,8 @@ def test_workspace_bytes(lib):
     # long GQA contexts split automatically into 512-token partitions
     assert pkv.paged_attention_workspace_bytes(128, 64, 8, 128, 16, 16384, 0) == \
         128 * 64 * 32 * 130 * 4 + 16
+    # grouped queries in a single pass still take their work from a ticket word
+    assert pkv.paged_attention_workspace_bytes(128, 64, 8, 128, 16, 2048, -1) == 16
     # beyond 1024 sequences the tensor-core split runs one CTA per item: no ticket
     assert pkv.paged_attention_workspace_bytes(1100, 16, 2, 64, 16, 1000, 512) == \
         1100 * 16 * 2 * 66 * 4

@@ -2,7 +2,7 @@
 
 Engines that reserve nearly all GPU memory for their block pool, plugins inside
 a runtime that owns the allocator, and latency-bound loops that cannot afford
-cudaMalloc cannot pass a workspace; this entry point takes its split-K scratch
+cudaMalloc cannot pass a workspace; this entry point takes its scratch
 from an array built into the library instead.  The test calls it through the C
 ABI, twice in a row on the same inputs, and checks each result against the
 regular paged_attention_decode with a caller-owned workspace, within the
@@ -45,6 +45,7 @@ CASES = [
     (_workload("mha_split", 8, 8, 64, 8, [5, 129, 700]), 32),          # CUDA-core kernel + merge
     (_workload("auto", 8, 8, 128, 16, [17, 2500]), 0),                 # library's choice (splits)
     (_workload("single", 4, 4, 128, 16, [40, 90]), -1),                # no scratch needed
+    (_workload("gqa_single", 16, 2, 128, 16, [40, 900]), -1),          # only the work counter
 ]
 
 

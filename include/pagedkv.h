@@ -69,6 +69,7 @@ extern "C" {
                                          max_context_len / the table (clamped) */
 #define PAGEDKV_DEVERR_SLOT 4u        /* a slot beyond the pool: that token was skipped */
 #define PAGEDKV_DEVERR_TIMEOUT 8u     /* a pipeline wait gave up after ~2 s; output invalid */
+#define PAGEDKV_DEVERR_INTERNAL 16u   /* a kernel found its launch set-up inconsistent and did nothing */
 
 /* Message of the calling thread's last failed call ("" if none). */
 PAGEDKV_API const char *pagedkv_last_error(void);

@@ -27,4 +27,5 @@ from ._native import (  # noqa: F401
     DEVERR_CONTEXT_LEN,
     DEVERR_SLOT,
     DEVERR_TIMEOUT,
+    DEVERR_INTERNAL,
 )

@@ -19,7 +19,7 @@ _lib = None
 _lock = threading.Lock()
 
 OK, EINVAL, EUNSUPPORTED, ECUDA, EWORKSPACE, ENOMEM, ENOENT, ERANGE = 0, -1, -2, -3, -4, -5, -6, -7
-DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT, DEVERR_INTERNAL = 1, 2, 4, 8, 16
 
 
 class PagedKVError(RuntimeError):

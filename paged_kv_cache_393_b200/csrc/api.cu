@@ -121,7 +121,7 @@ const Tuning& tuning() {
 
 struct Plan {
   bool mma = false;
-  bool persistent = false;   // tensor-core split-K with a ticket-fed persistent grid
+  bool persistent = false;   // tensor-core kernel on a ticket-fed persistent grid
   int hpc = 1, kvc = 1;      // CUDA-core kernel: query heads / kv heads per CTA
   bool split = false;
   int part_tokens = 0;

@@ -39,6 +39,9 @@
 //    streams chunks across item boundaries without draining the ring.  The
 //    items' query tiles travel through a small queue (bulk copies) with their
 //    descriptors, and each finished item is merged while the next streams in.
+//    (Merging the split-K partitions inside this kernel, by the CTA that
+//    stores a context's last partition, was measured slower than the separate
+//    merge kernel: those merges land at the end of the launch.)
 #include "common.cuh"
 #include "kernels.h"
 
@@ -490,7 +493,7 @@ __device__ __forceinline__ int4 item_of_ticket(int t, int num_kv_heads, int num_
   return make_int4(lo, kvh, u - pref_f[lo], part_tokens);
 }
 
-constexpr int TAIL_KEYS = 256;  // chunk-count keys of the partial-partition sort
+constexpr int TAIL_KEYS = 64;  // partial partitions of 63+ chunks share the top key  // chunk-count keys of the partial-partition sort
 
 template <int D, int BS>
 __global__ void __launch_bounds__((NW + 1) * 32)
@@ -499,9 +502,15 @@ __global__ void __launch_bounds__((NW + 1) * 32)
                                  const PersistentArgs pa) {
   using Geo = StageGeom<D>;
   constexpr uint32_t QTILE_BYTES = 8 * D * 2;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // The 128-byte TMA swizzle needs 1024-byte aligned stages; the dynamic
+  // shared memory is declared with that alignment (no slack is allocated), and
+  // a CTA that finds it otherwise reports it and does nothing.
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw;
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) flag_error(p.err, ERR_INTERNAL);
+    return;
+  }
   const int stages = p.stages;
   const int B = p.num_seqs;
   const uint32_t ring = smem_u32(smem);
@@ -808,7 +817,7 @@ size_t mma_smem_bytes(int head_dim, int block_size, int stages) {
 
 size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs) {
   const size_t merge = (size_t)NW * 8 * (2 + head_dim + 4) * sizeof(float);
-  return 1024 + (size_t)stages * mma_stage_bytes(head_dim, 16) + IQ * 8ull * head_dim * 2 + merge +
+  return (size_t)stages * mma_stage_bytes(head_dim, 16) + IQ * 8ull * head_dim * 2 + merge +
          IQ * sizeof(int4) + (3ull * num_seqs + 1 + TAIL_KEYS + 1 + 32) * sizeof(int) + 8 +
          (2ull * stages + 2 * IQ) * sizeof(uint64_t) + 16;
 }

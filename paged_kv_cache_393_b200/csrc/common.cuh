@@ -20,6 +20,7 @@ constexpr unsigned ERR_BLOCK_ID = 1u;
 constexpr unsigned ERR_CONTEXT_LEN = 2u;
 constexpr unsigned ERR_SLOT = 4u;
 constexpr unsigned ERR_TIMEOUT = 8u;
+constexpr unsigned ERR_INTERNAL = 16u;
 
 constexpr unsigned long long WAIT_TIMEOUT_NS = 2000000000ull;  // 2 s
 

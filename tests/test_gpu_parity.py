@@ -90,6 +90,8 @@ SMALL = [
     (_fixed("gqa8_d64_bs8_long", 16, 2, 64, 8, [1500, 33]), -1),
     (_fixed("mha128_bs64_long", 4, 4, 128, 64, [1000, 1777]), -1),
     (_fixed("mha64_bs32_long", 8, 8, 64, 32, [1300, 7]), -1),
+    # many small partitions into one merge
+    (_fixed("gqa8_d128_250_parts", 16, 2, 128, 16, [4000, 33]), 16),
     # more sequences than the persistent tensor-core grid takes: one CTA per item
     (_fixed("gqa8_1030_seqs_split", 16, 2, 64, 16, [1 + (7 * i) % 97 for i in range(1030)]), 32),
 ]

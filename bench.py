@@ -217,7 +217,7 @@ def run_ours(args):
     pkv.load_library()
     w = wl.get(args.workload)
     if w.lens == "cow":
-        raise SystemExit("the bench times fixed-length batches; the cow workload is a parity test")
+        return run_cow(args, w, dev, world, rank, local)
     gb = PagedBatch(w, dev)
     part = w.partition_size
     B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
@@ -347,6 +347,111 @@ def run_ours(args):
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_cow(args, w, dev, world, rank, local):
+    """The copy-on-write workload: 32 prompts of 1000 tokens forked into 8 samples,
+    then decode steps.  Step 0 copies the 224 shared partial tail blocks
+    (copy_blocks) before its scatter and attention; the steps are replayed in
+    order (every write is idempotent, so replays leave the cache unchanged)."""
+    import numpy as np
+    import torch
+
+    import paged_kv_cache_393_b200 as pkv
+    from paged_kv_cache_393_b200.batch import CowBatch
+    gb = CowBatch(w, dev)
+    B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
+    steps_host = [gb.prepare_step() for _ in range(w.decode_steps)]
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    steps = []
+    for h in steps_host:
+        steps.append(dict(q=up(h["q"]), k=up(h["k"]), v=up(h["v"]), slots=up(h["slots"]),
+                          tables=up(h["tables"]), lens=up(h["lens"]),
+                          pairs=up(h["pairs"]) if len(h["pairs"]) else None,
+                          kv_bytes=int(h["lens"].astype(np.int64).sum())
+                          * wl.kv_bytes_per_token(Hk, D)))
+    out = torch.empty((B, H, D), dtype=torch.float16, device=dev)
+    need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, 0)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    n_pairs = len(steps_host[0]["pairs"])
+    copy_bytes = 2 * n_pairs * 2 * Hk * w.block_size * D * 2   # K and V blocks read + written
+
+    def run_step(j, ev=None):
+        st = steps[j]
+        if st["pairs"] is not None:
+            if ev is not None:
+                ev[0].record(stream)
+            pkv.copy_blocks([gb.key_cache], [gb.value_cache], st["pairs"], stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+        pkv.reshape_and_cache(st["k"], st["v"], gb.key_cache, gb.value_cache, st["slots"],
+                              stream=stream)
+        pkv.paged_attention_decode(out, st["q"], gb.key_cache, gb.value_cache, st["tables"],
+                                   st["lens"], w.scale, gb.max_context_len, 0, ws, stream=stream)
+
+    for j in range(w.decode_steps):   # first pass: the steps in order
+        run_step(j)
+    for j in range(max(args.warmup, 3)):
+        run_step(j % w.decode_steps)
+    torch.cuda.synchronize(dev)
+    pkv.device_errors(clear=True)
+    K = args.steps
+    copy_ev = []
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    for j in range(20):
+        run_step(j % w.decode_steps)
+    barrier(world, local)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    kv_total = 0
+    launches = 0
+    for i in range(K):
+        j = i % w.decode_steps
+        ev = None
+        if steps[j]["pairs"] is not None:
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            copy_ev.append(ev)
+            launches += 1
+        run_step(j, ev)
+        launches += 2
+        kv_total += steps[j]["kv_bytes"]
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, local)
+    clocks = sampler.stop()
+    flags = pkv.device_errors(clear=True)
+    if flags:
+        raise SystemExit("device error flags %#x during the timed steps" % flags)
+    ms_max, kv_all = aggregate(t0.elapsed_time(t1), float(kv_total), world, dev)
+    ms_per_step = ms_max / K
+    copy_us = (sum(a.elapsed_time(b) for a, b in copy_ev) / len(copy_ev) * 1e3) if copy_ev else None
+    prefix_blocks = w.prompts * (w.prompt_len // w.block_size)
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        print(json.dumps({
+            "metric": METRIC, "value": round(kv_all / (ms_max / 1e3) / 1e9, 2), "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "accumulate": "f32", "data": "synthetic",
+            "config": {"workload": "cow: %d prompts x %d tokens forked into %d samples, %d decode "
+                                   "steps replayed in order; K/V bytes counted per sample "
+                                   "(shared prefix blocks counted once per reader)" % (
+                                       w.prompts, w.prompt_len, w.samples, w.decode_steps),
+                       "seed": w.seed, "l2": "no flush; shared prefix blocks (%d x 128 KiB x 2) "
+                                             "can hit in L2" % prefix_blocks,
+                       "parallelism": "replicas x%d" % world},
+            "tokens_per_s": round(B * world / (ms_per_step / 1e3), 1),
+            "copy_blocks": {"pairs": n_pairs, "bytes": copy_bytes, "avg_us": copy_us,
+                            "GB_per_s": round(copy_bytes / (copy_us / 1e6) / 1e9, 1) if copy_us else None,
+                            "peak": peak, "peak_kind": peak_kind},
+            "gpu_launches": launches, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+        }), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -2,14 +2,16 @@
 """Paged decode step benchmark (B200, sm_100a).
 
 One step = the whole decode hot path over one batch: copy_blocks for pending
-copy-on-write pairs (none in the llama7b batch), reshape_and_cache of every
-sequence's new token, and paged_attention_decode (plus the split-K merge when
-the workload splits).  The default workload is the Llama-2-7B-shaped batch:
+copy-on-write pairs (none in the llama7b batch), then the new token of every
+sequence written into its slot and the attention over the updated cache.  By
+default both happen in one paged_attention_decode_append launch (plus the
+split-K merge when the workload splits); --step separate runs reshape_and_cache
+and paged_attention_decode instead.  The default workload is the Llama-2-7B-shaped batch:
 256 sequences, 32 = 32 heads, head_dim 128, block_size 16, contexts uniform in
 [500, 1524], 32768-block pool.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload llama7b|gqa|bs_sweep_8|...]
+                    [--workload llama7b|gqa|bs_sweep_8|...] [--step fused|separate]
 
 Prints ONE JSON line (rank 0).  value = K+V bytes the attention reads per step,
 summed over ranks, divided by the device time of the K timed steps (max over
@@ -48,6 +50,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--step", choices=["fused", "separate"], default="fused",
+                    help="fused: one paged_attention_decode_append call writes the new tokens "
+                         "and attends; separate: reshape_and_cache then paged_attention_decode")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
@@ -225,18 +230,25 @@ def run_ours(args):
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
     splits = need > 0
-    launches_per_step = 2 + (1 if splits else 0)   # reshape, attention[, merge]
+    fused = args.step == "fused"
+    launches_per_step = (1 if fused else 2) + (1 if splits else 0)   # [reshape,] attention[, merge]
     G = H // Hk
     kernel_file = "attention_mma.cu" if (2 <= G <= 8 and w.block_size >= 8) else "attention_simt.cu"
 
     def attention():
-        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
-                                   gb.context_lens, w.scale, gb.max_context_len, part, ws,
-                                   stream=stream)
+        if fused:
+            pkv.paged_attention_decode_append(gb.out, gb.q, gb.k_new, gb.v_new, gb.key_cache,
+                                              gb.value_cache, gb.block_tables, gb.context_lens,
+                                              w.scale, gb.max_context_len, part, ws, stream=stream)
+        else:
+            pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache,
+                                       gb.block_tables, gb.context_lens, w.scale,
+                                       gb.max_context_len, part, ws, stream=stream)
 
     def cache_update():
-        pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots,
-                              stream=stream)
+        if not fused:
+            pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots,
+                                  stream=stream)
 
     for _ in range(max(args.warmup, 3)):
         cache_update()
@@ -281,6 +293,8 @@ def run_ours(args):
     # (K+V rows read, q read, out written, table entries and lengths read)
     nblk = (gb.lens_host + w.block_size - 1) // w.block_size
     attn_bytes = (kv_bytes + 2 * B * H * D * 2 + int(nblk.sum()) * 4 + B * 4)
+    if fused:
+        attn_bytes += 2 * B * Hk * D * 2 * 2    # new K/V rows read and written
     if splits:
         parts = (gb.lens_host + part - 1) // part
         attn_bytes += int(parts.sum()) * H * (D + 2) * 4 * 2    # partials written + read
@@ -292,7 +306,7 @@ def run_ours(args):
     e2e = None
     if args.e2e_steps > 0:
         sess = pkv.DecodeSession(gb.key_cache, gb.value_cache, B, H, gb.max_blocks,
-                                 gb.max_context_len, part)
+                                 gb.max_context_len, part, fused=fused)
         pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
         hq, hk, hv = pin(gb.q_host), pin(gb.k_new_host), pin(gb.v_new_host)
         hs, ht, hl = pin(gb.slots_host), pin(gb.tables_host), pin(gb.lens_host)
@@ -330,6 +344,7 @@ def run_ours(args):
                                 "%d..%d" % (gb.lens_host.min(), gb.lens_host.max()),
                                 w.num_blocks),
                 "seed": w.seed, "partition_size": part, "kv_bytes_per_step": kv_bytes,
+                "step": args.step,
                 "l2": "no flush: each step reads %.2f GB of K/V, far above the 126 MB L2"
                       % (kv_bytes / 1e9),
                 "parallelism": "replicas x%d" % world},
@@ -356,7 +371,9 @@ def run_cow(args, w, dev, world, rank, local):
     """The copy-on-write workload: 32 prompts of 1000 tokens forked into 8 samples,
     then decode steps.  Step 0 copies the 224 shared partial tail blocks
     (copy_blocks) before its scatter and attention; the steps are replayed in
-    order (every write is idempotent, so replays leave the cache unchanged)."""
+    order.  Replays do the same work; their cache contents may differ (a replayed
+    step-0 copy overwrites later rows of the copied blocks), which the timing
+    does not depend on."""
     import numpy as np
     import torch
 
@@ -388,10 +405,16 @@ def run_cow(args, w, dev, world, rank, local):
             pkv.copy_blocks([gb.key_cache], [gb.value_cache], st["pairs"], stream=stream)
             if ev is not None:
                 ev[1].record(stream)
-        pkv.reshape_and_cache(st["k"], st["v"], gb.key_cache, gb.value_cache, st["slots"],
-                              stream=stream)
-        pkv.paged_attention_decode(out, st["q"], gb.key_cache, gb.value_cache, st["tables"],
-                                   st["lens"], w.scale, gb.max_context_len, 0, ws, stream=stream)
+        if args.step == "fused":
+            pkv.paged_attention_decode_append(out, st["q"], st["k"], st["v"], gb.key_cache,
+                                              gb.value_cache, st["tables"], st["lens"], w.scale,
+                                              gb.max_context_len, 0, ws, stream=stream)
+        else:
+            pkv.reshape_and_cache(st["k"], st["v"], gb.key_cache, gb.value_cache, st["slots"],
+                                  stream=stream)
+            pkv.paged_attention_decode(out, st["q"], gb.key_cache, gb.value_cache, st["tables"],
+                                       st["lens"], w.scale, gb.max_context_len, 0, ws,
+                                       stream=stream)
 
     for j in range(w.decode_steps):   # first pass: the steps in order
         run_step(j)
@@ -419,7 +442,7 @@ def run_cow(args, w, dev, world, rank, local):
             copy_ev.append(ev)
             launches += 1
         run_step(j, ev)
-        launches += 2
+        launches += 1 if args.step == "fused" else 2
         kv_total += steps[j]["kv_bytes"]
     t1.record(stream)
     torch.cuda.synchronize(dev)
@@ -443,8 +466,9 @@ def run_cow(args, w, dev, world, rank, local):
                                    "steps replayed in order; K/V bytes counted per sample "
                                    "(shared prefix blocks counted once per reader)" % (
                                        w.prompts, w.prompt_len, w.samples, w.decode_steps),
-                       "seed": w.seed, "l2": "no flush; shared prefix blocks (%d x 128 KiB x 2) "
-                                             "can hit in L2" % prefix_blocks,
+                       "seed": w.seed, "step": args.step,
+                       "l2": "no flush; shared prefix blocks (%d x 128 KiB x 2) "
+                             "can hit in L2" % prefix_blocks,
                        "parallelism": "replicas x%d" % world},
             "tokens_per_s": round(B * world / (ms_per_step / 1e3), 1),
             "copy_blocks": {"pairs": n_pairs, "bytes": copy_bytes, "avg_us": copy_us,

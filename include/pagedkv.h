@@ -78,6 +78,14 @@ PAGEDKV_API const char *pagedkv_last_error(void);
  * Synchronizes the device first.  Returns PAGEDKV_OK or PAGEDKV_ECUDA. */
 PAGEDKV_API int pagedkv_device_errors(unsigned int *flags, int clear);
 
+/* Self-test of the failure path every kernel pipeline uses.  Enqueues a kernel
+ * that waits on a barrier nothing completes, with the same bounded wait as the
+ * attention kernels, for timeout_us microseconds (1 .. 1e6); the wait then
+ * gives up, sets PAGEDKV_DEVERR_TIMEOUT in the error word and the kernel
+ * returns normally.  It never faults and never hangs, and the device stays
+ * usable.  Read the result with pagedkv_device_errors.  Errors: EINVAL, ECUDA. */
+PAGEDKV_API int pagedkv_selftest_wait_timeout(unsigned int timeout_us, void *stream);
+
 /* ---- paged decode attention ------------------------------------------------
  *
  * For every sequence b < num_seqs and query head h < num_heads, with
@@ -133,6 +141,40 @@ PAGEDKV_API int paged_attention_decode(void *out, const void *q,
 PAGEDKV_API size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
                                        int head_dim, int block_size, int max_context_len,
                                        int partition_size);
+
+/* ---- fused append + decode ----------------------------------------------------------
+ *
+ * One decode step in one call: each sequence's new K/V row is written into the
+ * cache and the attention then reads it, as reshape_and_cache followed by
+ * paged_attention_decode would (the new token scattered into its block, then
+ * the block-table gather: lpnh.cn/news/1824136 §3.1 and §3.2 steps 3-4).
+ *
+ * The new token is position L_b - 1 of sequence b, so its slot is implied by
+ * the table: row (L_b - 1) % block_size of block
+ * block_tables[b][(L_b - 1) / block_size]; no slot mapping is passed.  That
+ * block must belong to sequence b alone (a shared block is copied first:
+ * copy_blocks), as it must for reshape_and_cache.
+ *
+ *   k_new, v_new   device fp16 [num_seqs][num_kv_heads][head_dim], 16-byte aligned
+ *   key_cache,
+ *   value_cache    as for paged_attention_decode; written at the new slots only
+ *   the rest       as for paged_attention_decode (same workspace size)
+ *
+ * Results: out as paged_attention_decode computes it on the updated cache, and
+ * the cache bytes as reshape_and_cache writes them.  A sequence whose length is
+ * rejected on the device (L_b <= 0 or > max_context_len) or whose block id is
+ * out of range gets no write; the error word says so.
+ * num_seqs == 0 is a no-op.  Errors: EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+PAGEDKV_API int paged_attention_decode_append(void *out, const void *q,
+                           const void *k_new, const void *v_new,
+                           void *key_cache, void *value_cache,
+                           const int32_t *block_tables, const int32_t *context_lens,
+                           float scale, int block_size, int num_kv_heads,
+                           int num_seqs, int num_heads, int head_dim,
+                           int max_blocks_per_seq, int num_blocks, int max_context_len,
+                           int partition_size, void *workspace, size_t workspace_bytes,
+                           void *stream);
 
 /* ---- allocation-free decode ------------------------------------------------------
  *
@@ -294,6 +336,24 @@ PAGEDKV_API int bm_num_free(pagedkv_block_manager *bm);
 /* Copies the free list (bottom to top) to out and returns its length; with
  * out == NULL only returns the length.  ERANGE if cap is too small. */
 PAGEDKV_API int bm_free_list(pagedkv_block_manager *bm, int32_t *out, int cap);
+
+/* Occupancy of the pool (the utilisation and fragmentation the pages discuss:
+ * tail waste per block size, 5688vip ch. 4 "块大小选择"; lpnh.cn/news/2758356
+ * §5.1-§5.3).  A physical block's filled slots are the most tokens any
+ * sequence referencing it keeps in it. */
+typedef struct pagedkv_bm_stats {
+  int64_t num_blocks;      /* pool size */
+  int64_t free_blocks;     /* on the free list */
+  int64_t used_blocks;     /* refcount > 0 */
+  int64_t num_seqs;        /* live sequences */
+  int64_t logical_tokens;  /* sum of sequence lengths (shared tokens counted per sequence) */
+  int64_t filled_slots;    /* physical slots holding a token */
+  int64_t allocated_slots; /* used_blocks * block_size */
+  int64_t table_entries;   /* sum of table lengths (= sum of refcounts) */
+} pagedkv_bm_stats;
+
+/* Fills *out.  OK or EINVAL. */
+PAGEDKV_API int bm_stats(pagedkv_block_manager *bm, pagedkv_bm_stats *out);
 
 /* Message of the calling thread's last failed bm_* call ("" if none). */
 PAGEDKV_API const char *bm_last_error(void);

@@ -280,6 +280,22 @@ class BlockManagerModel:
     def num_free(self) -> int:
         return len(self.free)
 
+    def stats(self):
+        """Pool occupancy.  A physical block's filled slots are the most tokens any
+        sequence referencing it keeps in it; allocated slots are whole used blocks."""
+        bs = self.block_size
+        fill = {}
+        for seq, table in self.tables.items():
+            L = self.lens[seq]
+            for j, blk in enumerate(table):
+                fill[blk] = max(fill.get(blk, 0), min(bs, L - j * bs))
+        used = sum(1 for r in self.refcount if r > 0)
+        return {"num_blocks": self.num_blocks, "free_blocks": len(self.free),
+                "used_blocks": used, "num_seqs": len(self.tables),
+                "logical_tokens": sum(self.lens.values()), "filled_slots": sum(fill.values()),
+                "allocated_slots": used * bs,
+                "table_entries": sum(len(t) for t in self.tables.values())}
+
     def slots_of(self, seq: int):
         """Flat slots of every token of the sequence, in logical order."""
         bs = self.block_size

@@ -7,7 +7,8 @@ device memory and streams.  There is no CPU fallback: if the library is
 missing, every call raises.
 
 Functions mirror the C names:
-    paged_attention_decode, paged_attention_workspace_bytes, reshape_and_cache,
+    paged_attention_decode, paged_attention_decode_append (fused: new K/V row
+    written, then attended), paged_attention_workspace_bytes, reshape_and_cache,
     copy_blocks, device_errors, BlockManager (bm_*), decode_step (host buffers
     in, host result out).
 """
@@ -21,8 +22,10 @@ from ._native import (  # noqa: F401
     library_path,
     load_library,
     paged_attention_decode,
+    paged_attention_decode_append,
     paged_attention_workspace_bytes,
     reshape_and_cache,
+    selftest_wait_timeout,
     DEVERR_BLOCK_ID,
     DEVERR_CONTEXT_LEN,
     DEVERR_SLOT,

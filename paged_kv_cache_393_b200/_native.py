@@ -48,7 +48,10 @@ def load_library():
         sig = {
             "pagedkv_last_error": ([], ctypes.c_char_p),
             "pagedkv_device_errors": ([ctypes.POINTER(ctypes.c_uint), I], I),
+            "pagedkv_selftest_wait_timeout": ([ctypes.c_uint, P], I),
             "paged_attention_decode": ([P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
+            "paged_attention_decode_append": (
+                [P, P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
             "paged_attention_workspace_bytes": ([I, I, I, I, I, I, I], Z),
             "reshape_and_cache": ([P, P, P, P, P, I, I, I, I, I, P], I),
             "copy_blocks": ([P, P, P, I, I, Z, I, P], I),
@@ -67,6 +70,7 @@ def load_library():
             "bm_num_free": ([P], I),
             "bm_free_list": ([P, P, I], I),
             "bm_last_error": ([], ctypes.c_char_p),
+            "bm_stats": ([P, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -115,6 +119,23 @@ def paged_attention_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
 def paged_attention_decode(out, q, key_cache, value_cache, block_tables, context_lens, scale,
                            max_context_len, partition_size=0, workspace=None, stream=None):
     """out[B][H][D] = paged decode attention of q over the pools; see include/pagedkv.h."""
+    return _decode("paged_attention_decode", out, q, None, None, key_cache, value_cache,
+                   block_tables, context_lens, scale, max_context_len, partition_size, workspace,
+                   stream)
+
+
+def paged_attention_decode_append(out, q, k_new, v_new, key_cache, value_cache, block_tables,
+                                  context_lens, scale, max_context_len, partition_size=0,
+                                  workspace=None, stream=None):
+    """One fused step: k_new/v_new ([B][Hk][D]) are written at position L_b - 1 through the
+    block tables, then out = paged decode attention over the updated pools."""
+    return _decode("paged_attention_decode_append", out, q, k_new, v_new, key_cache, value_cache,
+                   block_tables, context_lens, scale, max_context_len, partition_size, workspace,
+                   stream)
+
+
+def _decode(name, out, q, k_new, v_new, key_cache, value_cache, block_tables, context_lens, scale,
+            max_context_len, partition_size, workspace, stream):
     lib = load_library()
     B, H, D = q.shape
     N, Hk, bs, D2 = key_cache.shape
@@ -123,11 +144,15 @@ def paged_attention_decode(out, q, key_cache, value_cache, block_tables, context
             tuple(q.shape), tuple(key_cache.shape), tuple(value_cache.shape), tuple(out.shape)))
     if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
         raise ValueError("block_tables must be [B][max_blocks] and context_lens [B]")
-    ptrs = [_cuda(out, "out", torch.float16, 3), _cuda(q, "q", torch.float16, 3),
-            _cuda(key_cache, "key_cache", torch.float16, 4),
-            _cuda(value_cache, "value_cache", torch.float16, 4),
-            _cuda(block_tables, "block_tables", torch.int32, 2),
-            _cuda(context_lens, "context_lens", torch.int32, 1)]
+    ptrs = [_cuda(out, "out", torch.float16, 3), _cuda(q, "q", torch.float16, 3)]
+    if k_new is not None:
+        if tuple(k_new.shape) != (B, Hk, D) or tuple(v_new.shape) != (B, Hk, D):
+            raise ValueError("k_new and v_new must be [B][Hk][D]")
+        ptrs += [_cuda(k_new, "k_new", torch.float16, 3), _cuda(v_new, "v_new", torch.float16, 3)]
+    ptrs += [_cuda(key_cache, "key_cache", torch.float16, 4),
+             _cuda(value_cache, "value_cache", torch.float16, 4),
+             _cuda(block_tables, "block_tables", torch.int32, 2),
+             _cuda(context_lens, "context_lens", torch.int32, 1)]
     need = paged_attention_workspace_bytes(B, H, Hk, D, bs, max_context_len, partition_size)
     ws_ptr, ws_bytes = None, 0
     if need:
@@ -135,10 +160,10 @@ def paged_attention_decode(out, q, key_cache, value_cache, block_tables, context
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         _cuda(workspace, "workspace", workspace.dtype)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
-    st = lib.paged_attention_decode(*ptrs, float(scale), bs, Hk, B, H, D, block_tables.shape[1], N,
-                                    int(max_context_len), int(partition_size), ws_ptr, ws_bytes,
-                                    _stream(stream, q.device))
-    _check(st, "paged_attention_decode")
+    st = getattr(lib, name)(*ptrs, float(scale), bs, Hk, B, H, D, block_tables.shape[1], N,
+                            int(max_context_len), int(partition_size), ws_ptr, ws_bytes,
+                            _stream(stream, q.device))
+    _check(st, name)
     return out
 
 
@@ -184,6 +209,14 @@ def copy_blocks(key_caches, value_caches, pairs, stream=None):
     _check(st, "copy_blocks")
 
 
+def selftest_wait_timeout(timeout_us: int, stream=None):
+    """Enqueues the bounded-wait self-test (see include/pagedkv.h)."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib.pagedkv_selftest_wait_timeout(int(timeout_us), _stream(stream, dev)),
+           "pagedkv_selftest_wait_timeout")
+
+
 def device_errors(clear: bool = True) -> int:
     """Error bits the kernels raised on the current device (synchronizes the device)."""
     flags = ctypes.c_uint(0)
@@ -197,17 +230,20 @@ class DecodeSession:
 
     Holds device staging buffers for one batch shape.  ``step`` copies the
     step's inputs from (pinned) host memory, runs copy_blocks for pending
-    copy-on-write pairs, reshape_and_cache for the new tokens and
-    paged_attention_decode, and copies the output back into a host tensor.
+    copy-on-write pairs, then either reshape_and_cache for the new tokens and
+    paged_attention_decode, or (fused=True) paged_attention_decode_append, which
+    writes the new tokens at position L-1 through the tables itself and needs no
+    slots; finally it copies the output back into a host tensor.
     """
 
     def __init__(self, key_cache, value_cache, num_seqs, num_heads, max_blocks, max_context_len,
-                 partition_size=0, max_pairs=0):
+                 partition_size=0, max_pairs=0, fused=False):
         dev = key_cache.device
         N, Hk, bs, D = key_cache.shape
         self.key_cache, self.value_cache = key_cache, value_cache
         self.max_context_len = int(max_context_len)
         self.partition_size = partition_size
+        self.fused = bool(fused)
         self.q = torch.empty((num_seqs, num_heads, D), dtype=torch.float16, device=dev)
         self.k = torch.empty((num_seqs, Hk, D), dtype=torch.float16, device=dev)
         self.v = torch.empty_like(self.k)
@@ -221,29 +257,39 @@ class DecodeSession:
         self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 
     def h2d_bytes(self, num_pairs=0) -> int:
-        ts = (self.q, self.k, self.v, self.slots, self.tables, self.lens)
+        ts = (self.q, self.k, self.v, self.tables, self.lens) + (() if self.fused else (self.slots,))
         return sum(t.numel() * t.element_size() for t in ts) + num_pairs * 16
 
     def d2h_bytes(self) -> int:
         return self.out.numel() * self.out.element_size()
 
     def step(self, q, k, v, slots, tables, lens, out_host, pairs=None, stream=None):
+        """slots may be None when the session is fused."""
         s = torch.cuda.current_stream(self.q.device) if stream is None else stream
+        scale = 1.0 / (self.q.shape[2] ** 0.5)
         with torch.cuda.stream(s):
             self.q.copy_(q, non_blocking=True)
             self.k.copy_(k, non_blocking=True)
             self.v.copy_(v, non_blocking=True)
-            self.slots.copy_(slots, non_blocking=True)
+            if not self.fused:
+                self.slots.copy_(slots, non_blocking=True)
             self.tables.copy_(tables, non_blocking=True)
             self.lens.copy_(lens, non_blocking=True)
             if pairs is not None and len(pairs):
                 n = pairs.shape[0]
                 self.pairs[:n].copy_(pairs, non_blocking=True)
                 copy_blocks([self.key_cache], [self.value_cache], self.pairs[:n], stream=s)
-            reshape_and_cache(self.k, self.v, self.key_cache, self.value_cache, self.slots, stream=s)
-            paged_attention_decode(self.out, self.q, self.key_cache, self.value_cache, self.tables,
-                                   self.lens, 1.0 / (self.q.shape[2] ** 0.5), self.max_context_len,
-                                   self.partition_size, self.workspace, stream=s)
+            if self.fused:
+                paged_attention_decode_append(self.out, self.q, self.k, self.v, self.key_cache,
+                                              self.value_cache, self.tables, self.lens, scale,
+                                              self.max_context_len, self.partition_size,
+                                              self.workspace, stream=s)
+            else:
+                reshape_and_cache(self.k, self.v, self.key_cache, self.value_cache, self.slots,
+                                  stream=s)
+                paged_attention_decode(self.out, self.q, self.key_cache, self.value_cache,
+                                       self.tables, self.lens, scale, self.max_context_len,
+                                       self.partition_size, self.workspace, stream=s)
             out_host.copy_(self.out, non_blocking=True)
         return out_host
 
@@ -343,6 +389,14 @@ class BlockManager:
 
     def num_free(self) -> int:
         return self._chk(self._lib.bm_num_free(self._h), "bm_num_free")
+
+    def stats(self) -> dict:
+        """Pool occupancy: see pagedkv_bm_stats in include/pagedkv.h."""
+        out = (ctypes.c_int64 * 8)()
+        self._chk(self._lib.bm_stats(self._h, out), "bm_stats")
+        keys = ("num_blocks", "free_blocks", "used_blocks", "num_seqs", "logical_tokens",
+                "filled_slots", "allocated_slots", "table_entries")
+        return dict(zip(keys, [int(x) for x in out]))
 
     def free_list(self):
         n = self._chk(self._lib.bm_free_list(self._h, None, 0), "bm_free_list")

@@ -1,6 +1,7 @@
 // C ABI of libpagedkv.so: argument checks, launch planning and dispatch.
 // Declarations and the contract of every entry point: include/pagedkv.h.
 #include "../../include/pagedkv.h"
+#include "common.cuh"
 #include "kernels.h"
 
 #include <cuda.h>
@@ -239,6 +240,19 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
   return PAGEDKV_OK;
 }
 
+// The bounded wait every pipeline uses, on an mbarrier that nothing completes:
+// after timeout_ns the wait gives up, the error word gets ERR_TIMEOUT, and the
+// kernel completes the phase itself and returns.
+__global__ void selftest_wait_kernel(unsigned long long timeout_ns, unsigned* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t a = smem_u32(&bar);
+  mbar_init(a, 1);
+  fence_barrier_init();
+  if (!mbar_wait(a, 0, timeout_ns)) flag_error(err, ERR_TIMEOUT);
+  mbar_arrive(a);  // leave the barrier's phase complete
+}
+
 }  // namespace
 
 // Records a failure for pagedkv_last_error() from another translation unit.
@@ -266,6 +280,19 @@ int pagedkv_device_errors(unsigned int* flags, int clear) {
   return PAGEDKV_OK;
 }
 
+int pagedkv_selftest_wait_timeout(unsigned int timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 1000000u)
+    return fail(PAGEDKV_EINVAL, "timeout_us must be in [1, 1000000]");
+  unsigned* err = nullptr;
+  int st = error_word(&err);
+  if (st != PAGEDKV_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)timeout_us * 1000ull, err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return PAGEDKV_OK;
+}
+
 size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                        int block_size, int max_context_len, int partition_size) {
   Plan plan;
@@ -275,12 +302,17 @@ size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_h
   return plan.ws_bytes;
 }
 
-int paged_attention_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
-                           const int32_t* block_tables, const int32_t* context_lens, float scale,
-                           int block_size, int num_kv_heads, int num_seqs, int num_heads,
-                           int head_dim, int max_blocks_per_seq, int num_blocks,
-                           int max_context_len, int partition_size, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace pkv {
+namespace {
+
+// Both decode entry points; k_new / v_new are NULL for the plain one.
+int decode(void* out, const void* q, const void* k_new, const void* v_new, const void* key_cache,
+           const void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+           float scale, int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+           int max_blocks_per_seq, int num_blocks, int max_context_len, int partition_size,
+           void* workspace, size_t workspace_bytes, void* stream) {
   if (num_seqs == 0) return PAGEDKV_OK;
   if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
     return fail(PAGEDKV_EINVAL, "a required pointer is NULL");
@@ -333,6 +365,8 @@ int paged_attention_decode(void* out, const void* q, const void* key_cache, cons
   p.part_tokens = plan.part_tokens;
   p.num_parts = plan.num_parts;
   p.stages = plan.stages;
+  p.k_new = static_cast<const __half*>(k_new);
+  p.v_new = static_cast<const __half*>(v_new);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   cudaError_t e;
@@ -362,6 +396,38 @@ int paged_attention_decode(void* out, const void* q, const void* key_cache, cons
     if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
   }
   return PAGEDKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+int paged_attention_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, float scale,
+                           int block_size, int num_kv_heads, int num_seqs, int num_heads,
+                           int head_dim, int max_blocks_per_seq, int num_blocks,
+                           int max_context_len, int partition_size, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return decode(out, q, nullptr, nullptr, key_cache, value_cache, block_tables, context_lens,
+                scale, block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq,
+                num_blocks, max_context_len, partition_size, workspace, workspace_bytes, stream);
+}
+
+int paged_attention_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
+                                  void* key_cache, void* value_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, float scale, int block_size,
+                                  int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                                  int max_blocks_per_seq, int num_blocks, int max_context_len,
+                                  int partition_size, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (num_seqs == 0) return PAGEDKV_OK;
+  if (!k_new || !v_new) return fail(PAGEDKV_EINVAL, "k_new and v_new are required");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    return fail(PAGEDKV_EINVAL, "k_new and v_new must be 16-byte aligned");
+  return decode(out, q, k_new, v_new, key_cache, value_cache, block_tables, context_lens, scale,
+                block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq,
+                num_blocks, max_context_len, partition_size, workspace, workspace_bytes, stream);
 }
 
 int reshape_and_cache(const void* k, const void* v, void* key_cache, void* value_cache,

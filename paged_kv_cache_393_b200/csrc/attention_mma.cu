@@ -127,14 +127,35 @@ __device__ __forceinline__ void issue_stage(uint32_t kdst, uint32_t full, const 
 
 // Streams the nchunks chunks of one item (its table row starts at `row`) into
 // the ring, the item's first chunk having global chunk index gc0.  Run by the
-// whole producer warp; lane 0 issues.  Returns false (warp-uniform) when it
+// whole producer warp; lane 0 issues.  With a fused append (new_tok >= 0: the
+// item ends its context, and its token new_tok is the new one) the warp writes
+// the new K/V rows of sequence b, kv head kvh, into their slot before it issues
+// the chunk that reads them.  Returns false (warp-uniform) when it
 // gave up; *issued_end is one past the last global chunk issued.
 template <int D, int BS>
-__device__ bool produce_item(const int32_t* row, int nblk, int nchunks, int gc0, int kvh,
-                             const DecodeParams& p, int* s_ids, uint64_t* bars, int stages,
-                             uint32_t ring, const CUtensorMap* km, const CUtensorMap* vm,
-                             uint64_t policy, volatile int* abort_flag, int lane, int* issued_end) {
+__device__ bool produce_item(const int32_t* row, int nblk, int nchunks, int gc0, int kvh, int b,
+                             int new_tok, const DecodeParams& p, int* s_ids, uint64_t* bars,
+                             int stages, uint32_t ring, const CUtensorMap* km,
+                             const CUtensorMap* vm, uint64_t policy, volatile int* abort_flag,
+                             int lane, int* issued_end) {
   using Geo = StageGeom<D>;
+  NewRows<D, 1> fresh;
+  if (new_tok >= 0) fresh.load(p.k_new, p.v_new, b, p.num_kv_heads, kvh, lane);
+  // issues chunk c (lane 0 only); false when the wait for a free stage gave up
+  auto issue = [&](int c, int w0) -> bool {
+    const int gc = gc0 + c;
+    const int st = gc % stages;
+    const int round = gc / stages;
+    if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
+      *abort_flag = 1;
+      flag_error(p.err, ERR_TIMEOUT);
+      return false;
+    }
+    issue_stage<D, BS>(ring + (uint32_t)st * 2 * Geo::TILE_BYTES, smem_u32(&bars[st]), s_ids, w0,
+                       c, nblk, kvh, p.num_kv_heads, km, vm, policy);
+    *issued_end = gc + 1;
+    return true;
+  };
   bool ok = true;
   for (int w0 = 0; w0 < nblk; w0 += 32) {
     if (w0 + lane < nblk) {
@@ -146,28 +167,31 @@ __device__ bool produce_item(const int32_t* row, int nblk, int nchunks, int gc0,
       s_ids[lane] = id;
     }
     __syncwarp();
-    if (lane == 0 && ok) {
-      const int c_end = min(nchunks, (w0 + 32) * BS / CHUNK);
-      for (int c = w0 * BS / CHUNK; c < c_end; ++c) {
-        if (*abort_flag) {
-          ok = false;
-          break;
+    const int c_begin = w0 * BS / CHUNK;
+    const int c_end = min(nchunks, (w0 + 32) * BS / CHUNK);
+    // With an append, the rows are stored once the item's first chunks (up to a
+    // ring's worth) are issued, and always before its last chunk.
+    const bool append_here = new_tok >= 0 && w0 == 0;
+    const int c_split = append_here ? min(c_end, min(stages, nchunks - 1)) : c_end;
+    auto issue_range = [&](int c0, int c1) {
+      if (lane == 0 && ok) {
+        for (int c = c0; c < c1; ++c) {
+          if (*abort_flag || !issue(c, w0)) {
+            ok = false;
+            break;
+          }
         }
-        const int gc = gc0 + c;
-        const int st = gc % stages;
-        const int round = gc / stages;
-        if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
-          *abort_flag = 1;
-          flag_error(p.err, ERR_TIMEOUT);
-          ok = false;
-          break;
-        }
-        issue_stage<D, BS>(ring + (uint32_t)st * 2 * Geo::TILE_BYTES, smem_u32(&bars[st]), s_ids,
-                           w0, c, nblk, kvh, p.num_kv_heads, km, vm, policy);
-        *issued_end = gc + 1;
       }
+      ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+    };
+    issue_range(c_begin, c_split);
+    if (append_here && ok) {
+      const int id = row[new_tok / BS];  // re-read: a bad id was replaced by 0 for reading only
+      if (id >= 0 && id < p.num_blocks)
+        fresh.store(const_cast<__half*>(p.k_cache), const_cast<__half*>(p.v_cache),
+                    p.num_kv_heads, BS, kvh, id, new_tok % BS, lane);
     }
-    ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+    issue_range(c_split, c_end);
     __syncwarp();  // s_ids is rewritten for the next window
   }
   return ok;
@@ -412,9 +436,11 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       prefetch_tensor_map(&v_map);
     }
     const int32_t* row = p.block_tables + (size_t)b * p.max_blocks + tok0 / BS;
+    const int new_tok =
+        (p.k_new && tok0 + ntok == L && p.context_lens[b] == L) ? ntok - 1 : -1;
     int issued_end = 0;
-    produce_item<D, BS>(row, nblk, nchunks, 0, kvh, p, s_ids, bars, stages, ring, &k_map, &v_map,
-                        l2_evict_first_policy(), abort_flag, lane, &issued_end);
+    produce_item<D, BS>(row, nblk, nchunks, 0, kvh, b, new_tok, p, s_ids, bars, stages, ring,
+                        &k_map, &v_map, l2_evict_first_policy(), abort_flag, lane, &issued_end);
     if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued_end);
     return;
   }
@@ -668,8 +694,11 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       const int nchunks = (d.w + CHUNK - 1) / CHUNK;
       const int nblk = (d.w + BS - 1) / BS;
       const int32_t* row = p.block_tables + (size_t)d.x * p.max_blocks + d.z * pt / BS;
-      if (!produce_item<D, BS>(row, nblk, nchunks, gc, d.y, p, s_ids, bars, stages, ring, &k_map,
-                               &v_map, policy, abort_flag, lane, &issued_end))
+      const int L = s_lens[d.x];
+      const int new_tok =
+          (p.k_new && d.z * pt + d.w == L && p.context_lens[d.x] == L) ? d.w - 1 : -1;
+      if (!produce_item<D, BS>(row, nblk, nchunks, gc, d.y, d.x, new_tok, p, s_ids, bars, stages,
+                               ring, &k_map, &v_map, policy, abort_flag, lane, &issued_end))
         break;
       gc += nchunks;
       have = next_item(&d);

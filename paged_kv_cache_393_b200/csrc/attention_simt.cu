@@ -128,6 +128,57 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
     const uint64_t policy = l2_evict_first_policy();
     const uint32_t ring = smem_u32(tiles);
     int issued = 0;
+    // Fused append: the partition that ends the context writes the new rows of
+    // its kv heads (token L-1) before it issues the stage that reads them.
+    const int new_tok =
+        (p.k_new && tok0 + ntok == L && p.context_lens[b] == L) ? ntok - 1 : -1;
+    NewRows<D, KVC> fresh;
+    if (new_tok >= 0) fresh.load(p.k_new, p.v_new, b, p.num_kv_heads, kv0, lane);
+
+    // Issues stage c (lane 0 only); false when the wait for a free slot gave up.
+    auto issue = [&](int c, int w0) -> bool {
+      const int st = c % stages;
+      const int round = c / stages;
+      if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
+        *abort_flag = 1;
+        flag_error(p.err, ERR_TIMEOUT);
+        return false;
+      }
+      const uint32_t full = smem_u32(&bars[st]);
+      const uint32_t kdst = ring + (uint32_t)st * 2 * TILE_BYTES;
+      const uint32_t vdst = kdst + TILE_BYTES;
+      if (BS >= CHUNK) {
+        const int tok = c * CHUNK;
+        const int phys = s_ids[tok / BS - w0];
+        const int r0 = tok % BS;
+        mbar_arrive_expect_tx(full, 2 * TILE_BYTES);
+        if (BS == CHUNK) {  // the KVC heads of one block are one contiguous tile
+          const size_t off = ((size_t)phys * p.num_kv_heads + kv0) * (size_t)(BS * D);
+          bulk_load(kdst, p.k_cache + off, TILE_BYTES, full, policy);
+          bulk_load(vdst, p.v_cache + off, TILE_BYTES, full, policy);
+        } else {
+#pragma unroll
+          for (int h = 0; h < KVC; ++h) {
+            const size_t off = (((size_t)phys * p.num_kv_heads + kv0 + h) * BS + r0) * (size_t)D;
+            bulk_load(kdst + h * CHUNK * D * 2, p.k_cache + off, CHUNK * D * 2, full, policy);
+            bulk_load(vdst + h * CHUNK * D * 2, p.v_cache + off, CHUNK * D * 2, full, policy);
+          }
+        }
+      } else {
+        const int first = c * NB;                // first block of the stage
+        const int nb = min(NB, nblk - first);
+        mbar_arrive_expect_tx(full, 2u * nb * SUB_BYTES);
+        for (int k = 0; k < nb; ++k) {
+          const size_t off =
+              ((size_t)s_ids[first + k - w0] * p.num_kv_heads + kv0) * (size_t)(BS * D);
+          bulk_load(kdst + k * SUB_BYTES, p.k_cache + off, SUB_BYTES, full, policy);
+          bulk_load(vdst + k * SUB_BYTES, p.v_cache + off, SUB_BYTES, full, policy);
+        }
+      }
+      issued = c + 1;
+      return true;
+    };
+
     // table entries are read 32 at a time by the lanes and staged in shared memory
     for (int w0 = 0; w0 < nblk; w0 += 32) {
       if (w0 + lane < nblk) {
@@ -139,50 +190,25 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
         s_ids[lane] = id;
       }
       __syncwarp();
+      const int c_begin = w0 * BS / CHUNK;
+      const int c_end = min(nchunks, (w0 + 32) * BS / CHUNK);
+      // With an append, the rows are stored once the first ring fill is issued
+      // (those copies are in flight meanwhile) and always before the last stage.
+      const bool append_here = new_tok >= 0 && w0 == 0;
+      const int c_split = append_here ? min(c_end, min(stages, nchunks - 1)) : c_end;
       if (lane == 0) {
-        const int c_end = min(nchunks, (w0 + 32) * BS / CHUNK);
-        for (int c = w0 * BS / CHUNK; c < c_end && !*abort_flag; ++c) {
-          const int st = c % stages;
-          const int round = c / stages;
-          if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
-            *abort_flag = 1;
-            flag_error(p.err, ERR_TIMEOUT);
-            break;
-          }
-          const uint32_t full = smem_u32(&bars[st]);
-          const uint32_t kdst = ring + (uint32_t)st * 2 * TILE_BYTES;
-          const uint32_t vdst = kdst + TILE_BYTES;
-          if (BS >= CHUNK) {
-            const int tok = c * CHUNK;
-            const int phys = s_ids[tok / BS - w0];
-            const int r0 = tok % BS;
-            mbar_arrive_expect_tx(full, 2 * TILE_BYTES);
-            if (BS == CHUNK) {  // the KVC heads of one block are one contiguous tile
-              const size_t off = ((size_t)phys * p.num_kv_heads + kv0) * (size_t)(BS * D);
-              bulk_load(kdst, p.k_cache + off, TILE_BYTES, full, policy);
-              bulk_load(vdst, p.v_cache + off, TILE_BYTES, full, policy);
-            } else {
-#pragma unroll
-              for (int h = 0; h < KVC; ++h) {
-                const size_t off =
-                    (((size_t)phys * p.num_kv_heads + kv0 + h) * BS + r0) * (size_t)D;
-                bulk_load(kdst + h * CHUNK * D * 2, p.k_cache + off, CHUNK * D * 2, full, policy);
-                bulk_load(vdst + h * CHUNK * D * 2, p.v_cache + off, CHUNK * D * 2, full, policy);
-              }
-            }
-          } else {
-            const int first = c * NB;                // first block of the stage
-            const int nb = min(NB, nblk - first);
-            mbar_arrive_expect_tx(full, 2u * nb * SUB_BYTES);
-            for (int k = 0; k < nb; ++k) {
-              const size_t off =
-                  ((size_t)s_ids[first + k - w0] * p.num_kv_heads + kv0) * (size_t)(BS * D);
-              bulk_load(kdst + k * SUB_BYTES, p.k_cache + off, SUB_BYTES, full, policy);
-              bulk_load(vdst + k * SUB_BYTES, p.v_cache + off, SUB_BYTES, full, policy);
-            }
-          }
-          issued = c + 1;
-        }
+        for (int c = c_begin; c < c_split && !*abort_flag; ++c)
+          if (!issue(c, w0)) break;
+      }
+      if (append_here && !__shfl_sync(0xffffffffu, *abort_flag, 0)) {
+        const int id = row[new_tok / BS];  // re-read: a bad id was replaced by 0 for reading only
+        if (id >= 0 && id < p.num_blocks)
+          fresh.store(const_cast<__half*>(p.k_cache), const_cast<__half*>(p.v_cache),
+                      p.num_kv_heads, BS, kv0, id, new_tok % BS, lane);
+      }
+      if (lane == 0) {
+        for (int c = c_split; c < c_end && !*abort_flag; ++c)
+          if (!issue(c, w0)) break;
       }
       __syncwarp();  // s_ids is rewritten for the next window
     }

@@ -15,6 +15,7 @@
 //    unsynchronised counts free shared blocks early).
 #include "../../include/pagedkv.h"
 
+#include <algorithm>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -257,6 +258,37 @@ int bm_free_list(pagedkv_block_manager* m, int32_t* out, int cap) {
   if (cap < n) return bm_fail(PAGEDKV_ERANGE, "free list of %lld does not fit", n);
   if (n) memcpy(out, m->free_list.data(), n * sizeof(int32_t));
   return n;
+}
+
+int bm_stats(pagedkv_block_manager* m, pagedkv_bm_stats* out) {
+  if (!m || !out) return bm_fail(PAGEDKV_EINVAL, "NULL argument");
+  std::lock_guard<std::mutex> lock(m->mu);
+  std::vector<int32_t> fill(m->num_blocks, 0);
+  int64_t logical = 0, entries = 0;
+  for (const auto& kv : m->seqs) {
+    const auto& s = kv.second;
+    logical += s.len;
+    entries += (int64_t)s.table.size();
+    for (size_t j = 0; j < s.table.size(); ++j) {
+      const int64_t in_block = std::min<int64_t>(m->block_size, s.len - (int64_t)j * m->block_size);
+      int32_t& f = fill[s.table[j]];
+      if (in_block > f) f = (int32_t)in_block;
+    }
+  }
+  int64_t used = 0, filled = 0;
+  for (int b = 0; b < m->num_blocks; ++b) {
+    if (m->refcount[b] > 0) ++used;
+    filled += fill[b];
+  }
+  out->num_blocks = m->num_blocks;
+  out->free_blocks = (int64_t)m->free_list.size();
+  out->used_blocks = used;
+  out->num_seqs = (int64_t)m->seqs.size();
+  out->logical_tokens = logical;
+  out->filled_slots = filled;
+  out->allocated_slots = used * m->block_size;
+  out->table_entries = entries;
+  return PAGEDKV_OK;
 }
 
 // Message of the calling thread's last failed bm_* call.

@@ -77,11 +77,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete; false after the timeout.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          unsigned long long timeout_ns = WAIT_TIMEOUT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > WAIT_TIMEOUT_NS) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
   return true;
 }
@@ -120,6 +121,75 @@ __device__ __forceinline__ void tensor_load_2d(uint32_t dst, const CUtensorMap* 
 __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
+
+// ---- fused append -----------------------------------------------------------------
+//
+// The attention kernels can write the step's new K/V row themselves (the
+// scatter of the new token into its block, then the gather that reads it back:
+// lpnh.cn/news/1824136 §3.1).  The producer warp stores the row with ordinary
+// (generic-proxy) stores, orders them before its own later copies with a proxy
+// fence, and only then issues the copy of the stage that holds the row, so the
+// consumers read it like any other row.
+
+// 16-byte relaxed store at gpu scope.  Several CTAs may store the same new row
+// (query groups split over CTAs); relaxed stores of identical bytes do not race.
+__device__ __forceinline__ void st_relaxed_gpu_v4(void* ptr, uint4 v) {
+  asm volatile("st.relaxed.gpu.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Orders this thread's earlier generic-proxy global writes before its later
+// async-proxy (bulk / tensor copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// The new K and V rows of NH consecutive kv heads (kv0 ..), spread as 16-byte
+// vectors over the 32 lanes of a warp: vectors [0, NH*D/8) are K, the rest V.
+template <int D, int NH>
+struct NewRows {
+  static constexpr int VPH = D / 8;             // vectors per head row
+  static constexpr int NV = 2 * NH * VPH;
+  static constexpr int PER_LANE = (NV + 31) / 32;
+  uint4 v[PER_LANE];
+
+  // k_new / v_new are [num_seqs][num_kv_heads][D]; the NH rows are contiguous.
+  __device__ __forceinline__ void load(const __half* k_new, const __half* v_new, int b,
+                                       int num_kv_heads, int kv0, int lane) {
+    const size_t row0 = ((size_t)b * num_kv_heads + kv0) * D;
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+      const int idx = lane + 32 * i;
+      if (idx < NV) {
+        const bool is_v = idx >= NH * VPH;
+        const int off = is_v ? idx - NH * VPH : idx;
+        v[i] = __ldg(reinterpret_cast<const uint4*>((is_v ? v_new : k_new) + row0) + off);
+      }
+    }
+  }
+
+  // Stores the rows into row r of physical block phys of the pools
+  // ([N][Hk][bs][D]) and fences them before this warp's later copies.
+  // Called by all 32 lanes.
+  __device__ __forceinline__ void store(__half* k_cache, __half* v_cache, int num_kv_heads,
+                                        int bs, int kv0, int phys, int r, int lane) const {
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+      const int idx = lane + 32 * i;
+      if (idx < NV) {
+        const bool is_v = idx >= NH * VPH;
+        const int off = is_v ? idx - NH * VPH : idx;
+        const int h = off / VPH;
+        __half* dst = (is_v ? v_cache : k_cache) +
+                      (((size_t)phys * num_kv_heads + kv0 + h) * bs + r) * D + (off % VPH) * 8;
+        st_relaxed_gpu_v4(dst, v[i]);
+      }
+    }
+    fence_proxy_async_global();
+    __syncwarp();
+  }
+};
 
 // ---- warp-level tensor-core helpers --------------------------------------------
 

@@ -26,6 +26,10 @@ struct DecodeParams {
   int part_tokens;             // tokens per partition (a multiple of 16 and of bs)
   int num_parts;               // partitions per sequence in the grid
   int stages;                  // depth of the shared-memory ring
+  // Fused append (NULL = none): this step's new K/V rows, [B][Hk][D], which the
+  // kernel writes to position L_b - 1 through the block table before reading it.
+  const __half* k_new;
+  const __half* v_new;
 };
 
 // Consumer warps of the grouped-query (tensor-core) kernel; plus one producer warp.

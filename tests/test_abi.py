@@ -80,6 +80,35 @@ def test_decode_rejects_bad_arguments_on_the_host(lib, over, code):
     assert lib.pagedkv_last_error().decode()
 
 
+def _decode_append(lib, kn=FAKE, vn=FAKE, **over):
+    a = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, scale=0.1, bs=16, hk=8, b=4,
+             h=8, d=128, maxblk=8, n=64, maxlen=100, part=0, ws=None, wsb=0)
+    a.update(over)
+    return lib.paged_attention_decode_append(a["out"], a["q"], kn, vn, a["kc"], a["vc"], a["bt"],
+                                             a["cl"], a["scale"], a["bs"], a["hk"], a["b"], a["h"],
+                                             a["d"], a["maxblk"], a["n"], a["maxlen"], a["part"],
+                                             a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(kn=None), nat.EINVAL),
+    (dict(vn=None), nat.EINVAL),
+    (dict(kn=FAKE + 8), nat.EINVAL),                  # misaligned
+    (dict(q=None), nat.EINVAL),
+    (dict(d=96), nat.EUNSUPPORTED),
+    (dict(part=32), nat.EWORKSPACE),
+])
+def test_fused_append_rejects_bad_arguments_on_the_host(lib, over, code):
+    assert _decode_append(lib, **over) == code
+    assert lib.pagedkv_last_error().decode()
+    assert _decode_append(lib, b=0, kn=None, q=None) == nat.OK   # empty batch: no-op
+
+
+def test_self_test_rejects_bad_timeouts_on_the_host(lib):
+    assert lib.pagedkv_selftest_wait_timeout(0, None) == nat.EINVAL
+    assert lib.pagedkv_selftest_wait_timeout(1_000_001, None) == nat.EINVAL
+
+
 def test_empty_batch_is_a_no_op(lib):
     assert _decode(lib, b=0, q=None) == nat.OK
 

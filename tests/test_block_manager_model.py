@@ -34,6 +34,20 @@ def test_block_counts_and_tail_waste(oracle_mod, row):
     assert len(m.block_table(s)) == blocks
     assert tokens - (blocks - 1) * bs == tail
     assert blocks * bs == capacity and capacity - tokens == wasted
+    st = m.stats()
+    assert st["allocated_slots"] == capacity and st["filled_slots"] == tokens
+    assert st["allocated_slots"] - st["filled_slots"] == wasted
+
+
+def test_stats_count_shared_blocks_once(oracle_mod):
+    m = _model(oracle_mod, 64, 16)
+    p = m.add_seq(1000)                        # 62 full blocks and a tail of 8
+    m.fork(p, 7)
+    st = m.stats()
+    assert st["used_blocks"] == 63 and st["allocated_slots"] == 63 * 16
+    assert st["filled_slots"] == 1000          # one copy of the shared prefix
+    assert st["logical_tokens"] == 8 * 1000 and st["table_entries"] == 8 * 63
+    assert st["num_seqs"] == 8 and st["free_blocks"] == 1
 
 
 def test_block_counts_grow_on_demand(oracle_mod):

@@ -22,6 +22,7 @@ def _same_state(native, model, ids):
         assert native.seq_len(s) == model.lens[s]
     assert native.free_list() == model.free
     assert [native.refcount(b) for b in range(model.num_blocks)] == model.refcount
+    assert native.stats() == model.stats()
 
 
 def test_block_table_figure():
@@ -164,3 +165,19 @@ def test_concurrent_callers_keep_counts_consistent():
     for s in live:
         bm.free_seq(s)
     assert bm.num_free() == N
+
+
+def test_block_size_trade_off_on_the_llama7b_batch():
+    # smaller blocks: less tail waste, longer tables, more allocations per append
+    from paged_kv_cache_393_b200 import bm_bench
+    r = {bs: bm_bench.run(bs, steps=20) for bs in (8, 16, 32, 64)}
+    waste = [r[bs]["tail_waste"] for bs in (8, 16, 32, 64)]
+    entries = [r[bs]["table_entries"] for bs in (8, 16, 32, 64)]
+    allocs = [r[bs]["blocks_allocated_per_1000_appends"] for bs in (8, 16, 32, 64)]
+    assert waste == sorted(waste) and entries == sorted(entries, reverse=True)
+    assert allocs == sorted(allocs, reverse=True)
+    # a uniform tail wastes about (bs - 1) / 2 slots per sequence
+    for bs in (8, 16, 32, 64):
+        st = r[bs]["stats"]
+        per_seq = (st["allocated_slots"] - st["filled_slots"]) / st["num_seqs"]
+        assert abs(per_seq - (bs - 1) / 2) < 0.25 * bs

@@ -39,19 +39,37 @@ def _bits(t):
     return t.detach().cpu().numpy().view(np.uint16)
 
 
-def _run_and_compare(pkv, w, partition_size=0, sample=None, check_pool=True):
+def _run_and_compare(pkv, w, partition_size=0, sample=None, check_pool=True, fused=False):
     from paged_kv_cache_393_b200.batch import PagedBatch
     gb = PagedBatch(w, DEV)
     ob = OracleBatch(w, sample)
     # the product block manager and the oracle's model agree exactly
     assert [gb.bm.block_table(s) for s in gb.seqs] == ob.tables
     assert np.array_equal(gb.slots_host, ob.new_slots)
-    # one decode step: scatter the new token, then attend
-    pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
-    pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
-                               gb.context_lens, w.scale, gb.max_context_len, partition_size)
+    if fused:
+        # one call writes the new token at position L-1 through the table, then attends
+        pkv.paged_attention_decode_append(gb.out, gb.q, gb.k_new, gb.v_new, gb.key_cache,
+                                          gb.value_cache, gb.block_tables, gb.context_lens,
+                                          w.scale, gb.max_context_len, partition_size)
+    else:
+        # one decode step: scatter the new token, then attend
+        pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
+        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                                   gb.context_lens, w.scale, gb.max_context_len, partition_size)
     torch.cuda.synchronize()
     assert pkv.device_errors() == 0
+    if fused:
+        # the same kernels over the same (now updated) cache give the same outputs: bit for
+        # bit where the schedule is static; the persistent tensor-core kernel hands out work
+        # at run time, so which warp sums which chunk (the fp32 order) can differ
+        fused_out = gb.out.clone()
+        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                                   gb.context_lens, w.scale, gb.max_context_len, partition_size)
+        G = w.num_heads // w.num_kv_heads
+        if 2 <= G <= 8 and w.block_size >= 8 and w.num_seqs <= 1024:
+            assert_attention_close(fused_out.cpu().numpy(), gb.out.cpu().numpy())
+        else:
+            assert np.array_equal(_bits(fused_out), _bits(gb.out))
     if check_pool:
         idx = torch.tensor(ob.blocks, dtype=torch.long, device=DEV)
         assert np.array_equal(_bits(gb.key_cache[idx]), ob.key_cache.view(np.uint16))

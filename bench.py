@@ -187,8 +187,13 @@ def hbm_peak():
 
 
 def kernel_source_hash(path: str) -> str:
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256/16 of a kernel file together with the headers every kernel file includes."""
+    h = hashlib.sha256()
+    d = os.path.dirname(path)
+    for f in (path, os.path.join(d, "common.cuh"), os.path.join(d, "kernels.h")):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel_file: str, workload: str):

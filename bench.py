@@ -50,9 +50,11 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b")
     ap.add_argument("--e2e-steps", type=int, default=300)
-    ap.add_argument("--step", choices=["fused", "separate"], default="fused",
+    ap.add_argument("--step", choices=["fused", "separate", "shared"], default="fused",
                     help="fused: one paged_attention_decode_append call writes the new tokens "
-                         "and attends; separate: reshape_and_cache then paged_attention_decode")
+                         "and attends; separate: reshape_and_cache then paged_attention_decode; "
+                         "shared (cow workload): the fused shared-prefix call, which reads each "
+                         "group's shared prompt blocks once")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
@@ -388,15 +390,27 @@ def run_cow(args, w, dev, world, rank, local):
     B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
     steps_host = [gb.prepare_step() for _ in range(w.decode_steps)]
     up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    shared = args.step == "shared"
     steps = []
+    unique_total = 0
     for h in steps_host:
-        steps.append(dict(q=up(h["q"]), k=up(h["k"]), v=up(h["v"]), slots=up(h["slots"]),
-                          tables=up(h["tables"]), lens=up(h["lens"]),
-                          pairs=up(h["pairs"]) if len(h["pairs"]) else None,
-                          kv_bytes=int(h["lens"].astype(np.int64).sum())
-                          * wl.kv_bytes_per_token(Hk, D)))
+        st = dict(q=up(h["q"]), k=up(h["k"]), v=up(h["v"]), slots=up(h["slots"]),
+                  tables=up(h["tables"]), lens=up(h["lens"]),
+                  pairs=up(h["pairs"]) if len(h["pairs"]) else None,
+                  kv_bytes=int(h["lens"].astype(np.int64).sum()) * wl.kv_bytes_per_token(Hk, D))
+        if shared:
+            pre, groups = pkv.prefix_groups(h["tables"], h["lens"], w.block_size, 8 // (H // Hk))
+            st["pre"], st["groups"] = up(pre), up(groups)
+            # K/V bytes the shared-prefix call reads: each group's prefix once, the rest per sequence
+            uniq = int((h["lens"] - pre).astype(np.int64).sum()) + int(groups[:, 0].sum()) * w.block_size
+            st["unique_bytes"] = uniq * wl.kv_bytes_per_token(Hk, D)
+        steps.append(st)
     out = torch.empty((B, H, D), dtype=torch.float16, device=dev)
-    need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, 0)
+    if shared:
+        need = pkv.paged_attention_shared_prefix_workspace_bytes(B, H, Hk, D, w.block_size,
+                                                                 gb.max_context_len, 0)
+    else:
+        need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, 0)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
     n_pairs = len(steps_host[0]["pairs"])
@@ -410,7 +424,12 @@ def run_cow(args, w, dev, world, rank, local):
             pkv.copy_blocks([gb.key_cache], [gb.value_cache], st["pairs"], stream=stream)
             if ev is not None:
                 ev[1].record(stream)
-        if args.step == "fused":
+        if shared:
+            pkv.paged_attention_decode_shared_prefix(
+                out, st["q"], gb.key_cache, gb.value_cache, st["tables"], st["lens"], st["pre"],
+                st["groups"], w.scale, gb.max_context_len, 0, ws, k_new=st["k"], v_new=st["v"],
+                stream=stream)
+        elif args.step == "fused":
             pkv.paged_attention_decode_append(out, st["q"], st["k"], st["v"], gb.key_cache,
                                               gb.value_cache, st["tables"], st["lens"], w.scale,
                                               gb.max_context_len, 0, ws, stream=stream)
@@ -447,8 +466,9 @@ def run_cow(args, w, dev, world, rank, local):
             copy_ev.append(ev)
             launches += 1
         run_step(j, ev)
-        launches += 1 if args.step == "fused" else 2
+        launches += {"fused": 1, "separate": 2, "shared": 3}[args.step]   # shared: prefix, suffix, merge
         kv_total += steps[j]["kv_bytes"]
+        unique_total += steps[j].get("unique_bytes", 0)
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world, local)
@@ -476,6 +496,8 @@ def run_cow(args, w, dev, world, rank, local):
                              "can hit in L2" % prefix_blocks,
                        "parallelism": "replicas x%d" % world},
             "tokens_per_s": round(B * world / (ms_per_step / 1e3), 1),
+            "unique_kv_GB_per_s": round(unique_total * world / (ms_max / 1e3) / 1e9, 2)
+            if shared else None,
             "copy_blocks": {"pairs": n_pairs, "bytes": copy_bytes, "avg_us": copy_us,
                             "GB_per_s": round(copy_bytes / (copy_us / 1e6) / 1e9, 1) if copy_us else None,
                             "peak": peak, "peak_kind": peak_kind},

@@ -70,6 +70,8 @@ extern "C" {
 #define PAGEDKV_DEVERR_SLOT 4u        /* a slot beyond the pool: that token was skipped */
 #define PAGEDKV_DEVERR_TIMEOUT 8u     /* a pipeline wait gave up after ~2 s; output invalid */
 #define PAGEDKV_DEVERR_INTERNAL 16u   /* a kernel found its launch set-up inconsistent and did nothing */
+#define PAGEDKV_DEVERR_PREFIX 32u     /* a shared-prefix group or prefix length was inconsistent:
+                                         that sequence's prefix was not used (output invalid) */
 
 /* Message of the calling thread's last failed call ("" if none). */
 PAGEDKV_API const char *pagedkv_last_error(void);
@@ -175,6 +177,88 @@ PAGEDKV_API int paged_attention_decode_append(void *out, const void *q,
                            int max_blocks_per_seq, int num_blocks, int max_context_len,
                            int partition_size, void *workspace, size_t workspace_bytes,
                            void *stream);
+
+/* ---- shared-prefix decode -----------------------------------------------------------
+ *
+ * Sequences forked from one prompt (parallel sampling, beam search) or served
+ * from one cached prefix reference the same physical blocks at the start of
+ * their block tables (copy-on-write sharing: lpnh.cn/news/2758356 §4.1-§4.2;
+ * prefix caching: n1n.ai "前缀缓存").  paged_attention_decode reads such a
+ * block once per sequence; this call reads it once per group:
+ *
+ *   prefix pass   for every group, kv head and partition of the shared prefix,
+ *                 one tensor-core tile whose columns are the members' query
+ *                 heads of that kv head;
+ *   suffix pass   every sequence over the rest of its context [P_b, L_b);
+ *   merge         the partial softmax states of both, as split-K merges them.
+ *
+ * The result is paged_attention_decode's (same formula, fp32 accumulation,
+ * within rounding of it).  With k_new / v_new given, the new rows are written
+ * first as paged_attention_decode_append writes them (they always lie in the
+ * suffix).
+ *
+ *   seq_prefix_tokens  device int32 [num_seqs]: P_b, the tokens of sequence b
+ *                  that its group's prefix pass covers; 0 = none.  A multiple of
+ *                  block_size and at most L_b - 1.
+ *   groups         device int32 [num_groups][PAGEDKV_GROUP_WIDTH]: the group's
+ *                  prefix length in blocks, then up to 8 member sequence indices
+ *                  (-1 = unused).  A group may hold at most 8 / G members
+ *                  (G = num_heads / num_kv_heads).  Every member's first
+ *                  (prefix blocks) table entries must equal the first member's,
+ *                  and its seq_prefix_tokens must be that many tokens.  A member
+ *                  breaking these rules is left out of the prefix pass and sets
+ *                  PAGEDKV_DEVERR_PREFIX; its output is then invalid.  May be
+ *                  NULL when num_groups is 0.
+ *   partition_size 0 or -1 = 512 tokens; else as for paged_attention_decode.
+ *                  The call always splits.
+ *   workspace      at least paged_attention_shared_prefix_workspace_bytes(...).
+ *   the rest       as for paged_attention_decode / _append.
+ *
+ * Needs block_size >= 8 and G <= 8 (else EUNSUPPORTED).  pagedkv_prefix_groups
+ * builds seq_prefix_tokens and groups from host copies of the tables.
+ * num_seqs == 0 is a no-op.  Errors: EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
+ */
+#define PAGEDKV_GROUP_WIDTH 9
+#define PAGEDKV_GROUP_MAX_MEMBERS 8
+
+PAGEDKV_API int paged_attention_decode_shared_prefix(void *out, const void *q,
+                           const void *k_new, const void *v_new,
+                           void *key_cache, void *value_cache,
+                           const int32_t *block_tables, const int32_t *context_lens,
+                           const int32_t *seq_prefix_tokens, const int32_t *groups,
+                           int num_groups, float scale, int block_size, int num_kv_heads,
+                           int num_seqs, int num_heads, int head_dim,
+                           int max_blocks_per_seq, int num_blocks, int max_context_len,
+                           int partition_size, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Workspace bytes paged_attention_decode_shared_prefix needs (0 for arguments it
+ * would reject). */
+PAGEDKV_API size_t paged_attention_shared_prefix_workspace_bytes(int num_seqs, int num_heads,
+                           int num_kv_heads, int head_dim, int block_size,
+                           int max_context_len, int partition_size);
+
+/* Host helper: groups of a batch that share table prefixes.
+ *
+ * From host copies of the block tables ([num_seqs][max_blocks_per_seq], -1
+ * padded) and context lengths: sequences whose tables start with the same
+ * physical blocks are grouped, at most max_members (1..8; pass 8 / G) per group,
+ * with prefix = the members' common leading blocks, counting only whole blocks
+ * before each member's last token.  Sequences are bucketed by their first
+ * block, sorted by table inside a bucket and cut in that order into groups;
+ * a run with fewer than 2 members or no common block forms no group.
+ *
+ *   seq_prefix_tokens  host int32 [num_seqs] out: prefix blocks * block_size of
+ *                      the sequence's group, 0 = none
+ *   groups             host int32 [groups_capacity][PAGEDKV_GROUP_WIDTH] out
+ *
+ * Returns the number of groups written (>= 0), or EINVAL, or ERANGE when more
+ * than groups_capacity groups exist (seq_prefix_tokens is then all 0).  A
+ * capacity of num_seqs / 2 always suffices. */
+PAGEDKV_API int pagedkv_prefix_groups(const int32_t *block_tables, const int32_t *context_lens,
+                           int num_seqs, int max_blocks_per_seq, int block_size,
+                           int max_members, int32_t *seq_prefix_tokens, int32_t *groups,
+                           int groups_capacity);
 
 /* ---- allocation-free decode ------------------------------------------------------
  *

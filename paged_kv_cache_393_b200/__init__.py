@@ -8,7 +8,9 @@ missing, every call raises.
 
 Functions mirror the C names:
     paged_attention_decode, paged_attention_decode_append (fused: new K/V row
-    written, then attended), paged_attention_workspace_bytes, reshape_and_cache,
+    written, then attended), paged_attention_decode_shared_prefix + prefix_groups
+    (shared prefixes read once per group), paged_attention_workspace_bytes,
+    reshape_and_cache,
     copy_blocks, device_errors, BlockManager (bm_*), decode_step (host buffers
     in, host result out).
 """
@@ -23,7 +25,10 @@ from ._native import (  # noqa: F401
     load_library,
     paged_attention_decode,
     paged_attention_decode_append,
+    paged_attention_decode_shared_prefix,
+    paged_attention_shared_prefix_workspace_bytes,
     paged_attention_workspace_bytes,
+    prefix_groups,
     reshape_and_cache,
     selftest_wait_timeout,
     DEVERR_BLOCK_ID,
@@ -31,4 +36,6 @@ from ._native import (  # noqa: F401
     DEVERR_SLOT,
     DEVERR_TIMEOUT,
     DEVERR_INTERNAL,
+    DEVERR_PREFIX,
+    GROUP_WIDTH,
 )

@@ -20,6 +20,8 @@ _lock = threading.Lock()
 
 OK, EINVAL, EUNSUPPORTED, ECUDA, EWORKSPACE, ENOMEM, ENOENT, ERANGE = 0, -1, -2, -3, -4, -5, -6, -7
 DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT, DEVERR_INTERNAL = 1, 2, 4, 8, 16
+DEVERR_PREFIX = 32
+GROUP_WIDTH, GROUP_MAX_MEMBERS = 9, 8
 
 
 class PagedKVError(RuntimeError):
@@ -53,6 +55,10 @@ def load_library():
             "paged_attention_decode_append": (
                 [P, P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
             "paged_attention_workspace_bytes": ([I, I, I, I, I, I, I], Z),
+            "paged_attention_decode_shared_prefix": (
+                [P, P, P, P, P, P, P, P, P, P, I, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
+            "paged_attention_shared_prefix_workspace_bytes": ([I, I, I, I, I, I, I], Z),
+            "pagedkv_prefix_groups": ([P, P, I, I, I, I, P, P, I], I),
             "reshape_and_cache": ([P, P, P, P, P, I, I, I, I, I, P], I),
             "copy_blocks": ([P, P, P, I, I, Z, I, P], I),
             "bm_create": ([I, I, P], P),
@@ -164,6 +170,79 @@ def _decode(name, out, q, k_new, v_new, key_cache, value_cache, block_tables, co
                             int(max_context_len), int(partition_size), ws_ptr, ws_bytes,
                             _stream(stream, q.device))
     _check(st, name)
+    return out
+
+
+def paged_attention_shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                  block_size, max_context_len,
+                                                  partition_size=0) -> int:
+    return int(load_library().paged_attention_shared_prefix_workspace_bytes(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size))
+
+
+def prefix_groups(block_tables, context_lens, block_size, max_members):
+    """Host grouping of a batch by shared table prefixes (pagedkv_prefix_groups).
+
+    block_tables: int32 [B][max_blocks] (-1 padded), context_lens: int32 [B] (numpy).
+    Returns (seq_prefix_tokens int32 [B], groups int32 [n][GROUP_WIDTH])."""
+    lib = load_library()
+    t = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    B = t.shape[0]
+    if t.ndim != 2 or lens.shape != (B,):
+        raise ValueError("block_tables must be [B][max_blocks] and context_lens [B]")
+    pre = np.zeros(B, np.int32)
+    cap = max(B // 2, 1)
+    groups = np.zeros((cap, GROUP_WIDTH), np.int32)
+    n = lib.pagedkv_prefix_groups(_np_ptr(t), _np_ptr(lens), B, t.shape[1], int(block_size),
+                                  int(max_members), _np_ptr(pre), _np_ptr(groups), cap)
+    _check(n, "pagedkv_prefix_groups")
+    return pre, groups[:n].copy()
+
+
+def paged_attention_decode_shared_prefix(out, q, key_cache, value_cache, block_tables,
+                                         context_lens, seq_prefix_tokens, groups, scale,
+                                         max_context_len, partition_size=0, workspace=None,
+                                         k_new=None, v_new=None, stream=None):
+    """Paged decode attention that reads each group's shared prefix once (device tensors:
+    seq_prefix_tokens int32 [B], groups int32 [n][GROUP_WIDTH]); with k_new/v_new the new
+    rows are written first, as paged_attention_decode_append does."""
+    lib = load_library()
+    B, H, D = q.shape
+    N, Hk, bs, D2 = key_cache.shape
+    if D2 != D or tuple(value_cache.shape) != tuple(key_cache.shape) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
+        raise ValueError("block_tables must be [B][max_blocks] and context_lens [B]")
+    if tuple(seq_prefix_tokens.shape) != (B,) or groups.dim() != 2 or groups.shape[1] != GROUP_WIDTH:
+        raise ValueError("seq_prefix_tokens must be [B] and groups [n][%d]" % GROUP_WIDTH)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    kn = vn = None
+    if k_new is not None:
+        if tuple(k_new.shape) != (B, Hk, D) or tuple(v_new.shape) != (B, Hk, D):
+            raise ValueError("k_new and v_new must be [B][Hk][D]")
+        kn, vn = _cuda(k_new, "k_new", torch.float16, 3), _cuda(v_new, "v_new", torch.float16, 3)
+    ng = groups.shape[0]
+    gptr = _cuda(groups, "groups", torch.int32, 2) if ng else None
+    need = paged_attention_shared_prefix_workspace_bytes(B, H, Hk, D, bs, max_context_len,
+                                                         partition_size)
+    ws_ptr, ws_bytes = None, 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _cuda(workspace, "workspace", workspace.dtype)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = lib.paged_attention_decode_shared_prefix(
+        _cuda(out, "out", torch.float16, 3), _cuda(q, "q", torch.float16, 3), kn, vn,
+        _cuda(key_cache, "key_cache", torch.float16, 4),
+        _cuda(value_cache, "value_cache", torch.float16, 4),
+        _cuda(block_tables, "block_tables", torch.int32, 2),
+        _cuda(context_lens, "context_lens", torch.int32, 1),
+        _cuda(seq_prefix_tokens, "seq_prefix_tokens", torch.int32, 1), gptr, ng, float(scale),
+        bs, Hk, B, H, D, block_tables.shape[1], N, int(max_context_len), int(partition_size),
+        ws_ptr, ws_bytes, _stream(stream, q.device))
+    _check(st, "paged_attention_decode_shared_prefix")
     return out
 
 

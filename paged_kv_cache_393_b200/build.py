@@ -18,7 +18,7 @@ BUILD = os.path.join(ROOT, "_build", "pagedkv")
 LIB = os.path.join(HERE, "libpagedkv.so")
 
 SOURCES = ["api.cu", "attention_simt.cu", "attention_mma.cu", "split_merge.cu", "cache_ops.cu",
-           "block_manager.cpp", "noalloc.cu"]
+           "block_manager.cpp", "noalloc.cu", "prefix_groups.cpp"]
 HEADERS = [os.path.join(CSRC, h) for h in ("common.cuh", "kernels.h")] + [
     os.path.join(ROOT, "include", "pagedkv.h")]
 

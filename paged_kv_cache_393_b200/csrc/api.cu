@@ -130,6 +130,8 @@ struct Plan {
   int stages = 2;
   size_t smem = 0;
   size_t ws_bytes = 0;
+  bool cascade = false;      // shared-prefix decode: prefix pass + suffix pass + merge
+  int prefix_stages = 0;     // ring depth of the prefix pass
 };
 
 bool valid_block_size(int bs) { return bs == 4 || bs == 8 || bs == 16 || bs == 32 || bs == 64; }
@@ -141,7 +143,7 @@ int largest_divisor_of(int n, const int* choices, int count) {
 }
 
 int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-              int block_size, int max_context_len, int partition_size) {
+              int block_size, int max_context_len, int partition_size, bool cascade = false) {
   if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
     return fail(PAGEDKV_EINVAL, "num_heads (%d) must be a positive multiple of num_kv_heads (%d)",
                 num_heads, num_kv_heads);
@@ -153,7 +155,12 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
   if (num_seqs < 0 || num_seqs > 65535)
     return fail(PAGEDKV_EUNSUPPORTED, "num_seqs %d outside [0, 65535]", num_seqs);
   const int G = num_heads / num_kv_heads;
+  if (cascade && (G > 8 || block_size < 8))
+    return fail(PAGEDKV_EUNSUPPORTED,
+                "shared-prefix decode needs block_size >= 8 and at most 8 query heads per kv "
+                "head (block_size %d, %d)", block_size, G);
   Plan p;
+  p.cascade = cascade;
   p.mma = G >= 2 && G <= 8 && block_size >= 8;
   const Tuning& tn = tuning();
   if (!p.mma) {
@@ -180,7 +187,11 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
   // split-K: explicit, or automatic for long contexts / too few CTAs to fill the GPU
   const int unit = p.mma ? 16 : block_size;
   const int align = block_size > 16 ? block_size : 16;
-  if (partition_size > 0) {
+  if (cascade && partition_size <= 0) {
+    // always split: the prefix and suffix passes each leave partial results
+    p.split = true;
+    p.part_tokens = AUTO_PARTITION % align == 0 ? AUTO_PARTITION : align;
+  } else if (partition_size > 0) {
     if (partition_size % align != 0)
       return fail(PAGEDKV_EINVAL, "partition_size %d must be a multiple of 16 and of block_size",
                   partition_size);
@@ -201,7 +212,8 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
   }
   (void)unit;
   if (p.split) {
-    p.num_parts = (max_context_len + p.part_tokens - 1) / p.part_tokens;
+    // a shared prefix can end inside a partition: one more slot per (sequence, head)
+    p.num_parts = (max_context_len + p.part_tokens - 1) / p.part_tokens + (cascade ? 1 : 0);
     if (p.num_parts > MAX_PARTITIONS)
       return fail(PAGEDKV_EUNSUPPORTED, "%d partitions exceed %d: use a larger partition_size",
                   p.num_parts, MAX_PARTITIONS);
@@ -234,6 +246,14 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     while (st > 2 && simt_smem_bytes(head_dim, block_size, p.kvc, st) > MAX_SMEM) --st;
     p.stages = st;
     p.smem = simt_smem_bytes(head_dim, block_size, p.kvc, st);
+  }
+  if (cascade) {
+    int st = tn.mma_stages > 0 ? tn.mma_stages : 4;
+    st = ((st + MMA_CONSUMER_WARPS - 1) / MMA_CONSUMER_WARPS) * MMA_CONSUMER_WARPS;
+    st = st > 16 ? 16 : st;
+    while (st > MMA_CONSUMER_WARPS && mma_smem_bytes(head_dim, block_size, st) > MAX_SMEM)
+      st -= MMA_CONSUMER_WARPS;
+    p.prefix_stages = st;
   }
   if (p.smem > MAX_SMEM) return fail(PAGEDKV_EUNSUPPORTED, "shared memory plan too large");
   *plan = p;
@@ -307,13 +327,22 @@ size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_h
 namespace pkv {
 namespace {
 
-// Both decode entry points; k_new / v_new are NULL for the plain one.
+// Every decode entry point.  k_new / v_new are NULL without a fused append;
+// cascade selects the shared-prefix form (seq_prefix_tokens, groups).
 int decode(void* out, const void* q, const void* k_new, const void* v_new, const void* key_cache,
            const void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
            float scale, int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
            int max_blocks_per_seq, int num_blocks, int max_context_len, int partition_size,
-           void* workspace, size_t workspace_bytes, void* stream) {
+           void* workspace, size_t workspace_bytes, void* stream, bool cascade = false,
+           const int32_t* seq_prefix_tokens = nullptr, const int32_t* groups = nullptr,
+           int num_groups = 0) {
   if (num_seqs == 0) return PAGEDKV_OK;
+  if (cascade) {
+    if (!seq_prefix_tokens) return fail(PAGEDKV_EINVAL, "seq_prefix_tokens is required");
+    if (num_groups < 0 || num_groups > 65535)
+      return fail(PAGEDKV_EINVAL, "num_groups %d outside [0, 65535]", num_groups);
+    if (num_groups > 0 && !groups) return fail(PAGEDKV_EINVAL, "groups is NULL");
+  }
   if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
     return fail(PAGEDKV_EINVAL, "a required pointer is NULL");
   if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache))
@@ -326,9 +355,10 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
                 max_context_len, max_blocks_per_seq, block_size);
   Plan plan;
   int st = make_plan(&plan, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                     max_context_len, partition_size);
+                     max_context_len, partition_size, cascade);
   if (st != PAGEDKV_OK) return st;
-  if (plan.mma && (long long)num_blocks * num_kv_heads * block_size > 0x7fffffffLL)
+  const bool maps = plan.mma || (cascade && num_groups > 0);  // tensor-core passes need tensor maps
+  if (maps && (long long)num_blocks * num_kv_heads * block_size > 0x7fffffffLL)
     return fail(PAGEDKV_EUNSUPPORTED, "pool of %lld rows exceeds the tensor-map range",
                 (long long)num_blocks * num_kv_heads * block_size);
   if (plan.ws_bytes > 0) {
@@ -367,16 +397,30 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
   p.stages = plan.stages;
   p.k_new = static_cast<const __half*>(k_new);
   p.v_new = static_cast<const __half*>(v_new);
+  p.seq_prefix_tokens = cascade ? seq_prefix_tokens : nullptr;
+  p.groups = cascade ? groups : nullptr;
+  p.num_groups = cascade ? num_groups : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   cudaError_t e;
-  if (plan.mma) {
-    CUtensorMap km, vm;
+  CUtensorMap km, vm;
+  if (maps) {
     const int rows = num_blocks * num_kv_heads * block_size;
     st = encode_pool_map(&km, key_cache, rows, head_dim, block_size);
     if (st != PAGEDKV_OK) return st;
     st = encode_pool_map(&vm, value_cache, rows, head_dim, block_size);
     if (st != PAGEDKV_OK) return st;
+  }
+  if (cascade && num_groups > 0) {
+    // prefix pass first; the suffix pass and the merge follow in stream order
+    DecodeParams pp = p;
+    pp.stages = plan.prefix_stages;
+    pp.k_new = pp.v_new = nullptr;
+    const int prefix_parts = (max_context_len + plan.part_tokens - 1) / plan.part_tokens;
+    e = launch_mma_prefix(pp, km, vm, prefix_parts, s);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-prefix pass launch");
+  }
+  if (plan.mma) {
     if (plan.persistent) {
       const size_t parts_bytes =
           plan.split ? (size_t)num_seqs * num_heads * plan.num_parts * (head_dim + 2) * sizeof(float)
@@ -428,6 +472,35 @@ int paged_attention_decode_append(void* out, const void* q, const void* k_new, c
   return decode(out, q, k_new, v_new, key_cache, value_cache, block_tables, context_lens, scale,
                 block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq,
                 num_blocks, max_context_len, partition_size, workspace, workspace_bytes, stream);
+}
+
+int paged_attention_decode_shared_prefix(
+    void* out, const void* q, const void* k_new, const void* v_new, void* key_cache,
+    void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+    const int32_t* seq_prefix_tokens, const int32_t* groups, int num_groups, float scale,
+    int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+    int max_blocks_per_seq, int num_blocks, int max_context_len, int partition_size,
+    void* workspace, size_t workspace_bytes, void* stream) {
+  if (num_seqs == 0) return PAGEDKV_OK;
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(PAGEDKV_EINVAL, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
+    return fail(PAGEDKV_EINVAL, "k_new and v_new must be 16-byte aligned");
+  return decode(out, q, k_new, v_new, key_cache, value_cache, block_tables, context_lens, scale,
+                block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq,
+                num_blocks, max_context_len, partition_size, workspace, workspace_bytes, stream,
+                true, seq_prefix_tokens, groups, num_groups);
+}
+
+size_t paged_attention_shared_prefix_workspace_bytes(int num_seqs, int num_heads,
+                                                     int num_kv_heads, int head_dim,
+                                                     int block_size, int max_context_len,
+                                                     int partition_size) {
+  Plan plan;
+  if (make_plan(&plan, num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                partition_size, true) != PAGEDKV_OK)
+    return 0;
+  return plan.ws_bytes;
 }
 
 int reshape_and_cache(const void* k, const void* v, void* key_cache, void* value_cache,

@@ -310,6 +310,19 @@ __device__ __forceinline__ void load_q_fragments(uint32_t (&qb)[D / 16][2], cons
   }
 }
 
+// Same fragments when every column comes from its own row: `qrow` is this
+// lane's column (lane >> 2), NULL for a zero column.
+template <int D>
+__device__ __forceinline__ void load_q_column(uint32_t (&qb)[D / 16][2], const __half* qrow,
+                                              int lane) {
+  const int t = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    qb[ks][0] = qrow ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
+    qb[ks][1] = qrow ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t + 8) : 0u;
+  }
+}
+
 // Each warp's state into the merge buffers (after the per-head sums are reduced).
 template <int D>
 __device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, float* s_o, int warp,
@@ -340,29 +353,30 @@ __device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, f
 // Merges the consumer warps' states of item (b, kvh, part) and stores the result:
 // the fp16 output when the item is the whole context, else the partition's
 // (max, sum, unnormalised output) for the merge kernel.
-template <int D>
-__device__ __forceinline__ void store_item(const float* s_m, const float* s_l, const float* s_o,
-                                           const DecodeParams& p, int b, int kvh, int part, int G,
-                                           bool whole) {
-  using Geo = StageGeom<D>;
-  for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
-    const int head = idx / D;
+template <int D, typename ColumnRow>
+__device__ __forceinline__ void store_columns(const float* s_m, const float* s_l, const float* s_o,
+                                              const DecodeParams& p, int ncols, ColumnRow row_of,
+                                              int part, bool whole) {
+  // row_of(c): the (sequence * num_heads + head) row of column c, or -1 to skip it
+  for (int idx = threadIdx.x; idx < ncols * D; idx += NW * 32) {
+    const int col = idx / D;
     const int d = idx % D;
+    const long long bh = row_of(col);
+    if (bh < 0) continue;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * 8 + head]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * 8 + col]);
     float num = 0.f, den = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      const float a = rescale_factor(s_m[w * 8 + head], M);
-      num = fmaf(a, s_o[(w * 8 + head) * Geo::OSTRIDE + d], num);
-      den = fmaf(a, s_l[w * 8 + head], den);
+      const float a = rescale_factor(s_m[w * 8 + col], M);
+      num = fmaf(a, s_o[(w * 8 + col) * StageGeom<D>::OSTRIDE + d], num);
+      den = fmaf(a, s_l[w * 8 + col], den);
     }
-    const size_t bh = (size_t)b * p.num_heads + kvh * G + head;
     if (whole) {
-      p.out[bh * D + d] = __float2half_rn(num / den);
+      p.out[(size_t)bh * D + d] = __float2half_rn(num / den);
     } else {
-      const size_t slot = bh * p.num_parts + part;
+      const size_t slot = (size_t)bh * p.num_parts + part;
       p.ws_o[slot * D + d] = num;
       if (d == 0) {
         p.ws_ml[slot * 2] = M;
@@ -370,6 +384,16 @@ __device__ __forceinline__ void store_item(const float* s_m, const float* s_l, c
       }
     }
   }
+}
+
+// Merges the consumer warps' states of one item (columns = the G query heads
+// of kv head kvh of sequence b) into out, or into partial slot `part`.
+template <int D>
+__device__ __forceinline__ void store_item(const float* s_m, const float* s_l, const float* s_o,
+                                           const DecodeParams& p, int b, int kvh, int part, int G,
+                                           bool whole) {
+  const long long row0 = (long long)b * p.num_heads + (long long)kvh * G;
+  store_columns<D>(s_m, s_l, s_o, p, G, [&](int c) { return row0 + c; }, part, whole);
 }
 
 // ---- one CTA per (sequence, kv head, partition) ---------------------------------
@@ -413,11 +437,16 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     }
     return;
   }
-  const int tok0 = part * p.part_tokens;
+  // with a shared prefix this kernel covers the suffix [P, L) (see the CUDA-core kernel)
+  bool bad_prefix = false;
+  const int P = prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad_prefix);
+  if (bad_prefix && reporter) flag_error(p.err, ERR_PREFIX);
+  const int tok0 = P + part * p.part_tokens;
   const int ntok = min(L, tok0 + p.part_tokens) - tok0;
   if (ntok <= 0) return;
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
   const int nblk = (ntok + BS - 1) / BS;
+  const int slot_part = (P + p.part_tokens - 1) / p.part_tokens + part;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -481,7 +510,162 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   write_state<D>(a, s_m, s_l, s_o, warp, lane);
   named_barrier_sync(1, NW * 32);
-  store_item<D>(s_m, s_l, s_o, p, b, kvh, part, G, !SPLIT || L <= p.part_tokens);
+  store_item<D>(s_m, s_l, s_o, p, b, kvh, slot_part, G, !SPLIT || (P == 0 && L <= p.part_tokens));
+}
+
+// ---- shared-prefix pass ------------------------------------------------------------
+//
+// Sequences forked from one prompt share the prompt's blocks through their
+// tables (lpnh.cn/news/2758356 §4.1-§4.2; n1n.ai "前缀缓存").  This pass reads
+// such a shared prefix once for all sequences of a group: CTA = (kv head,
+// group, prefix partition), and the columns of the tensor-core tile are the
+// members' query heads of that kv head (member-major, G per member, at most 8
+// columns), so every K/V stage feeds all members.  Each member's partial
+// result goes to its prefix slots; the suffix pass covers the tokens after the
+// prefix and the merge combines the two.
+//
+// A member is used only if its prefix length matches the group's and its table
+// entries over this partition equal those of the group's first usable member;
+// otherwise it is dropped from the tile and PAGEDKV_DEVERR_PREFIX is raised.
+
+template <int D, int BS>
+__global__ void __launch_bounds__((NW + 1) * 32)
+    mma_prefix_kernel(const __grid_constant__ CUtensorMap k_map,
+                      const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
+  using Geo = StageGeom<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ int s_member[GROUP_MAX_MEMBERS];  // sequence of each member slot, -1 = none
+  __shared__ int s_reject[GROUP_MAX_MEMBERS];
+  const int stages = p.stages;
+  const uint32_t ring = smem_u32(smem);
+  int* s_ids = reinterpret_cast<int*>(smem + (size_t)stages * 2 * Geo::TILE_BYTES);  // [32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_ids + 32);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * stages);
+  float* s_m = reinterpret_cast<float*>(smem);  // merge buffers over the drained ring
+  float* s_l = s_m + NW * 8;
+  float* s_o = s_l + NW * 8;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kvh = blockIdx.x;
+  const int grp = blockIdx.y;
+  const int part = blockIdx.z;
+  const int G = p.num_heads / p.num_kv_heads;
+  const int max_members = 8 / G;  // columns are member-major, G heads each
+  const int32_t* gd = p.groups + (size_t)grp * GROUP_WIDTH;
+  const int pblocks = gd[0];
+  if (pblocks <= 0 || pblocks > p.max_blocks) {
+    if (threadIdx.x == 0 && kvh == 0 && part == 0) flag_error(p.err, ERR_PREFIX);
+    return;
+  }
+  const int P = pblocks * BS;
+  const int tok0 = part * p.part_tokens;
+  if (tok0 >= P) return;
+  const int ntok = min(P, tok0 + p.part_tokens) - tok0;
+  const int nchunks = (ntok + CHUNK - 1) / CHUNK;
+  const int nblk = (ntok + BS - 1) / BS;
+  const int blk0 = tok0 / BS;
+  const bool reporter = kvh == 0 && part == 0;
+
+  if (threadIdx.x < GROUP_MAX_MEMBERS) {
+    const int i = threadIdx.x;
+    const int m = gd[1 + i];
+    bool ok = m >= 0 && m < p.num_seqs && i < max_members;
+    if (ok) {
+      const int L = min(p.context_lens[m], p.max_context_len);
+      bool bad = false;
+      ok = L > 0 && prefix_tokens_of(p.seq_prefix_tokens, m, L, BS, &bad) == P;
+    }
+    if (!ok && m != -1 && reporter) flag_error(p.err, ERR_PREFIX);
+    s_member[i] = ok ? m : -1;
+    s_reject[i] = 0;
+  }
+  __syncthreads();
+  int first = -1;
+  for (int i = 0; i < GROUP_MAX_MEMBERS && first < 0; ++i) first = s_member[i];
+  if (first < 0) return;  // no usable member (uniform)
+  const int32_t* ref_row = p.block_tables + (size_t)first * p.max_blocks + blk0;
+  for (int idx = threadIdx.x; idx < GROUP_MAX_MEMBERS * nblk; idx += blockDim.x) {
+    const int i = idx / nblk;
+    const int m = s_member[i];
+    if (m >= 0 && m != first && p.block_tables[(size_t)m * p.max_blocks + blk0 + idx % nblk] !=
+                                    ref_row[idx % nblk])
+      s_reject[i] = 1;
+  }
+  __syncthreads();
+  if (threadIdx.x < GROUP_MAX_MEMBERS && s_reject[threadIdx.x]) {
+    s_member[threadIdx.x] = -1;
+    flag_error(p.err, ERR_PREFIX);
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);
+      mbar_init(smem_u32(&bars[stages + s]), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == NW) {
+    // ---------------- producer warp: the first usable member's table ----------------
+    if (lane == 0) {
+      prefetch_tensor_map(&k_map);
+      prefetch_tensor_map(&v_map);
+    }
+    int issued_end = 0;
+    produce_item<D, BS>(ref_row, nblk, nchunks, 0, kvh, first, -1, p, s_ids, bars, stages, ring,
+                        &k_map, &v_map, l2_evict_first_policy(), abort_flag, lane, &issued_end);
+    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued_end);
+    return;
+  }
+
+  // ---------------- consumer warps ----------------
+  // this lane's query column (lane >> 2): head kvh*G + (col % G) of member col / G
+  uint32_t qb[Geo::MT][2];
+  {
+    const int col = lane >> 2;
+    const int m = s_member[col / G];
+    const __half* qrow =
+        m >= 0 ? p.q + ((size_t)m * p.num_heads + (size_t)kvh * G + col % G) * D : nullptr;
+    load_q_column<D>(qb, qrow, lane);
+  }
+  Acc<D> a;
+  a.reset();
+  bool gave_up = false;
+  for (int c = 0; c < nchunks; ++c) {
+    const int st = c % stages;
+    if (st % NW != warp) continue;
+    if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {
+      gave_up = true;
+      break;
+    }
+    const bool ready = mbar_wait(smem_u32(&bars[st]), (c / stages) & 1);
+    if (!__all_sync(0xffffffffu, ready)) {
+      if (lane == 0) {
+        *abort_flag = 1;
+        flag_error(p.err, ERR_TIMEOUT);
+      }
+      gave_up = true;
+      break;
+    }
+    consume_stage<D>(a, ring + (uint32_t)st * 2 * Geo::TILE_BYTES, min(CHUNK, ntok - c * CHUNK),
+                     qb, p.scale_log2, lane);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars[stages + st]));
+  }
+  if (named_barrier_or(1, NW * 32, gave_up)) return;
+  write_state<D>(a, s_m, s_l, s_o, warp, lane);
+  named_barrier_sync(1, NW * 32);
+  store_columns<D>(
+      s_m, s_l, s_o, p, max_members * G,
+      [&](int c) -> long long {
+        const int m = s_member[c / G];
+        return m < 0 ? -1 : (long long)m * p.num_heads + (long long)kvh * G + c % G;
+      },
+      part, false);
 }
 
 // ---- persistent split-K kernel ---------------------------------------------------
@@ -569,12 +753,16 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   // per-sequence partition counts; the partial tails' chunk-count keys
   for (int k = threadIdx.x; k < TAIL_KEYS; k += blockDim.x) tail_run[k] = 0;
   __syncthreads();
+  // s_lens[b]: the tokens this kernel covers, L minus a shared prefix's tokens
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     int L = p.context_lens[b];
     if (L > p.max_context_len || L <= 0) {
       if (blockIdx.x == 0) flag_error(p.err, ERR_CONTEXT_LEN);
       L = L <= 0 ? 0 : p.max_context_len;
     }
+    bool bad_prefix = false;
+    L -= L > 0 ? prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad_prefix) : 0;
+    if (bad_prefix && blockIdx.x == 0) flag_error(p.err, ERR_PREFIX);
     s_lens[b] = L;
     if (L == 0 && pa.write_zeros && blockIdx.x == 0) {
       for (int i = 0; i < p.num_heads * D; ++i)
@@ -645,6 +833,13 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   }
   __syncthreads();
   const int total = p.num_kv_heads * (pref_f[B] + *s_num_tail);
+  // shared-prefix tokens of sequence b (0 without a prefix), as in the prologue
+  auto prefix_of = [&](int b) -> int {
+    if (!p.seq_prefix_tokens) return 0;
+    const int L = min(p.context_lens[b], p.max_context_len);
+    bool bad = false;
+    return L > 0 ? prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad) : 0;
+  };
 
   if (warp == NW) {
     // ---------------- producer warp ----------------
@@ -693,10 +888,11 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       if (done || !ok) break;
       const int nchunks = (d.w + CHUNK - 1) / CHUNK;
       const int nblk = (d.w + BS - 1) / BS;
-      const int32_t* row = p.block_tables + (size_t)d.x * p.max_blocks + d.z * pt / BS;
-      const int L = s_lens[d.x];
+      const int P = prefix_of(d.x);
+      const int32_t* row = p.block_tables + (size_t)d.x * p.max_blocks + (P + d.z * pt) / BS;
+      const int Ls = s_lens[d.x];
       const int new_tok =
-          (p.k_new && d.z * pt + d.w == L && p.context_lens[d.x] == L) ? d.w - 1 : -1;
+          (p.k_new && d.z * pt + d.w == Ls && p.context_lens[d.x] == P + Ls) ? d.w - 1 : -1;
       if (!produce_item<D, BS>(row, nblk, nchunks, gc, d.y, d.x, new_tok, p, s_ids, bars, stages,
                                ring, &k_map, &v_map, policy, abort_flag, lane, &issued_end))
         break;
@@ -760,7 +956,9 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     if (named_barrier_or(1, NW * 32, stop || gave_up)) break;
     write_state<D>(a, s_m, s_l, s_o, warp, lane);
     named_barrier_sync(1, NW * 32);
-    store_item<D>(s_m, s_l, s_o, p, d.x, d.y, d.z, G, s_lens[d.x] <= pt);
+    const int P = prefix_of(d.x);
+    store_item<D>(s_m, s_l, s_o, p, d.x, d.y, (P + pt - 1) / pt + d.z, G,
+                  P == 0 && s_lens[d.x] <= pt);
   }
   // the merge kernel may be scheduled once every CTA got here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -866,6 +1064,36 @@ cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& km, cons
   PKV_MMA_CASE(128, 16)
   PKV_MMA_CASE(128, 32)
   PKV_MMA_CASE(128, 64)
+  return cudaErrorInvalidValue;
+}
+
+template <int D, int BS>
+cudaError_t launch_prefix_instance(const DecodeParams& p, const CUtensorMap& km,
+                                   const CUtensorMap& vm, int prefix_parts, cudaStream_t stream) {
+  static std::atomic<int> granted[MAX_DEVICES];
+  auto kernel = mma_prefix_kernel<D, BS>;
+  const size_t smem = mma_smem_bytes(D, BS, p.stages);
+  cudaError_t e = allow_smem(kernel, smem, granted);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(p.num_kv_heads, p.num_groups, prefix_parts);
+  kernel<<<grid, (NW + 1) * 32, smem, stream>>>(km, vm, p);
+  return cudaGetLastError();
+}
+
+#define PKV_MMA_PREFIX_CASE(D_, BS_)            \
+  if (p.head_dim == D_ && p.block_size == BS_) \
+    return launch_prefix_instance<D_, BS_>(p, km, vm, prefix_parts, stream);
+
+cudaError_t launch_mma_prefix(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
+                              int prefix_parts, cudaStream_t stream) {
+  PKV_MMA_PREFIX_CASE(64, 8)
+  PKV_MMA_PREFIX_CASE(64, 16)
+  PKV_MMA_PREFIX_CASE(64, 32)
+  PKV_MMA_PREFIX_CASE(64, 64)
+  PKV_MMA_PREFIX_CASE(128, 8)
+  PKV_MMA_PREFIX_CASE(128, 16)
+  PKV_MMA_PREFIX_CASE(128, 32)
+  PKV_MMA_PREFIX_CASE(128, 64)
   return cudaErrorInvalidValue;
 }
 

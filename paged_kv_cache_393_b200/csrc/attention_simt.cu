@@ -105,9 +105,17 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
     }
     return;  // a split launch leaves the zeros to the merge kernel
   }
-  const int tok0 = part * p.part_tokens;            // first token of this partition
+  // With a shared prefix, its group's pass covers tokens [0, P) and this kernel
+  // the suffix [P, L): its partitions start at P, and their partial results go
+  // after the prefix partitions' slots.
+  bool bad_prefix = false;
+  const int P = prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad_prefix);
+  if (bad_prefix && reporter) flag_error(p.err, ERR_PREFIX);
+  const int tok0 = P + part * p.part_tokens;        // first token of this partition
   const int ntok = min(L, tok0 + p.part_tokens) - tok0;
   if (ntok <= 0) return;                            // partition beyond this context
+  const int slot_part = (P + p.part_tokens - 1) / p.part_tokens + part;
+  const bool direct = !SPLIT || (P == 0 && L <= p.part_tokens);
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
   const int blk0 = tok0 / BS;
   const int nblk = (ntok + BS - 1) / BS;
@@ -306,7 +314,7 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (sub == 0) {
     const size_t bh = (size_t)b * p.num_heads + h;
-    if (!SPLIT || L <= p.part_tokens) {
+    if (direct) {
       uint4 packed;
       packed.x = pack_half2(acc[0] / l, acc[1] / l);
       packed.y = pack_half2(acc[2] / l, acc[3] / l);
@@ -314,7 +322,7 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
       packed.w = pack_half2(acc[6] / l, acc[7] / l);
       *reinterpret_cast<uint4*>(p.out + bh * D + col) = packed;
     } else {
-      const size_t slot = bh * p.num_parts + part;
+      const size_t slot = bh * p.num_parts + slot_part;
       float4* dst = reinterpret_cast<float4*>(p.ws_o + slot * D + col);
       dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
       dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);

@@ -21,11 +21,27 @@ constexpr unsigned ERR_CONTEXT_LEN = 2u;
 constexpr unsigned ERR_SLOT = 4u;
 constexpr unsigned ERR_TIMEOUT = 8u;
 constexpr unsigned ERR_INTERNAL = 16u;
+constexpr unsigned ERR_PREFIX = 32u;
 
 constexpr unsigned long long WAIT_TIMEOUT_NS = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ void flag_error(unsigned* err, unsigned bit) {
   if (err) atomicOr(err, bit);
+}
+
+// Tokens of a sequence that its shared-prefix group covers (0 = none): a whole
+// number of blocks that leaves at least the last token to the sequence itself.
+// Any other value is reported through *bad and treated as 0 by every kernel.
+__device__ __forceinline__ int prefix_tokens_of(const int32_t* seq_prefix_tokens, int b, int L,
+                                                int bs, bool* bad) {
+  if (!seq_prefix_tokens) return 0;
+  const int P = seq_prefix_tokens[b];
+  if (P == 0) return 0;
+  if (P < 0 || P % bs != 0 || P > L - 1) {
+    *bad = true;
+    return 0;
+  }
+  return P;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -30,7 +30,18 @@ struct DecodeParams {
   // kernel writes to position L_b - 1 through the block table before reading it.
   const __half* k_new;
   const __half* v_new;
+  // Shared-prefix (cascade) decode (NULL = none).  seq_prefix_tokens[b] tokens of
+  // sequence b are covered by its group's prefix pass; the rest by the suffix
+  // pass.  Partial slots of (b, h): prefix partitions first, then suffix ones.
+  const int32_t* seq_prefix_tokens;  // [B]
+  const int32_t* groups;             // [num_groups][GROUP_WIDTH]: prefix blocks, members
+  int num_groups;
 };
+
+// A shared-prefix group: its prefix length in blocks, then up to 8 member
+// sequences (-1 = unused).
+constexpr int GROUP_WIDTH = 9;
+constexpr int GROUP_MAX_MEMBERS = 8;
 
 // Consumer warps of the grouped-query (tensor-core) kernel; plus one producer warp.
 constexpr int MMA_CONSUMER_WARPS = 2;
@@ -59,6 +70,11 @@ cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMa
                                          bool split, cudaStream_t stream);
 size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs);
 constexpr int PERSISTENT_MAX_SEQS = 1024;
+
+// Shared-prefix pass: CTA = (kv head, group, prefix partition); the members'
+// query rows for that kv head are the columns of one tensor-core tile.
+cudaError_t launch_mma_prefix(const DecodeParams& p, const CUtensorMap& k_map,
+                              const CUtensorMap& v_map, int prefix_parts, cudaStream_t stream);
 
 // Merges the partitions of a split launch into `out` (a programmatic dependent
 // launch after the partition pass on the same stream).

@@ -5,7 +5,9 @@
 //     out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i,   M = max_i m_i,
 // the same online-softmax rescaling the partition kernels use inside a
 // partition.  Contexts that fit in one partition were written by the
-// partition kernel itself and are skipped here.
+// partition kernel itself and are skipped here.  With shared prefixes the
+// slots of a (sequence, head) are its prefix partitions, then the partitions
+// of the rest of its context.
 //
 // One CTA per (sequence, head): warp 0 turns the partition maxima into
 // normalised weights in shared memory, then the threads split into groups
@@ -34,7 +36,11 @@ __global__ void __launch_bounds__(MERGE_THREADS) split_merge_kernel(const Decode
   const int b = blockIdx.y;
   int L = p.context_lens[b];
   if (L > p.max_context_len) L = p.max_context_len;  // flagged by the partition pass
-  const int P = L <= 0 ? 0 : (L + p.part_tokens - 1) / p.part_tokens;
+  // partial slots: a shared prefix's partitions (if any), then the rest of the context's
+  bool bad = false;
+  const int pre = L <= 0 ? 0 : prefix_tokens_of(p.seq_prefix_tokens, b, L, p.block_size, &bad);
+  const int np = (pre + p.part_tokens - 1) / p.part_tokens;
+  const int P = L <= 0 ? 0 : np + (L - pre + p.part_tokens - 1) / p.part_tokens;
   if (P == 1) return;  // written by the partition pass
   __half* out = p.out + ((size_t)b * p.num_heads + h) * D;
   if (P == 0) {

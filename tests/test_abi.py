@@ -104,6 +104,43 @@ def test_fused_append_rejects_bad_arguments_on_the_host(lib, over, code):
     assert _decode_append(lib, b=0, kn=None, q=None) == nat.OK   # empty batch: no-op
 
 
+def _decode_shared(lib, pre=FAKE, groups=FAKE, ng=1, kn=None, vn=None, **over):
+    a = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, cl=FAKE, scale=0.1, bs=16, hk=8, b=4,
+             h=8, d=128, maxblk=8, n=64, maxlen=100, part=0, ws=None, wsb=0)
+    a.update(over)
+    return lib.paged_attention_decode_shared_prefix(
+        a["out"], a["q"], kn, vn, a["kc"], a["vc"], a["bt"], a["cl"], pre, groups, ng, a["scale"],
+        a["bs"], a["hk"], a["b"], a["h"], a["d"], a["maxblk"], a["n"], a["maxlen"], a["part"],
+        a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(pre=None), nat.EINVAL),
+    (dict(groups=None), nat.EINVAL),                  # groups required when num_groups > 0
+    (dict(ng=-1), nat.EINVAL),
+    (dict(ng=70000), nat.EINVAL),
+    (dict(kn=FAKE), nat.EINVAL),                      # k_new without v_new
+    (dict(kn=FAKE + 8, vn=FAKE), nat.EINVAL),         # misaligned
+    (dict(bs=4, maxblk=32), nat.EUNSUPPORTED),        # the prefix pass runs on the tensor cores
+    (dict(h=72, hk=4), nat.EUNSUPPORTED),             # more than 8 query heads per kv head
+    (dict(), nat.EWORKSPACE),                         # always split: needs a workspace
+])
+def test_shared_prefix_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert _decode_shared(lib, **kw) == code
+    assert lib.pagedkv_last_error().decode()
+
+
+def test_shared_prefix_workspace_bytes(lib):
+    # always split at 512 (or the given size), one extra slot per (sequence, head), plus the
+    # tensor-core kernel's work counter for grouped queries
+    f = lib.paged_attention_shared_prefix_workspace_bytes
+    assert f(4, 8, 8, 128, 16, 1200, 0) == 4 * 8 * (3 + 1) * 130 * 4
+    assert f(4, 8, 8, 128, 16, 1200, -1) == 4 * 8 * (3 + 1) * 130 * 4
+    assert f(4, 8, 8, 64, 16, 1200, 256) == 4 * 8 * (5 + 1) * 66 * 4
+    assert f(4, 16, 8, 128, 16, 1200, 0) == 4 * 16 * 4 * 130 * 4 + 16
+    assert f(4, 8, 8, 128, 4, 1200, 0) == 0            # rejected: block_size 4
+
+
 def test_self_test_rejects_bad_timeouts_on_the_host(lib):
     assert lib.pagedkv_selftest_wait_timeout(0, None) == nat.EINVAL
     assert lib.pagedkv_selftest_wait_timeout(1_000_001, None) == nat.EINVAL

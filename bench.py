@@ -57,6 +57,14 @@ def parse_args(argv=None):
                          "group's shared prompt blocks once")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="attention layers per decode step, each with its own pools (a copy of "
+                         "the workload's), run as one CUDA graph (LayeredDecodeStep)")
+    ap.add_argument("--partition-size", type=int, default=None,
+                    help="split-K partition size (default: the workload's)")
+    ap.add_argument("--eager", action="store_true",
+                    help="cow workload: launch every step from Python instead of replaying "
+                         "one CUDA graph per step")
     return ap.parse_args(argv)
 
 
@@ -230,8 +238,10 @@ def run_ours(args):
     w = wl.get(args.workload)
     if w.lens == "cow":
         return run_cow(args, w, dev, world, rank, local)
+    if args.layers > 1:
+        return run_layers(args, w, dev, world, rank, local)
     gb = PagedBatch(w, dev)
-    part = w.partition_size
+    part = w.partition_size if args.partition_size is None else args.partition_size
     B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
     need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, part)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
@@ -374,6 +384,85 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_layers(args, w, dev, world, rank, local):
+    """A decode step over args.layers attention layers (every layer its own pools, here copies
+    of the workload's), each layer's fused append + attention, replayed as one CUDA graph;
+    the same launches issued eagerly from Python are timed too."""
+    import torch
+
+    import paged_kv_cache_393_b200 as pkv
+    from paged_kv_cache_393_b200.batch import PagedBatch
+    gb = PagedBatch(w, dev)
+    Lyr = args.layers
+    pool_bytes = 2 * gb.key_cache.numel() * 2
+    free, _ = torch.cuda.mem_get_info(dev)
+    if pool_bytes * (Lyr - 1) > 0.85 * free:
+        raise SystemExit("%d layers need %.1f GB of pools, %.1f GB free: use fewer layers or a "
+                         "smaller workload" % (Lyr, pool_bytes * Lyr / 1e9, free / 1e9))
+    kcs, vcs = [gb.key_cache], [gb.value_cache]
+    for _ in range(Lyr - 1):
+        kcs.append(gb.key_cache.clone())
+        vcs.append(gb.value_cache.clone())
+    part = w.partition_size if args.partition_size is None else args.partition_size
+    B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
+    stream = torch.cuda.Stream(dev)
+    step = pkv.LayeredDecodeStep(kcs, vcs, B, H, gb.max_blocks, gb.max_context_len, w.scale, part,
+                                 stream=stream)
+    step.set_inputs(q=gb.q.expand(Lyr, -1, -1, -1), k_new=gb.k_new.expand(Lyr, -1, -1, -1),
+                    v_new=gb.v_new.expand(Lyr, -1, -1, -1), block_tables=gb.block_tables,
+                    context_lens=gb.context_lens)
+    need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, part)
+    launches_per_step = Lyr * (1 + (1 if need > 0 else 0))
+
+    def timed(K, fn):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        barrier(world, local)
+        torch.cuda.synchronize(dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(K):
+            fn()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, local)
+        return t0.elapsed_time(t1)
+
+    eager_ms = timed(max(args.steps // 4, 3), step.replay) / max(args.steps // 4, 3)
+    step.capture()
+    pkv.device_errors(clear=True)
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    K = args.steps
+    ms_total = timed(K, step.replay)
+    clocks = sampler.stop()
+    flags = pkv.device_errors(clear=True)
+    if flags:
+        raise SystemExit("device error flags %#x during the timed steps" % flags)
+    kv_bytes = gb.kv_bytes() * Lyr
+    ms_max, kv_all = aggregate(ms_total, float(kv_bytes) * K, world, dev)
+    ms_per_step = ms_max / K
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": round(kv_all / (ms_max / 1e3) / 1e9, 2), "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "accumulate": "f32", "data": "synthetic",
+            "config": {"workload": "%s x %d layers (every layer its own pools), one CUDA graph "
+                                   "per step" % (w.name, Lyr),
+                       "seed": w.seed, "partition_size": part, "layers": Lyr,
+                       "kv_bytes_per_step": kv_bytes, "parallelism": "replicas x%d" % world},
+            "tokens_per_s": round(B * world / (ms_per_step / 1e3), 1),
+            "us_per_layer": round(ms_per_step * 1e3 / Lyr, 2),
+            "eager_ms_per_step": round(eager_ms, 5),
+            "gpu_launches": K * launches_per_step, "clocks": clocks, "e2e": None,
+            "cpu_baseline": None,
+        }), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def run_cow(args, w, dev, world, rank, local):
     """The copy-on-write workload: 32 prompts of 1000 tokens forked into 8 samples,
     then decode steps.  Step 0 copies the 224 shared partial tail blocks
@@ -406,11 +495,13 @@ def run_cow(args, w, dev, world, rank, local):
             st["unique_bytes"] = uniq * wl.kv_bytes_per_token(Hk, D)
         steps.append(st)
     out = torch.empty((B, H, D), dtype=torch.float16, device=dev)
+    cpart = 0 if args.partition_size is None else args.partition_size
     if shared:
         need = pkv.paged_attention_shared_prefix_workspace_bytes(B, H, Hk, D, w.block_size,
-                                                                 gb.max_context_len, 0)
+                                                                 gb.max_context_len, cpart)
     else:
-        need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, 0)
+        need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len,
+                                                   cpart)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
     n_pairs = len(steps_host[0]["pairs"])
@@ -427,17 +518,17 @@ def run_cow(args, w, dev, world, rank, local):
         if shared:
             pkv.paged_attention_decode_shared_prefix(
                 out, st["q"], gb.key_cache, gb.value_cache, st["tables"], st["lens"], st["pre"],
-                st["groups"], w.scale, gb.max_context_len, 0, ws, k_new=st["k"], v_new=st["v"],
+                st["groups"], w.scale, gb.max_context_len, cpart, ws, k_new=st["k"], v_new=st["v"],
                 stream=stream)
         elif args.step == "fused":
             pkv.paged_attention_decode_append(out, st["q"], st["k"], st["v"], gb.key_cache,
                                               gb.value_cache, st["tables"], st["lens"], w.scale,
-                                              gb.max_context_len, 0, ws, stream=stream)
+                                              gb.max_context_len, cpart, ws, stream=stream)
         else:
             pkv.reshape_and_cache(st["k"], st["v"], gb.key_cache, gb.value_cache, st["slots"],
                                   stream=stream)
             pkv.paged_attention_decode(out, st["q"], gb.key_cache, gb.value_cache, st["tables"],
-                                       st["lens"], w.scale, gb.max_context_len, 0, ws,
+                                       st["lens"], w.scale, gb.max_context_len, cpart, ws,
                                        stream=stream)
 
     for j in range(w.decode_steps):   # first pass: the steps in order
@@ -446,29 +537,54 @@ def run_cow(args, w, dev, world, rank, local):
         run_step(j % w.decode_steps)
     torch.cuda.synchronize(dev)
     pkv.device_errors(clear=True)
-    K = args.steps
+    # the copy-on-write step alone, timed with events around eager launches
     copy_ev = []
+    if steps[0]["pairs"] is not None:
+        for _ in range(20):
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[0].record(stream)
+            pkv.copy_blocks([gb.key_cache], [gb.value_cache], steps[0]["pairs"], stream=stream)
+            ev[1].record(stream)
+            copy_ev.append(ev)
+    # One CUDA graph per step (the same launches, replayed without Python in the way)
+    graphs = None
+    if not args.eager:
+        graphs = []
+        for j in range(w.decode_steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                run_step(j)
+            graphs.append(g)
+        torch.cuda.synchronize(dev)
+    K = args.steps
     sampler = ClockSampler(gpu_id_for(local))
     sampler.start()
+
+    def replay(j):
+        if graphs is None:
+            run_step(j)
+        else:
+            with torch.cuda.stream(stream):   # a graph launches on the current stream
+                graphs[j].replay()
+
     for j in range(20):
-        run_step(j % w.decode_steps)
+        replay(j % w.decode_steps)
     barrier(world, local)
     torch.cuda.synchronize(dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     kv_total = 0
     launches = 0
+    h0 = time.perf_counter()
     for i in range(K):
         j = i % w.decode_steps
-        ev = None
         if steps[j]["pairs"] is not None:
-            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            copy_ev.append(ev)
             launches += 1
-        run_step(j, ev)
+        replay(j)
         launches += {"fused": 1, "separate": 2, "shared": 3}[args.step]   # shared: prefix, suffix, merge
         kv_total += steps[j]["kv_bytes"]
         unique_total += steps[j].get("unique_bytes", 0)
+    host_ms = (time.perf_counter() - h0) * 1e3
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world, local)
@@ -491,7 +607,7 @@ def run_cow(args, w, dev, world, rank, local):
                                    "steps replayed in order; K/V bytes counted per sample "
                                    "(shared prefix blocks counted once per reader)" % (
                                        w.prompts, w.prompt_len, w.samples, w.decode_steps),
-                       "seed": w.seed, "step": args.step,
+                       "seed": w.seed, "step": args.step, "partition_size": cpart,
                        "l2": "no flush; shared prefix blocks (%d x 128 KiB x 2) "
                              "can hit in L2" % prefix_blocks,
                        "parallelism": "replicas x%d" % world},
@@ -502,6 +618,8 @@ def run_cow(args, w, dev, world, rank, local):
                             "GB_per_s": round(copy_bytes / (copy_us / 1e6) / 1e9, 1) if copy_us else None,
                             "peak": peak, "peak_kind": peak_kind},
             "gpu_launches": launches, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+            "launch": "eager" if graphs is None else "one CUDA graph per step",
+            "host_issue_ms_per_step": round(host_ms / K, 4),
         }), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -12,7 +12,7 @@ Functions mirror the C names:
     (shared prefixes read once per group), paged_attention_workspace_bytes,
     reshape_and_cache,
     copy_blocks, device_errors, BlockManager (bm_*), decode_step (host buffers
-    in, host result out).
+    in, host result out), LayeredDecodeStep (every layer's decode as one CUDA graph).
 """
 from ._native import (  # noqa: F401
     BlockManager,
@@ -39,3 +39,4 @@ from ._native import (  # noqa: F401
     DEVERR_PREFIX,
     GROUP_WIDTH,
 )
+from .graph import LayeredDecodeStep  # noqa: F401,E402

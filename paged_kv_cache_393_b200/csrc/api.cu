@@ -101,6 +101,7 @@ int encode_pool_map(CUtensorMap* map, const void* pool, int rows, int head_dim, 
 
 constexpr int NUM_SMS_HINT = 148;
 constexpr int AUTO_PARTITION = 512;
+constexpr int SIMT_CTAS_PER_SM = 6;  // resident CUDA-core CTAs per SM at the usual 2-stage ring
 constexpr size_t MAX_SMEM = 227 * 1024;
 
 // Optional overrides of the tuning choices (for sweeps); read once.
@@ -198,13 +199,27 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     p.split = true;
     p.part_tokens = partition_size;
   } else if (partition_size == 0) {
-    const long long ctas = p.mma ? (long long)num_seqs * num_kv_heads
-                                 : (long long)num_seqs * (num_heads / p.hpc);
     const int auto_part = AUTO_PARTITION % align == 0 ? AUTO_PARTITION : align;
-    if (max_context_len > auto_part &&
-        (max_context_len > 4 * auto_part || ctas < 2LL * NUM_SMS_HINT)) {
-      p.split = true;
-      p.part_tokens = auto_part;
+    if (!p.mma) {
+      // CUDA-core kernel: split every context longer than a partition -- smaller, more uniform
+      // CTAs balance the end of the launch (measured faster at 256 and at 32 sequences) -- and
+      // halve the partition (down to 128 tokens) until there are ~4 waves of CTAs.
+      const long long groups = (long long)num_seqs * (num_heads / p.hpc);
+      int pt = auto_part;
+      while (pt > 128 && pt / 2 % align == 0 &&
+             groups * ((max_context_len + pt - 1) / pt) < 4LL * NUM_SMS_HINT * SIMT_CTAS_PER_SM)
+        pt /= 2;
+      if (max_context_len > pt) {
+        p.split = true;
+        p.part_tokens = pt;
+      }
+    } else {
+      const long long ctas = (long long)num_seqs * num_kv_heads;
+      if (max_context_len > auto_part &&
+          (max_context_len > 4 * auto_part || ctas < 2LL * NUM_SMS_HINT)) {
+        p.split = true;
+        p.part_tokens = auto_part;
+      }
     }
   } else if (partition_size != -1) {
     return fail(PAGEDKV_EINVAL, "partition_size %d invalid (-1, 0 or a positive size)",

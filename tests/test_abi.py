@@ -152,8 +152,14 @@ def test_empty_batch_is_a_no_op(lib):
 
 def test_workspace_bytes(lib):
     # single pass: no workspace
-    assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, 0) == 0
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, -1) == 0
+    assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 512, 0) == 0
+    # CUDA-core kernel, automatic: 512-token partitions for the 256-sequence batch, halved to
+    # 128 for 32 sequences (2 kv heads per CTA: 512 CTAs per partition, ~4 waves wanted)
+    assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, 0) == \
+        256 * 32 * 3 * 130 * 4
+    assert pkv.paged_attention_workspace_bytes(32, 32, 32, 128, 16, 1524, 0) == \
+        32 * 32 * 12 * 130 * 4
     # explicit split: B * H * P * (D + 2) floats (CUDA-core kernel, MHA)
     assert pkv.paged_attention_workspace_bytes(4, 8, 8, 64, 16, 1000, 256) == 4 * 8 * 4 * 66 * 4
     # tensor-core split-K runs persistent CTAs fed by a ticket word: 16 more bytes

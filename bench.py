@@ -490,6 +490,8 @@ def run_cow(args, w, dev, world, rank, local):
         if shared:
             pre, groups = pkv.prefix_groups(h["tables"], h["lens"], w.block_size, 8 // (H // Hk))
             st["pre"], st["groups"] = up(pre), up(groups)
+            st["max_prefix"] = int(groups[:, 0].max()) * w.block_size if len(groups) else 0
+            st["max_suffix"] = int((h["lens"] - pre).max())
             # K/V bytes the shared-prefix call reads: each group's prefix once, the rest per sequence
             uniq = int((h["lens"] - pre).astype(np.int64).sum()) + int(groups[:, 0].sum()) * w.block_size
             st["unique_bytes"] = uniq * wl.kv_bytes_per_token(Hk, D)
@@ -519,7 +521,8 @@ def run_cow(args, w, dev, world, rank, local):
             pkv.paged_attention_decode_shared_prefix(
                 out, st["q"], gb.key_cache, gb.value_cache, st["tables"], st["lens"], st["pre"],
                 st["groups"], w.scale, gb.max_context_len, cpart, ws, k_new=st["k"], v_new=st["v"],
-                stream=stream)
+                stream=stream, max_prefix_tokens=st["max_prefix"],
+                max_suffix_tokens=st["max_suffix"])
         elif args.step == "fused":
             pkv.paged_attention_decode_append(out, st["q"], st["k"], st["v"], gb.key_cache,
                                               gb.value_cache, st["tables"], st["lens"], w.scale,

@@ -209,6 +209,13 @@ PAGEDKV_API int paged_attention_decode_append(void *out, const void *q,
  *                  breaking these rules is left out of the prefix pass and sets
  *                  PAGEDKV_DEVERR_PREFIX; its output is then invalid.  May be
  *                  NULL when num_groups is 0.
+ *   max_prefix_tokens, max_suffix_tokens  host upper bounds of the groups' prefix
+ *                  lengths and of L_b - P_b over the batch (0 = max_context_len);
+ *                  they size the launch grids.  A bound below a real length
+ *                  leaves that work undone and sets PAGEDKV_DEVERR_PREFIX.  When
+ *                  max_suffix_tokens fits one partition, the suffix pass folds
+ *                  the prefix partials into every output itself and no merge
+ *                  kernel is launched.
  *   partition_size 0 or -1 = 512 tokens; else as for paged_attention_decode.
  *                  The call always splits.
  *   workspace      at least paged_attention_shared_prefix_workspace_bytes(...).
@@ -226,7 +233,8 @@ PAGEDKV_API int paged_attention_decode_shared_prefix(void *out, const void *q,
                            void *key_cache, void *value_cache,
                            const int32_t *block_tables, const int32_t *context_lens,
                            const int32_t *seq_prefix_tokens, const int32_t *groups,
-                           int num_groups, float scale, int block_size, int num_kv_heads,
+                           int num_groups, int max_prefix_tokens, int max_suffix_tokens,
+                           float scale, int block_size, int num_kv_heads,
                            int num_seqs, int num_heads, int head_dim,
                            int max_blocks_per_seq, int num_blocks, int max_context_len,
                            int partition_size, void *workspace, size_t workspace_bytes,

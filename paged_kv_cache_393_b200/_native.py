@@ -56,7 +56,7 @@ def load_library():
                 [P, P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
             "paged_attention_workspace_bytes": ([I, I, I, I, I, I, I], Z),
             "paged_attention_decode_shared_prefix": (
-                [P, P, P, P, P, P, P, P, P, P, I, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
+                [P, P, P, P, P, P, P, P, P, P, I, I, I, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
             "paged_attention_shared_prefix_workspace_bytes": ([I, I, I, I, I, I, I], Z),
             "pagedkv_prefix_groups": ([P, P, I, I, I, I, P, P, I], I),
             "reshape_and_cache": ([P, P, P, P, P, I, I, I, I, I, P], I),
@@ -203,10 +203,12 @@ def prefix_groups(block_tables, context_lens, block_size, max_members):
 def paged_attention_decode_shared_prefix(out, q, key_cache, value_cache, block_tables,
                                          context_lens, seq_prefix_tokens, groups, scale,
                                          max_context_len, partition_size=0, workspace=None,
-                                         k_new=None, v_new=None, stream=None):
+                                         k_new=None, v_new=None, stream=None,
+                                         max_prefix_tokens=0, max_suffix_tokens=0):
     """Paged decode attention that reads each group's shared prefix once (device tensors:
     seq_prefix_tokens int32 [B], groups int32 [n][GROUP_WIDTH]); with k_new/v_new the new
-    rows are written first, as paged_attention_decode_append does."""
+    rows are written first, as paged_attention_decode_append does.  max_prefix_tokens /
+    max_suffix_tokens: host upper bounds that size the grids (0 = max_context_len)."""
     lib = load_library()
     B, H, D = q.shape
     N, Hk, bs, D2 = key_cache.shape
@@ -239,7 +241,8 @@ def paged_attention_decode_shared_prefix(out, q, key_cache, value_cache, block_t
         _cuda(value_cache, "value_cache", torch.float16, 4),
         _cuda(block_tables, "block_tables", torch.int32, 2),
         _cuda(context_lens, "context_lens", torch.int32, 1),
-        _cuda(seq_prefix_tokens, "seq_prefix_tokens", torch.int32, 1), gptr, ng, float(scale),
+        _cuda(seq_prefix_tokens, "seq_prefix_tokens", torch.int32, 1), gptr, ng,
+        int(max_prefix_tokens), int(max_suffix_tokens), float(scale),
         bs, Hk, B, H, D, block_tables.shape[1], N, int(max_context_len), int(partition_size),
         ws_ptr, ws_bytes, _stream(stream, q.device))
     _check(st, "paged_attention_decode_shared_prefix")

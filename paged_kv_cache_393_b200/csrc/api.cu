@@ -350,13 +350,15 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
            int max_blocks_per_seq, int num_blocks, int max_context_len, int partition_size,
            void* workspace, size_t workspace_bytes, void* stream, bool cascade = false,
            const int32_t* seq_prefix_tokens = nullptr, const int32_t* groups = nullptr,
-           int num_groups = 0) {
+           int num_groups = 0, int max_prefix_tokens = 0, int max_suffix_tokens = 0) {
   if (num_seqs == 0) return PAGEDKV_OK;
   if (cascade) {
     if (!seq_prefix_tokens) return fail(PAGEDKV_EINVAL, "seq_prefix_tokens is required");
     if (num_groups < 0 || num_groups > 65535)
       return fail(PAGEDKV_EINVAL, "num_groups %d outside [0, 65535]", num_groups);
     if (num_groups > 0 && !groups) return fail(PAGEDKV_EINVAL, "groups is NULL");
+    if (max_prefix_tokens < 0 || max_suffix_tokens < 0)
+      return fail(PAGEDKV_EINVAL, "max_prefix_tokens and max_suffix_tokens must be >= 0");
   }
   if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens)
     return fail(PAGEDKV_EINVAL, "a required pointer is NULL");
@@ -409,6 +411,15 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
   p.max_context_len = max_context_len;
   p.part_tokens = plan.part_tokens;
   p.num_parts = plan.num_parts;
+  p.grid_parts = plan.num_parts;
+  if (cascade && max_suffix_tokens > 0) {
+    const int need = (max_suffix_tokens + plan.part_tokens - 1) / plan.part_tokens;
+    if (need < p.grid_parts) p.grid_parts = need;
+  }
+  // With a shared prefix and every suffix within one partition, the partition
+  // pass finishes every output itself: no merge.
+  const bool merged = cascade && max_suffix_tokens > 0 && max_suffix_tokens <= plan.part_tokens;
+  p.no_merge = merged ? 1 : 0;
   p.stages = plan.stages;
   p.k_new = static_cast<const __half*>(k_new);
   p.v_new = static_cast<const __half*>(v_new);
@@ -431,7 +442,12 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
     DecodeParams pp = p;
     pp.stages = plan.prefix_stages;
     pp.k_new = pp.v_new = nullptr;
-    const int prefix_parts = (max_context_len + plan.part_tokens - 1) / plan.part_tokens;
+    pp.no_merge = 0;  // its partial results are always folded in later
+    int prefix_parts = (max_context_len + plan.part_tokens - 1) / plan.part_tokens;
+    if (max_prefix_tokens > 0) {
+      const int need = (max_prefix_tokens + plan.part_tokens - 1) / plan.part_tokens;
+      if (need < prefix_parts) prefix_parts = need;
+    }
     e = launch_mma_prefix(pp, km, vm, prefix_parts, s);
     if (e != cudaSuccess) return cuda_fail(e, "shared-prefix pass launch");
   }
@@ -450,7 +466,7 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
     e = launch_simt_decode(p, plan.hpc, plan.kvc, plan.split, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
-  if (plan.split) {
+  if (plan.split && !merged) {
     e = launch_split_reduce(p, s);
     if (e != cudaSuccess) return cuda_fail(e, "split-K merge launch");
   }
@@ -492,7 +508,8 @@ int paged_attention_decode_append(void* out, const void* q, const void* k_new, c
 int paged_attention_decode_shared_prefix(
     void* out, const void* q, const void* k_new, const void* v_new, void* key_cache,
     void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
-    const int32_t* seq_prefix_tokens, const int32_t* groups, int num_groups, float scale,
+    const int32_t* seq_prefix_tokens, const int32_t* groups, int num_groups,
+    int max_prefix_tokens, int max_suffix_tokens, float scale,
     int block_size, int num_kv_heads, int num_seqs, int num_heads, int head_dim,
     int max_blocks_per_seq, int num_blocks, int max_context_len, int partition_size,
     void* workspace, size_t workspace_bytes, void* stream) {
@@ -504,7 +521,8 @@ int paged_attention_decode_shared_prefix(
   return decode(out, q, k_new, v_new, key_cache, value_cache, block_tables, context_lens, scale,
                 block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq,
                 num_blocks, max_context_len, partition_size, workspace, workspace_bytes, stream,
-                true, seq_prefix_tokens, groups, num_groups);
+                true, seq_prefix_tokens, groups, num_groups, max_prefix_tokens,
+                max_suffix_tokens);
 }
 
 size_t paged_attention_shared_prefix_workspace_bytes(int num_seqs, int num_heads,

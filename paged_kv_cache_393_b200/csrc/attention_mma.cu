@@ -356,8 +356,9 @@ __device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, f
 template <int D, typename ColumnRow>
 __device__ __forceinline__ void store_columns(const float* s_m, const float* s_l, const float* s_o,
                                               const DecodeParams& p, int ncols, ColumnRow row_of,
-                                              int part, bool whole) {
-  // row_of(c): the (sequence * num_heads + head) row of column c, or -1 to skip it
+                                              int part, bool whole, int prefix_slots = 0) {
+  // row_of(c): the (sequence * num_heads + head) row of column c, or -1 to skip it.
+  // prefix_slots > 0 (with whole): fold in that many finished shared-prefix partials first.
   for (int idx = threadIdx.x; idx < ncols * D; idx += NW * 32) {
     const int col = idx / D;
     const int d = idx % D;
@@ -373,9 +374,23 @@ __device__ __forceinline__ void store_columns(const float* s_m, const float* s_l
       num = fmaf(a, s_o[(w * 8 + col) * StageGeom<D>::OSTRIDE + d], num);
       den = fmaf(a, s_l[w * 8 + col], den);
     }
+    if (prefix_slots > 0) {
+      const size_t base = (size_t)bh * p.num_parts;
+      float M2 = M;
+      for (int i = 0; i < prefix_slots; ++i) M2 = fmaxf(M2, p.ws_ml[(base + i) * 2]);
+      const float a = rescale_factor(M, M2);
+      num *= a;
+      den *= a;
+      for (int i = 0; i < prefix_slots; ++i) {
+        const float w = rescale_factor(p.ws_ml[(base + i) * 2], M2);
+        num = fmaf(w, p.ws_o[(base + i) * D + d], num);
+        den = fmaf(w, p.ws_ml[(base + i) * 2 + 1], den);
+      }
+    }
     if (whole) {
       p.out[(size_t)bh * D + d] = __float2half_rn(num / den);
     } else {
+      if (p.no_merge && d == 0) flag_error(p.err, ERR_PREFIX);  // suffix bound too small
       const size_t slot = (size_t)bh * p.num_parts + part;
       p.ws_o[slot * D + d] = num;
       if (d == 0) {
@@ -391,9 +406,10 @@ __device__ __forceinline__ void store_columns(const float* s_m, const float* s_l
 template <int D>
 __device__ __forceinline__ void store_item(const float* s_m, const float* s_l, const float* s_o,
                                            const DecodeParams& p, int b, int kvh, int part, int G,
-                                           bool whole) {
+                                           bool whole, int prefix_slots = 0) {
   const long long row0 = (long long)b * p.num_heads + (long long)kvh * G;
-  store_columns<D>(s_m, s_l, s_o, p, G, [&](int c) { return row0 + c; }, part, whole);
+  store_columns<D>(s_m, s_l, s_o, p, G, [&](int c) { return row0 + c; }, part, whole,
+                   prefix_slots);
 }
 
 // ---- one CTA per (sequence, kv head, partition) ---------------------------------
@@ -431,7 +447,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   }
   if (L <= 0) {
     if (reporter) flag_error(p.err, ERR_CONTEXT_LEN);
-    if (!SPLIT) {
+    if (!SPLIT || p.seq_prefix_tokens) {
       for (int i = threadIdx.x; i < G * D; i += blockDim.x)
         p.out[((size_t)b * p.num_heads + kvh * G) * D + i] = __float2half_rn(0.f);
     }
@@ -442,11 +458,16 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   const int P = prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad_prefix);
   if (bad_prefix && reporter) flag_error(p.err, ERR_PREFIX);
   const int tok0 = P + part * p.part_tokens;
+  if (SPLIT && part == gridDim.z - 1 && tok0 + p.part_tokens < L && threadIdx.x == 0)
+    flag_error(p.err, ERR_PREFIX);  // the grid was sized below this suffix
   const int ntok = min(L, tok0 + p.part_tokens) - tok0;
   if (ntok <= 0) return;
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
   const int nblk = (ntok + BS - 1) / BS;
-  const int slot_part = (P + p.part_tokens - 1) / p.part_tokens + part;
+  const int np = (P + p.part_tokens - 1) / p.part_tokens;  // prefix slots
+  const int slot_part = np + part;
+  // covering a shared prefix's whole suffix: fold in the finished prefix partials here
+  const bool merge_prefix = SPLIT && P > 0 && L - P <= p.part_tokens;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -510,7 +531,8 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   write_state<D>(a, s_m, s_l, s_o, warp, lane);
   named_barrier_sync(1, NW * 32);
-  store_item<D>(s_m, s_l, s_o, p, b, kvh, slot_part, G, !SPLIT || (P == 0 && L <= p.part_tokens));
+  store_item<D>(s_m, s_l, s_o, p, b, kvh, slot_part, G,
+                !SPLIT || (P == 0 && L <= p.part_tokens) || merge_prefix, merge_prefix ? np : 0);
 }
 
 // ---- shared-prefix pass ------------------------------------------------------------
@@ -562,6 +584,8 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   }
   const int P = pblocks * BS;
   const int tok0 = part * p.part_tokens;
+  if (part == gridDim.z - 1 && tok0 + p.part_tokens < P && threadIdx.x == 0 && kvh == 0)
+    flag_error(p.err, ERR_PREFIX);  // the grid was sized below this prefix
   if (tok0 >= P) return;
   const int ntok = min(P, tok0 + p.part_tokens) - tok0;
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
@@ -672,7 +696,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
 
 struct PersistentArgs {
   unsigned int* ticket;  // zeroed before the launch
-  int write_zeros;       // no merge kernel follows: write the zero outputs of empty contexts
+  int write_zeros;       // no merge kernel may follow: write the zero outputs of empty contexts
 };
 
 // Work item of ticket t: every full partition (part_tokens tokens) comes first,
@@ -956,9 +980,11 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     if (named_barrier_or(1, NW * 32, stop || gave_up)) break;
     write_state<D>(a, s_m, s_l, s_o, warp, lane);
     named_barrier_sync(1, NW * 32);
+    // a whole suffix (one item) is finished here, a shared prefix's partials folded in
     const int P = prefix_of(d.x);
-    store_item<D>(s_m, s_l, s_o, p, d.x, d.y, (P + pt - 1) / pt + d.z, G,
-                  P == 0 && s_lens[d.x] <= pt);
+    const int np = (P + pt - 1) / pt;
+    const bool whole = s_lens[d.x] <= pt;
+    store_item<D>(s_m, s_l, s_o, p, d.x, d.y, np + d.z, G, whole, whole ? np : 0);
   }
   // the merge kernel may be scheduled once every CTA got here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -987,7 +1013,7 @@ cudaError_t launch_mma_instance(const DecodeParams& p, const CUtensorMap& km,
   const size_t smem = mma_smem_bytes(D, BS, p.stages);
   cudaError_t e = allow_smem(kernel, smem, granted);
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.num_kv_heads, p.num_seqs, SPLIT ? p.num_parts : 1);
+  const dim3 grid(p.num_kv_heads, p.num_seqs, SPLIT ? p.grid_parts : 1);
   kernel<<<grid, (NW + 1) * 32, smem, stream>>>(km, vm, p);
   return cudaGetLastError();
 }
@@ -1025,7 +1051,7 @@ cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap&
   if (e != cudaSuccess) return e;
   PersistentArgs pa;
   pa.ticket = ticket;
-  pa.write_zeros = split ? 0 : 1;
+  pa.write_zeros = (!split || p.seq_prefix_tokens) ? 1 : 0;
   kernel<<<(unsigned)ctas, (NW + 1) * 32, smem, stream>>>(km, vm, p, pa);
   return cudaGetLastError();
 }

@@ -99,11 +99,11 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
   }
   if (L <= 0) {
     if (reporter) flag_error(p.err, ERR_CONTEXT_LEN);
-    if (!SPLIT && warp < HPC && lane < LPR) {
+    if ((!SPLIT || p.seq_prefix_tokens) && warp < HPC && lane < LPR) {
       *reinterpret_cast<uint4*>(p.out + ((size_t)b * p.num_heads + h0 + warp) * D + lane * 8) =
           make_uint4(0, 0, 0, 0);
     }
-    return;  // a split launch leaves the zeros to the merge kernel
+    return;  // a plain split launch leaves the zeros to the merge kernel
   }
   // With a shared prefix, its group's pass covers tokens [0, P) and this kernel
   // the suffix [P, L): its partitions start at P, and their partial results go
@@ -112,10 +112,17 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
   const int P = prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad_prefix);
   if (bad_prefix && reporter) flag_error(p.err, ERR_PREFIX);
   const int tok0 = P + part * p.part_tokens;        // first token of this partition
+  if (SPLIT && part == gridDim.z - 1 && tok0 + p.part_tokens < L && threadIdx.x == 0)
+    flag_error(p.err, ERR_PREFIX);                  // the grid was sized below this suffix
   const int ntok = min(L, tok0 + p.part_tokens) - tok0;
   if (ntok <= 0) return;                            // partition beyond this context
-  const int slot_part = (P + p.part_tokens - 1) / p.part_tokens + part;
-  const bool direct = !SPLIT || (P == 0 && L <= p.part_tokens);
+  const int np = (P + p.part_tokens - 1) / p.part_tokens;  // prefix slots
+  const int slot_part = np + part;
+  // A CTA that covers a shared prefix's whole suffix finishes the output itself:
+  // the prefix pass ran to completion before this launch, so its partial
+  // results can be folded in here and no merge is needed.
+  const bool merge_prefix = SPLIT && P > 0 && L - P <= p.part_tokens;
+  const bool direct = !SPLIT || (P == 0 && L <= p.part_tokens) || merge_prefix;
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
   const int blk0 = tok0 / BS;
   const int nblk = (ntok + BS - 1) / BS;
@@ -315,6 +322,29 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
   if (sub == 0) {
     const size_t bh = (size_t)b * p.num_heads + h;
     if (direct) {
+      if (merge_prefix) {
+        const float* ml = p.ws_ml + bh * p.num_parts * 2;
+        float M = m;
+        for (int i = 0; i < np; ++i) M = fmaxf(M, ml[2 * i]);
+        const float a = rescale_factor(m, M);
+        l *= a;
+#pragma unroll
+        for (int d = 0; d < 8; ++d) acc[d] *= a;
+        for (int i = 0; i < np; ++i) {
+          const float w = rescale_factor(ml[2 * i], M);
+          const float4* o = reinterpret_cast<const float4*>(p.ws_o + (bh * p.num_parts + i) * D + col);
+          const float4 o0 = o[0], o1 = o[1];
+          l = fmaf(w, ml[2 * i + 1], l);
+          acc[0] = fmaf(w, o0.x, acc[0]);
+          acc[1] = fmaf(w, o0.y, acc[1]);
+          acc[2] = fmaf(w, o0.z, acc[2]);
+          acc[3] = fmaf(w, o0.w, acc[3]);
+          acc[4] = fmaf(w, o1.x, acc[4]);
+          acc[5] = fmaf(w, o1.y, acc[5]);
+          acc[6] = fmaf(w, o1.z, acc[6]);
+          acc[7] = fmaf(w, o1.w, acc[7]);
+        }
+      }
       uint4 packed;
       packed.x = pack_half2(acc[0] / l, acc[1] / l);
       packed.y = pack_half2(acc[2] / l, acc[3] / l);
@@ -322,6 +352,7 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
       packed.w = pack_half2(acc[6] / l, acc[7] / l);
       *reinterpret_cast<uint4*>(p.out + bh * D + col) = packed;
     } else {
+      if (p.no_merge && lane == 0) flag_error(p.err, ERR_PREFIX);  // suffix bound too small
       const size_t slot = bh * p.num_parts + slot_part;
       float4* dst = reinterpret_cast<float4*>(p.ws_o + slot * D + col);
       dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -357,7 +388,7 @@ cudaError_t launch_simt_instance(const DecodeParams& p, cudaStream_t stream) {
   const size_t smem = simt_smem_bytes(D, BS, KVC, p.stages);
   cudaError_t e = allow_smem(kernel, smem, granted);
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.num_heads / HPC, p.num_seqs, SPLIT ? p.num_parts : 1);
+  const dim3 grid(p.num_heads / HPC, p.num_seqs, SPLIT ? p.grid_parts : 1);
   kernel<<<grid, (HPC + 1) * 32, smem, stream>>>(p);
   return cudaGetLastError();
 }

@@ -24,7 +24,9 @@ struct DecodeParams {
   int num_seqs, num_heads, num_kv_heads, head_dim, block_size;
   int max_blocks, num_blocks, max_context_len;
   int part_tokens;             // tokens per partition (a multiple of 16 and of bs)
-  int num_parts;               // partitions per sequence in the grid
+  int num_parts;               // partial-result slots per (sequence, head)
+  int grid_parts;              // partitions in the launch grid (<= num_parts)
+  int no_merge;                // no merge kernel follows: a partial result here is an error
   int stages;                  // depth of the shared-memory ring
   // Fused append (NULL = none): this step's new K/V rows, [B][Hk][D], which the
   // kernel writes to position L_b - 1 through the block table before reading it.

@@ -40,8 +40,9 @@ __global__ void __launch_bounds__(MERGE_THREADS) split_merge_kernel(const Decode
   bool bad = false;
   const int pre = L <= 0 ? 0 : prefix_tokens_of(p.seq_prefix_tokens, b, L, p.block_size, &bad);
   const int np = (pre + p.part_tokens - 1) / p.part_tokens;
-  const int P = L <= 0 ? 0 : np + (L - pre + p.part_tokens - 1) / p.part_tokens;
-  if (P == 1) return;  // written by the partition pass
+  const int ns = L <= 0 ? 0 : (L - pre + p.part_tokens - 1) / p.part_tokens;
+  const int P = np + ns;
+  if (ns == 1) return;  // one partition after any prefix: finished by the partition pass
   __half* out = p.out + ((size_t)b * p.num_heads + h) * D;
   if (P == 0) {
     if (threadIdx.x < V4) *reinterpret_cast<uint2*>(out + threadIdx.x * 4) = make_uint2(0u, 0u);

@@ -109,7 +109,8 @@ def _decode_shared(lib, pre=FAKE, groups=FAKE, ng=1, kn=None, vn=None, **over):
              h=8, d=128, maxblk=8, n=64, maxlen=100, part=0, ws=None, wsb=0)
     a.update(over)
     return lib.paged_attention_decode_shared_prefix(
-        a["out"], a["q"], kn, vn, a["kc"], a["vc"], a["bt"], a["cl"], pre, groups, ng, a["scale"],
+        a["out"], a["q"], kn, vn, a["kc"], a["vc"], a["bt"], a["cl"], pre, groups, ng,
+        a.get("mp", 0), a.get("ms", 0), a["scale"],
         a["bs"], a["hk"], a["b"], a["h"], a["d"], a["maxblk"], a["n"], a["maxlen"], a["part"],
         a["ws"], a["wsb"], None)
 
@@ -119,6 +120,8 @@ def _decode_shared(lib, pre=FAKE, groups=FAKE, ng=1, kn=None, vn=None, **over):
     (dict(groups=None), nat.EINVAL),                  # groups required when num_groups > 0
     (dict(ng=-1), nat.EINVAL),
     (dict(ng=70000), nat.EINVAL),
+    (dict(mp=-1), nat.EINVAL),
+    (dict(ms=-5), nat.EINVAL),
     (dict(kn=FAKE), nat.EINVAL),                      # k_new without v_new
     (dict(kn=FAKE + 8, vn=FAKE), nat.EINVAL),         # misaligned
     (dict(bs=4, maxblk=32), nat.EUNSUPPORTED),        # the prefix pass runs on the tensor cores

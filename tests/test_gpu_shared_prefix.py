@@ -122,8 +122,16 @@ class ForkBatch:
         return ref, kc, vc, relabel
 
 
-def _run(pkv, fb, fused, partition_size=0, sample=None, max_members=None, expect_groups=True):
+def _bounds(fb, pre, groups):
+    """Host upper bounds of the prefix and suffix lengths (they size the grids)."""
+    mp = int(groups[:, 0].max()) * fb.bs if len(groups) else 0
+    return mp, int((fb.lens_host - pre).max())
+
+
+def _run(pkv, fb, fused, partition_size=0, sample=None, max_members=None, expect_groups=True,
+         bounds=True):
     pre, groups = fb.groups(max_members)
+    mp, ms = _bounds(fb, pre, groups) if bounds else (0, 0)
     if expect_groups:
         assert len(groups) > 0
     pre_d = torch.from_numpy(pre).to(DEV)
@@ -134,7 +142,7 @@ def _run(pkv, fb, fused, partition_size=0, sample=None, max_members=None, expect
     pkv.paged_attention_decode_shared_prefix(
         fb.out, fb.q, fb.kc, fb.vc, fb.tables, fb.lens, pre_d, groups_d, 1.0 / fb.D ** 0.5,
         fb.max_context_len, partition_size, k_new=fb.k_new if fused else None,
-        v_new=fb.v_new if fused else None)
+        v_new=fb.v_new if fused else None, max_prefix_tokens=mp, max_suffix_tokens=ms)
     torch.cuda.synchronize()
     assert pkv.device_errors() == 0
     sample = list(range(len(fb.seqs))) if sample is None else sample
@@ -169,7 +177,22 @@ CASES = [
 def test_forked_batches(pkv, case, fused):
     name, H, Hk, D, bs, prompts, samples, extra, part = case
     fb = ForkBatch(pkv, H, Hk, D, bs, prompts, samples, extra)
-    _run(pkv, fb, fused, part, expect_groups=samples > 1 and H // Hk < 8)
+    # the separate runs size the grids from max_context_len, the fused ones from host bounds
+    _run(pkv, fb, fused, part, expect_groups=samples > 1 and H // Hk < 8, bounds=fused)
+
+
+@pytest.mark.parametrize("H,Hk", [(8, 8), (8, 2)], ids=["mha", "gqa"])
+def test_bounds_below_the_real_lengths_are_flagged(pkv, H, Hk):
+    fb = ForkBatch(pkv, H, Hk, 128, 16, [1000, 300], 4, lambda i: 100 * i)
+    pre, groups = fb.groups()
+    mp, ms = _bounds(fb, pre, groups)
+    fb.write_new_tokens()
+    for bad in ((mp - 512, ms), (mp, 16)):           # one partition short
+        pkv.paged_attention_decode_shared_prefix(
+            fb.out, fb.q, fb.kc, fb.vc, fb.tables, fb.lens, torch.from_numpy(pre).to(DEV),
+            torch.from_numpy(groups).to(DEV), 1.0 / fb.D ** 0.5, fb.max_context_len, 64,
+            max_prefix_tokens=bad[0], max_suffix_tokens=bad[1])
+        assert pkv.device_errors() & pkv.DEVERR_PREFIX
 
 
 def test_more_sequences_than_the_persistent_grid(pkv):
@@ -236,6 +259,7 @@ def test_cow_workload_shared_prefix(pkv):
         assert host["pairs"].tolist() == [list(x) for x in model.take_copies()]
         pre, groups = pkv.prefix_groups(host["tables"], host["lens"], bs, 8)
         assert len(groups) == w.prompts and (pre == 992).all()
+        mp, ms = 992, int((host["lens"] - pre).max())
         dev = {k: torch.from_numpy(host[k]).to(DEV) for k in ("tables", "lens", "q", "k", "v")}
         if len(host["pairs"]):
             pkv.copy_blocks([gb.key_cache], [gb.value_cache], torch.from_numpy(host["pairs"]).to(DEV))
@@ -243,7 +267,8 @@ def test_cow_workload_shared_prefix(pkv):
         pkv.paged_attention_decode_shared_prefix(
             out, dev["q"], gb.key_cache, gb.value_cache, dev["tables"], dev["lens"],
             torch.from_numpy(pre).to(DEV), torch.from_numpy(groups).to(DEV), w.scale,
-            gb.max_context_len, k_new=dev["k"], v_new=dev["v"])
+            gb.max_context_len, k_new=dev["k"], v_new=dev["v"], max_prefix_tokens=mp,
+            max_suffix_tokens=ms)
         news.append((host["k"], host["v"]))
     torch.cuda.synchronize()
     assert pkv.device_errors() == 0

@@ -437,8 +437,24 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
     st = encode_pool_map(&vm, value_cache, rows, head_dim, block_size);
     if (st != PAGEDKV_OK) return st;
   }
-  if (cascade && num_groups > 0) {
-    // prefix pass first; the suffix pass and the merge follow in stream order
+  unsigned int* ticket = nullptr;  // the persistent kernel's work counter
+  if (plan.mma && plan.persistent) {
+    const size_t parts_bytes =
+        plan.split ? (size_t)num_seqs * num_heads * plan.num_parts * (head_dim + 2) * sizeof(float)
+                   : 0;
+    ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
+                                             ((parts_bytes + 15) / 16) * 16);
+  }
+  const bool prefix_pass = cascade && num_groups > 0;
+  if (prefix_pass) {
+    // Prefix pass first.  The suffix pass is its programmatic dependent: it may
+    // start on the SMs the prefix pass frees and waits for it only before it
+    // reads the prefix partials; the merge follows the suffix pass.  The work
+    // counter is zeroed before the prefix pass so nothing sits between the two.
+    if (ticket) {
+      e = cudaMemsetAsync(ticket, 0, sizeof(unsigned int), s);
+      if (e != cudaSuccess) return cuda_fail(e, "work counter reset");
+    }
     DecodeParams pp = p;
     pp.stages = plan.prefix_stages;
     pp.k_new = pp.v_new = nullptr;
@@ -450,15 +466,11 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
     }
     e = launch_mma_prefix(pp, km, vm, prefix_parts, s);
     if (e != cudaSuccess) return cuda_fail(e, "shared-prefix pass launch");
+    p.after_prefix = 1;
   }
   if (plan.mma) {
     if (plan.persistent) {
-      const size_t parts_bytes =
-          plan.split ? (size_t)num_seqs * num_heads * plan.num_parts * (head_dim + 2) * sizeof(float)
-                     : 0;
-      unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
-                                                             ((parts_bytes + 15) / 16) * 16);
-      e = launch_mma_decode_persistent(p, km, vm, ticket, plan.split, s);
+      e = launch_mma_decode_persistent(p, km, vm, ticket, plan.split, s, prefix_pass);
     } else {
       e = launch_mma_decode(p, km, vm, plan.split, s);
     }

@@ -531,6 +531,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   write_state<D>(a, s_m, s_l, s_o, warp, lane);
   named_barrier_sync(1, NW * 32);
+  if (p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");  // prefix partials ready
   store_item<D>(s_m, s_l, s_o, p, b, kvh, slot_part, G,
                 !SPLIT || (P == 0 && L <= p.part_tokens) || merge_prefix, merge_prefix ? np : 0);
 }
@@ -569,6 +570,9 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   float* s_l = s_m + NW * 8;
   float* s_o = s_l + NW * 8;
 
+  // the suffix pass may start on the SMs this grid frees; it waits for this grid
+  // before it reads the partial results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int kvh = blockIdx.x;
@@ -981,6 +985,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     write_state<D>(a, s_m, s_l, s_o, warp, lane);
     named_barrier_sync(1, NW * 32);
     // a whole suffix (one item) is finished here, a shared prefix's partials folded in
+    if (p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");  // prefix partials ready
     const int P = prefix_of(d.x);
     const int np = (P + pt - 1) / pt;
     const bool whole = s_lens[d.x] <= pt;
@@ -1014,14 +1019,14 @@ cudaError_t launch_mma_instance(const DecodeParams& p, const CUtensorMap& km,
   cudaError_t e = allow_smem(kernel, smem, granted);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.num_kv_heads, p.num_seqs, SPLIT ? p.grid_parts : 1);
-  kernel<<<grid, (NW + 1) * 32, smem, stream>>>(km, vm, p);
-  return cudaGetLastError();
+  return launch_kernel(p.after_prefix != 0, kernel, grid, dim3((NW + 1) * 32), smem, stream, km,
+                       vm, p);
 }
 
 template <int D, int BS>
 cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap& km,
                                        const CUtensorMap& vm, unsigned int* ticket, bool split,
-                                       cudaStream_t stream) {
+                                       cudaStream_t stream, bool ticket_zeroed) {
   static std::atomic<int> granted[MAX_DEVICES];
   static std::atomic<int> blocks_per_sm[MAX_DEVICES];
   static std::atomic<int> blocks_smem[MAX_DEVICES];
@@ -1047,13 +1052,15 @@ cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap&
   const long long items = (long long)p.num_kv_heads * p.num_seqs * p.num_parts;
   long long ctas = (long long)sms * blocks_per_sm[dev].load(std::memory_order_relaxed);
   if (ctas > items) ctas = items;
-  e = cudaMemsetAsync(ticket, 0, sizeof(unsigned int), stream);
-  if (e != cudaSuccess) return e;
+  if (!ticket_zeroed) {
+    e = cudaMemsetAsync(ticket, 0, sizeof(unsigned int), stream);
+    if (e != cudaSuccess) return e;
+  }
   PersistentArgs pa;
   pa.ticket = ticket;
   pa.write_zeros = (!split || p.seq_prefix_tokens) ? 1 : 0;
-  kernel<<<(unsigned)ctas, (NW + 1) * 32, smem, stream>>>(km, vm, p, pa);
-  return cudaGetLastError();
+  return launch_kernel(p.after_prefix != 0, kernel, dim3((unsigned)ctas), dim3((NW + 1) * 32),
+                       smem, stream, km, vm, p, pa);
 }
 
 }  // namespace
@@ -1125,11 +1132,11 @@ cudaError_t launch_mma_prefix(const DecodeParams& p, const CUtensorMap& km, cons
 
 #define PKV_MMA_PERSISTENT_CASE(D_, BS_)        \
   if (p.head_dim == D_ && p.block_size == BS_) \
-    return launch_persistent_instance<D_, BS_>(p, km, vm, ticket, split, stream);
+    return launch_persistent_instance<D_, BS_>(p, km, vm, ticket, split, stream, ticket_zeroed);
 
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& km,
                                          const CUtensorMap& vm, unsigned int* ticket, bool split,
-                                         cudaStream_t stream) {
+                                         cudaStream_t stream, bool ticket_zeroed) {
   PKV_MMA_PERSISTENT_CASE(64, 8)
   PKV_MMA_PERSISTENT_CASE(64, 16)
   PKV_MMA_PERSISTENT_CASE(64, 32)

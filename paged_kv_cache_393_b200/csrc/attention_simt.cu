@@ -319,6 +319,9 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
   }
   // the merge kernel (if any) may be scheduled once every CTA got here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the shared-prefix pass this launch may overlap must be done before its
+  // partials are read below (and before this grid counts as complete)
+  if (p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");
   if (sub == 0) {
     const size_t bh = (size_t)b * p.num_heads + h;
     if (direct) {
@@ -389,8 +392,7 @@ cudaError_t launch_simt_instance(const DecodeParams& p, cudaStream_t stream) {
   cudaError_t e = allow_smem(kernel, smem, granted);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.num_heads / HPC, p.num_seqs, SPLIT ? p.grid_parts : 1);
-  kernel<<<grid, (HPC + 1) * 32, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(p.after_prefix != 0, kernel, grid, dim3((HPC + 1) * 32), smem, stream, p);
 }
 
 }  // namespace

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace pkv {
 
 // Arguments of one paged decode-attention launch (both passes of split-K).
@@ -27,6 +29,8 @@ struct DecodeParams {
   int num_parts;               // partial-result slots per (sequence, head)
   int grid_parts;              // partitions in the launch grid (<= num_parts)
   int no_merge;                // no merge kernel follows: a partial result here is an error
+  int after_prefix;            // launched as a programmatic dependent of the shared-prefix pass:
+                               // wait for it (griddepcontrol.wait) before reading its partials
   int stages;                  // depth of the shared-memory ring
   // Fused append (NULL = none): this step's new K/V rows, [B][Hk][D], which the
   // kernel writes to position L_b - 1 through the block table before reading it.
@@ -44,6 +48,24 @@ struct DecodeParams {
 // sequences (-1 = unused).
 constexpr int GROUP_WIDTH = 9;
 constexpr int GROUP_MAX_MEMBERS = 8;
+
+// kernel<<<grid, block, smem, stream>>>(args...), as a programmatic dependent launch
+// (it may start while the previous kernel on the stream finishes) when pdl is set.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                                 size_t smem, cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Consumer warps of the grouped-query (tensor-core) kernel; plus one producer warp.
 constexpr int MMA_CONSUMER_WARPS = 2;
@@ -67,9 +89,11 @@ cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& k_map,
 // Persistent tensor-core kernel: a few CTAs per SM take (b, kv head, partition)
 // work items from `ticket` (a workspace word it zeroes first).  Without a
 // split every item is a whole context.
+// ticket_zeroed: the caller already zeroed the work counter on this stream.
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& k_map,
                                          const CUtensorMap& v_map, unsigned int* ticket,
-                                         bool split, cudaStream_t stream);
+                                         bool split, cudaStream_t stream,
+                                         bool ticket_zeroed = false);
 size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs);
 constexpr int PERSISTENT_MAX_SEQS = 1024;
 

@@ -350,28 +350,37 @@ __device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, f
   }
 }
 
-// Merges the consumer warps' states of item (b, kvh, part) and stores the result:
-// the fp16 output when the item is the whole context, else the partition's
-// (max, sum, unnormalised output) for the merge kernel.
+// Merges the consumer warps' states of an item's columns and stores the result:
+// the fp16 output when the item covers the whole context, else the partition's
+// (max, sum, unnormalised output) for the merge.
 template <int D, typename ColumnRow>
 __device__ __forceinline__ void store_columns(const float* s_m, const float* s_l, const float* s_o,
                                               const DecodeParams& p, int ncols, ColumnRow row_of,
                                               int part, bool whole, int prefix_slots = 0) {
   // row_of(c): the (sequence * num_heads + head) row of column c, or -1 to skip it.
   // prefix_slots > 0 (with whole): fold in that many finished shared-prefix partials first.
-  for (int idx = threadIdx.x; idx < ncols * D; idx += NW * 32) {
-    const int col = idx / D;
-    const int d = idx % D;
+  // Each thread takes 4 consecutive dims of one column.
+  constexpr int PER_COL = D / 4;
+  using Geo = StageGeom<D>;
+  if (!whole && p.no_merge && threadIdx.x == 0) flag_error(p.err, ERR_PREFIX);  // bound too small
+  for (int idx = threadIdx.x; idx < ncols * PER_COL; idx += NW * 32) {
+    const int col = idx / PER_COL;
+    const int d0 = (idx % PER_COL) * 4;
     const long long bh = row_of(col);
     if (bh < 0) continue;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * 8 + col]);
-    float num = 0.f, den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const float a = rescale_factor(s_m[w * 8 + col], M);
-      num = fmaf(a, s_o[(w * 8 + col) * StageGeom<D>::OSTRIDE + d], num);
+      const float4 o = *reinterpret_cast<const float4*>(s_o + (w * 8 + col) * Geo::OSTRIDE + d0);
+      num.x = fmaf(a, o.x, num.x);
+      num.y = fmaf(a, o.y, num.y);
+      num.z = fmaf(a, o.z, num.z);
+      num.w = fmaf(a, o.w, num.w);
       den = fmaf(a, s_l[w * 8 + col], den);
     }
     if (prefix_slots > 0) {
@@ -379,21 +388,29 @@ __device__ __forceinline__ void store_columns(const float* s_m, const float* s_l
       float M2 = M;
       for (int i = 0; i < prefix_slots; ++i) M2 = fmaxf(M2, p.ws_ml[(base + i) * 2]);
       const float a = rescale_factor(M, M2);
-      num *= a;
+      num.x *= a;
+      num.y *= a;
+      num.z *= a;
+      num.w *= a;
       den *= a;
       for (int i = 0; i < prefix_slots; ++i) {
         const float w = rescale_factor(p.ws_ml[(base + i) * 2], M2);
-        num = fmaf(w, p.ws_o[(base + i) * D + d], num);
+        const float4 o = *reinterpret_cast<const float4*>(p.ws_o + (base + i) * D + d0);
+        num.x = fmaf(w, o.x, num.x);
+        num.y = fmaf(w, o.y, num.y);
+        num.z = fmaf(w, o.z, num.z);
+        num.w = fmaf(w, o.w, num.w);
         den = fmaf(w, p.ws_ml[(base + i) * 2 + 1], den);
       }
     }
     if (whole) {
-      p.out[(size_t)bh * D + d] = __float2half_rn(num / den);
+      const float inv = 1.f / den;
+      *reinterpret_cast<uint2*>(p.out + (size_t)bh * D + d0) =
+          make_uint2(pack_half2(num.x * inv, num.y * inv), pack_half2(num.z * inv, num.w * inv));
     } else {
-      if (p.no_merge && d == 0) flag_error(p.err, ERR_PREFIX);  // suffix bound too small
       const size_t slot = (size_t)bh * p.num_parts + part;
-      p.ws_o[slot * D + d] = num;
-      if (d == 0) {
+      *reinterpret_cast<float4*>(p.ws_o + slot * D + d0) = num;
+      if (d0 == 0) {
         p.ws_ml[slot * 2] = M;
         p.ws_ml[slot * 2 + 1] = den;
       }

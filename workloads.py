@@ -88,6 +88,9 @@ WORKLOADS = {
                           partition_size=512),
     "cow": Workload("cow", 256, 32, 32, 128, 16, 32768, 1004, "cow",
                     prompts=32, prompt_len=1000, samples=8, decode_steps=200),
+    # an 8-prompt cut of cow (64 samples) for profiler captures of the shared-prefix pass
+    "cow_small": Workload("cow_small", 64, 32, 32, 128, 16, 8192, 1004, "cow",
+                          prompts=8, prompt_len=1000, samples=8, decode_steps=200),
     "gqa": Workload("gqa", 128, 64, 8, 128, 16, 131072, 1005, "lognormal",
                     lognormal_median=1024.0, lognormal_sigma=1.0, len_lo=64, len_hi=16384,
                     partition_size=512),

@@ -313,7 +313,9 @@ def run_ours(args):
     if fused:
         attn_bytes += 2 * B * Hk * D * 2 * 2    # new K/V rows read and written
     if splits:
-        parts = (gb.lens_host + part - 1) // part
+        pt = pkv.paged_attention_partition_tokens(B, H, Hk, D, w.block_size, gb.max_context_len,
+                                                  part)
+        parts = (gb.lens_host + pt - 1) // pt
         attn_bytes += int(parts.sum()) * H * (D + 2) * 4 * 2    # partials written + read
     peak, peak_kind = hbm_peak()
     achieved = attn_bytes / (attn_ms / 1e3) / 1e9

@@ -268,6 +268,13 @@ PAGEDKV_API int pagedkv_prefix_groups(const int32_t *block_tables, const int32_t
                            int max_members, int32_t *seq_prefix_tokens, int32_t *groups,
                            int groups_capacity);
 
+/* The partition size paged_attention_decode uses for these arguments: the tokens
+ * per split-K partition, 0 for a single pass (partition_size 0 lets the library
+ * choose), or a negative PAGEDKV_E* code for arguments it would reject. */
+PAGEDKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_dim, int block_size, int max_context_len,
+                                       int partition_size);
+
 /* ---- allocation-free decode ------------------------------------------------------
  *
  * The pages have no counterpart of this call; it serves callers that cannot

@@ -26,6 +26,7 @@ from ._native import (  # noqa: F401
     paged_attention_decode,
     paged_attention_decode_append,
     paged_attention_decode_shared_prefix,
+    paged_attention_partition_tokens,
     paged_attention_shared_prefix_workspace_bytes,
     paged_attention_workspace_bytes,
     prefix_groups,

@@ -55,6 +55,7 @@ def load_library():
             "paged_attention_decode_append": (
                 [P, P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
             "paged_attention_workspace_bytes": ([I, I, I, I, I, I, I], Z),
+            "paged_attention_partition_tokens": ([I, I, I, I, I, I, I], I),
             "paged_attention_decode_shared_prefix": (
                 [P, P, P, P, P, P, P, P, P, P, I, I, I, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
             "paged_attention_shared_prefix_workspace_bytes": ([I, I, I, I, I, I, I], Z),
@@ -120,6 +121,14 @@ def paged_attention_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
                                     max_context_len, partition_size=0) -> int:
     return int(load_library().paged_attention_workspace_bytes(
         num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size))
+
+
+def paged_attention_partition_tokens(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                     max_context_len, partition_size=0) -> int:
+    """Tokens per split-K partition the library uses (0 = single pass)."""
+    n = load_library().paged_attention_partition_tokens(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size)
+    return _check(n, "paged_attention_partition_tokens")
 
 
 def paged_attention_decode(out, q, key_cache, value_cache, block_tables, context_lens, scale,

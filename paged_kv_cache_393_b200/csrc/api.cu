@@ -337,6 +337,15 @@ size_t paged_attention_workspace_bytes(int num_seqs, int num_heads, int num_kv_h
   return plan.ws_bytes;
 }
 
+int paged_attention_partition_tokens(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                     int block_size, int max_context_len, int partition_size) {
+  Plan plan;
+  const int st = make_plan(&plan, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                           max_context_len, partition_size);
+  if (st != PAGEDKV_OK) return st;
+  return plan.split ? plan.part_tokens : 0;
+}
+
 }  // extern "C"
 
 namespace pkv {

@@ -178,6 +178,16 @@ def test_workspace_bytes(lib):
     assert pkv.paged_attention_workspace_bytes(1, 8, 3, 64, 16, 100, 0) == 0     # rejected shape
 
 
+def test_partition_tokens(lib):
+    f = pkv.paged_attention_partition_tokens
+    assert f(256, 32, 32, 128, 16, 1524, -1) == 0          # single pass asked for
+    assert f(256, 32, 32, 128, 16, 1524, 0) == 512         # automatic split
+    assert f(32, 32, 32, 128, 16, 1524, 0) == 128          # small batch: smaller partitions
+    assert f(128, 64, 8, 128, 16, 16384, 0) == 512         # long grouped-query contexts
+    assert f(256, 32, 32, 128, 16, 1524, 256) == 256
+    assert lib.paged_attention_partition_tokens(1, 8, 3, 64, 16, 100, 0) == nat.EINVAL
+
+
 def test_cache_ops_reject_bad_arguments_on_the_host(lib):
     assert lib.reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 64, 16, 8, None) == nat.OK
     assert lib.reshape_and_cache(None, FAKE, FAKE, FAKE, FAKE, 3, 4, 64, 16, 8, None) == nat.EINVAL

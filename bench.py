@@ -601,6 +601,44 @@ def run_cow(args, w, dev, world, rank, local):
     ms_per_step = ms_max / K
     copy_us = (sum(a.elapsed_time(b) for a, b in copy_ev) / len(copy_ev) * 1e3) if copy_ev else None
     prefix_blocks = w.prompts * (w.prompt_len // w.block_size)
+
+    # end to end through DecodeSession (host buffers in, host output back), the steps in order
+    # from the start (copy-on-write pairs at step 0); the host grouping of the shared-prefix
+    # step is inside the timed region
+    e2e = None
+    E = min(args.e2e_steps, w.decode_steps, 50)
+    if E > 0:
+        sess = pkv.DecodeSession(gb.key_cache, gb.value_cache, B, H, gb.max_blocks,
+                                 gb.max_context_len, cpart, max_pairs=max(n_pairs, 1),
+                                 fused=args.step != "separate", shared_prefix=shared)
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+        hs = [{k: pin(steps_host[j][k]) for k in ("q", "k", "v", "slots", "tables", "lens")}
+              for j in range(E)]
+        hpairs = pin(steps_host[0]["pairs"]) if n_pairs else None
+        hout = torch.empty((B, H, D), dtype=torch.float16).pin_memory()
+
+        def e2e_step(j):
+            h = hs[j]
+            sess.step(h["q"], h["k"], h["v"], h["slots"], h["tables"], h["lens"], hout,
+                      pairs=hpairs if j == 0 else None, stream=stream)
+
+        for j in range(min(3, E)):
+            e2e_step(j)
+        torch.cuda.synchronize(dev)
+        barrier(world, local)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        h2d = 0
+        for j in range(E):
+            e2e_step(j)
+            h2d += sess.h2d_bytes(n_pairs if j == 0 else 0)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms, e_bytes = aggregate(e0.elapsed_time(e1),
+                                  float(sum(steps[j]["kv_bytes"] for j in range(E))), world, dev)
+        e2e = {"value": round(e_bytes / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
+               "ms_per_step": round(e_ms / E, 4), "steps": E,
+               "h2d_bytes_per_step": int(h2d / E), "d2h_bytes_per_step": sess.d2h_bytes()}
     if rank == 0:
         peak, peak_kind = hbm_peak()
         print(json.dumps({
@@ -622,7 +660,7 @@ def run_cow(args, w, dev, world, rank, local):
             "copy_blocks": {"pairs": n_pairs, "bytes": copy_bytes, "avg_us": copy_us,
                             "GB_per_s": round(copy_bytes / (copy_us / 1e6) / 1e9, 1) if copy_us else None,
                             "peak": peak, "peak_kind": peak_kind},
-            "gpu_launches": launches, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+            "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "cpu_baseline": None,
             "launch": "eager" if graphs is None else "one CUDA graph per step",
             "host_issue_ms_per_step": round(host_ms / K, 4),
         }), flush=True)

@@ -324,17 +324,23 @@ class DecodeSession:
     copy-on-write pairs, then either reshape_and_cache for the new tokens and
     paged_attention_decode, or (fused=True) paged_attention_decode_append, which
     writes the new tokens at position L-1 through the tables itself and needs no
-    slots; finally it copies the output back into a host tensor.
+    slots, or (shared_prefix=True, fused as well) groups the batch by shared table
+    prefixes on the host (prefix_groups) and calls
+    paged_attention_decode_shared_prefix; finally it copies the output back into a
+    host tensor.
     """
 
     def __init__(self, key_cache, value_cache, num_seqs, num_heads, max_blocks, max_context_len,
-                 partition_size=0, max_pairs=0, fused=False):
+                 partition_size=0, max_pairs=0, fused=False, shared_prefix=False):
         dev = key_cache.device
         N, Hk, bs, D = key_cache.shape
         self.key_cache, self.value_cache = key_cache, value_cache
         self.max_context_len = int(max_context_len)
         self.partition_size = partition_size
-        self.fused = bool(fused)
+        self.shared_prefix = bool(shared_prefix)
+        self.fused = bool(fused) or self.shared_prefix
+        self.block_size = bs
+        self.max_members = max(1, 8 // (num_heads // Hk))
         self.q = torch.empty((num_seqs, num_heads, D), dtype=torch.float16, device=dev)
         self.k = torch.empty((num_seqs, Hk, D), dtype=torch.float16, device=dev)
         self.v = torch.empty_like(self.k)
@@ -343,13 +349,24 @@ class DecodeSession:
         self.lens = torch.empty(num_seqs, dtype=torch.int32, device=dev)
         self.out = torch.empty((num_seqs, num_heads, D), dtype=torch.float16, device=dev)
         self.pairs = torch.empty((max(max_pairs, 1), 2), dtype=torch.int64, device=dev)
-        need = paged_attention_workspace_bytes(num_seqs, num_heads, Hk, D, bs, max_context_len,
-                                               partition_size)
+        if self.shared_prefix:
+            self.prefix = torch.zeros(num_seqs, dtype=torch.int32, device=dev)
+            self.groups = torch.zeros((max(num_seqs // 2, 1), GROUP_WIDTH), dtype=torch.int32,
+                                      device=dev)
+            need = paged_attention_shared_prefix_workspace_bytes(num_seqs, num_heads, Hk, D, bs,
+                                                                 max_context_len, partition_size)
+        else:
+            need = paged_attention_workspace_bytes(num_seqs, num_heads, Hk, D, bs,
+                                                   max_context_len, partition_size)
         self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self._last_groups = 0
 
     def h2d_bytes(self, num_pairs=0) -> int:
         ts = (self.q, self.k, self.v, self.tables, self.lens) + (() if self.fused else (self.slots,))
-        return sum(t.numel() * t.element_size() for t in ts) + num_pairs * 16
+        n = sum(t.numel() * t.element_size() for t in ts) + num_pairs * 16
+        if self.shared_prefix:   # prefix lengths and the step's groups
+            n += self.prefix.numel() * 4 + self._last_groups * GROUP_WIDTH * 4
+        return n
 
     def d2h_bytes(self) -> int:
         return self.out.numel() * self.out.element_size()
@@ -370,7 +387,23 @@ class DecodeSession:
                 n = pairs.shape[0]
                 self.pairs[:n].copy_(pairs, non_blocking=True)
                 copy_blocks([self.key_cache], [self.value_cache], self.pairs[:n], stream=s)
-            if self.fused:
+            if self.shared_prefix:
+                t_host = tables.numpy() if isinstance(tables, torch.Tensor) else np.asarray(tables)
+                l_host = lens.numpy() if isinstance(lens, torch.Tensor) else np.asarray(lens)
+                pre, groups = prefix_groups(t_host, l_host, self.block_size, self.max_members)
+                n = groups.shape[0]
+                self._last_groups = n
+                self.prefix.copy_(torch.from_numpy(pre), non_blocking=False)
+                if n:
+                    self.groups[:n].copy_(torch.from_numpy(groups), non_blocking=False)
+                max_prefix = int(groups[:, 0].max()) * self.block_size if n else 0
+                max_suffix = int((l_host - pre).max()) if len(l_host) else 0
+                paged_attention_decode_shared_prefix(
+                    self.out, self.q, self.key_cache, self.value_cache, self.tables, self.lens,
+                    self.prefix, self.groups[:n], scale, self.max_context_len,
+                    self.partition_size, self.workspace, k_new=self.k, v_new=self.v, stream=s,
+                    max_prefix_tokens=max_prefix, max_suffix_tokens=max_suffix)
+            elif self.fused:
                 paged_attention_decode_append(self.out, self.q, self.k, self.v, self.key_cache,
                                               self.value_cache, self.tables, self.lens, scale,
                                               self.max_context_len, self.partition_size,

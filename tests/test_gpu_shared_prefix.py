@@ -286,3 +286,24 @@ def test_cow_workload_shared_prefix(pkv):
     ref = oracle.paged_attention(host["q"][chosen], kc_o, vc_o, t_o, l_o, w.scale, bs, Hk,
                                  nthreads=8)
     assert_attention_close(out.cpu().numpy()[chosen], ref)
+
+
+@pytest.mark.parametrize("H,Hk", [(8, 8), (8, 2)], ids=["mha", "gqa"])
+def test_decode_session_with_shared_prefixes(pkv, H, Hk):
+    # the host-buffer call: inputs from pinned host memory, groups built on the host per step
+    fb = ForkBatch(pkv, H, Hk, 128, 16, [700, 90], 4, lambda i: (11 * i) % 30)
+    sess = pkv.DecodeSession(fb.kc, fb.vc, len(fb.seqs), H, fb.max_blocks, fb.max_context_len,
+                             shared_prefix=True)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+    out = torch.empty((len(fb.seqs), H, 128), dtype=torch.float16).pin_memory()
+    kn = np.stack([a for a, _ in fb.new])
+    vn = np.stack([b for _, b in fb.new])
+    sess.step(pin(fb.q_host), pin(kn), pin(vn), None, pin(fb.tables_host), pin(fb.lens_host), out)
+    torch.cuda.synchronize()
+    assert pkv.device_errors() == 0
+    # 4 samples per prompt: one group each with MHA, two of 2 members with 4 heads per kv head
+    assert sess._last_groups == (2 if H == Hk else 4)
+    ref, kc, vc, relabel = fb.expected(list(range(len(fb.seqs))))
+    idx = torch.tensor(list(relabel), dtype=torch.long, device=DEV)
+    assert np.array_equal(_bits(fb.kc[idx]), kc.view(np.uint16))
+    assert_attention_close(out.numpy(), ref)

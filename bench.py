@@ -187,6 +187,14 @@ def gpu_id_for(device_index: int) -> str:
 
 # ---- peaks and ncu traffic -------------------------------------------------------------
 
+def describe(w) -> str:
+    """The workload string both arms put in config.workload."""
+    lens = wl.context_lens(w)
+    return ("%s: %d seqs, %d query / %d kv heads, head_dim %d, block_size %d, contexts %d..%d, "
+            "%d-block pool" % (w.name, w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim,
+                               w.block_size, lens.min(), lens.max(), w.num_blocks))
+
+
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -357,11 +365,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f16", "accumulate": "f32", "data": "synthetic",
             "config": {
-                "workload": "%s: %d seqs, %d query / %d kv heads, head_dim %d, block_size %d, "
-                            "contexts %s, %d-block pool" % (
-                                w.name, B, H, Hk, D, w.block_size,
-                                "%d..%d" % (gb.lens_host.min(), gb.lens_host.max()),
-                                w.num_blocks),
+                "workload": describe(w),
                 "seed": w.seed, "partition_size": part, "kv_bytes_per_step": kv_bytes,
                 "step": args.step,
                 "l2": "no flush: each step reads %.2f GB of K/V, far above the 126 MB L2"
@@ -743,7 +747,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": round(dt * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "seed": w.seed, "sample": sample},
+        "config": {"workload": describe(w), "seed": w.seed, "sample": sample,
+                   "parallelism": "replicas x%d" % max(args.gpus, 1)},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -74,6 +74,14 @@ def _run_and_compare(pkv, w, partition_size=0, sample=None, check_pool=True, fus
         idx = torch.tensor(ob.blocks, dtype=torch.long, device=DEV)
         assert np.array_equal(_bits(gb.key_cache[idx]), ob.key_cache.view(np.uint16))
         assert np.array_equal(_bits(gb.value_cache[idx]), ob.value_cache.view(np.uint16))
+        if sample is None:
+            # the whole pool: every block outside the tables still holds the sentinel
+            used = {b for t in ob.tables for b in t}
+            free = torch.tensor([b for b in range(w.num_blocks) if b not in used],
+                                dtype=torch.long, device=DEV)
+            if len(free):
+                for pool in (gb.key_cache, gb.value_cache):
+                    assert (_bits(pool[free]) == wl.SENTINEL_BITS).all()
     got = gb.out.cpu().numpy().astype(np.float64)[ob.sample]
     err = assert_attention_close(got, ob.attention())
     del gb

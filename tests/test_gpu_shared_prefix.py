@@ -150,6 +150,13 @@ def _run(pkv, fb, fused, partition_size=0, sample=None, max_members=None, expect
     idx = torch.tensor(list(relabel), dtype=torch.long, device=DEV)
     assert np.array_equal(_bits(fb.kc[idx]), kc.view(np.uint16))
     assert np.array_equal(_bits(fb.vc[idx]), vc.view(np.uint16))
+    # blocks no sequence references were never written
+    used = {b for x in fb.seqs for b in fb.model.block_table(x)}
+    free = [b for b in range(fb.N) if b not in used]
+    if free:
+        fi = torch.tensor(free, dtype=torch.long, device=DEV)
+        assert (_bits(fb.kc[fi]) == wl.SENTINEL_BITS).all()
+        assert (_bits(fb.vc[fi]) == wl.SENTINEL_BITS).all()
     err = assert_attention_close(fb.out.cpu().numpy()[sample], ref)
     # the plain decode over the same cache agrees too
     plain = torch.empty_like(fb.out)

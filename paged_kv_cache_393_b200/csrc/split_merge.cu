@@ -9,14 +9,15 @@
 // slots of a (sequence, head) are its prefix partitions, then the partitions
 // of the rest of its context.
 //
-// One warp per (sequence, head), four per CTA: the lanes stride over the
-// partitions for the maximum and the denominator (warp shuffles), then every
-// lane owns one float4 column of the output and adds the partitions' columns
-// with their weights, broadcast from the lane that computed them.  No shared
-// memory and no CTA barrier: a (sequence, head) is a short chain of dependent
-// loads, and the grid fits the GPU in about one wave.  The kernel is launched
-// as a programmatic dependent of the partition pass: its CTAs can be resident
-// before that pass ends and wait (griddepcontrol.wait) for its results.
+// One warp per (sequence, head), four per CTA.  The lanes stride over the
+// partitions for the maximum (warp shuffles); then the warp splits into four
+// groups of eight lanes, group g taking partitions g, g+4, g+8, ... and each
+// lane D/32 float4 columns of them, so a long context (tens of partitions) is a
+// short chain of loads with many in flight; two shuffles add the groups up.
+// No shared memory and no CTA barrier, and the grid fits the GPU in about one
+// wave.  The kernel is launched as a programmatic dependent of the partition
+// pass: its CTAs can be resident before that pass ends and wait
+// (griddepcontrol.wait) for its results.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,12 +25,18 @@ namespace pkv {
 namespace {
 
 constexpr int MERGE_WARPS = 4;
+constexpr int MERGE_GROUPS = 4;  // lane groups per warp, each over every 4th partition
 
 template <int D>
 __global__ void __launch_bounds__(MERGE_WARPS * 32) split_merge_kernel(const DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the partition pass
   constexpr int V4 = D / 4;                           // float4 columns of one output row
+  constexpr int GL = 32 / MERGE_GROUPS;               // lanes per group
+  constexpr int CPL = V4 / GL;                        // float4 columns per lane
+  static_assert(V4 % GL == 0, "columns must split evenly over a group");
   const int lane = threadIdx.x & 31;
+  const int grp = lane / GL;
+  const int sub = lane % GL;
   const long long row = (long long)blockIdx.x * MERGE_WARPS + (threadIdx.x >> 5);  // b * H + h
   if (row >= (long long)p.num_seqs * p.num_heads) return;
   const int b = (int)(row / p.num_heads);
@@ -54,30 +61,46 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) split_merge_kernel(const Dec
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const float4* src = reinterpret_cast<const float4*>(p.ws_o + row * p.num_parts * D);
   float den = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < P; i0 += 32) {
-    const int i = i0 + lane;
-    const float w = i < P ? rescale_factor(ml[2 * i], M) : 0.f;
-    den = fmaf(w, i < P ? ml[2 * i + 1] : 0.f, den);
-    const int n = min(32, P - i0);
-#pragma unroll 4
-    for (int j = 0; j < n; ++j) {
-      const float wj = __shfl_sync(0xffffffffu, w, j);
-      if (lane < V4) {
-        const float4 x = src[(size_t)(i0 + j) * V4 + lane];
-        acc.x = fmaf(wj, x.x, acc.x);
-        acc.y = fmaf(wj, x.y, acc.y);
-        acc.z = fmaf(wj, x.z, acc.z);
-        acc.w = fmaf(wj, x.w, acc.w);
-      }
+  float4 acc[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+  for (int i = grp; i < P; i += MERGE_GROUPS) {
+    const float w = rescale_factor(ml[2 * i], M);
+    if (sub == 0) den = fmaf(w, ml[2 * i + 1], den);
+    float4 x[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) x[c] = src[(size_t)i * V4 + c * GL + sub];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      acc[c].x = fmaf(w, x[c].x, acc[c].x);
+      acc[c].y = fmaf(w, x[c].y, acc[c].y);
+      acc[c].z = fmaf(w, x[c].z, acc[c].z);
+      acc[c].w = fmaf(w, x[c].w, acc[c].w);
     }
   }
+  // add up the four groups (lanes sub, sub + 8, sub + 16, sub + 24 hold the same columns)
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  if (lane < V4) {
+  for (int o = GL; o < 32; o <<= 1) {
+    den += __shfl_xor_sync(0xffffffffu, den, o);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      acc[c].x += __shfl_xor_sync(0xffffffffu, acc[c].x, o);
+      acc[c].y += __shfl_xor_sync(0xffffffffu, acc[c].y, o);
+      acc[c].z += __shfl_xor_sync(0xffffffffu, acc[c].z, o);
+      acc[c].w += __shfl_xor_sync(0xffffffffu, acc[c].w, o);
+    }
+  }
+  den = __shfl_sync(0xffffffffu, den, 0);  // only the groups' first lanes counted l
+  if (grp == 0) {
     const float inv = 1.f / den;
-    *reinterpret_cast<uint2*>(out + lane * 4) =
-        make_uint2(pack_half2(acc.x * inv, acc.y * inv), pack_half2(acc.z * inv, acc.w * inv));
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const int col = c * GL + sub;
+      *reinterpret_cast<uint2*>(out + col * 4) =
+          make_uint2(pack_half2(acc[c].x * inv, acc[c].y * inv),
+                     pack_half2(acc[c].z * inv, acc[c].w * inv));
+    }
   }
 }
 

@@ -178,3 +178,27 @@ def test_random_operations_keep_the_invariants(oracle_mod):
     for s in live:
         m.free_seq(s)
     assert m.num_free() == N and not any(m.refcount)
+
+
+def test_appended_slot_is_the_table_position_of_the_last_token(oracle_mod):
+    # the fused append writes token L-1 at row (L-1) % bs of block table[(L-1) // bs]; that
+    # must be the slot append_token hands out, through growth, forks and copy-on-write
+    rng = np.random.default_rng(5)
+    N, bs = 128, 4
+    m = _model(oracle_mod, N, bs, free_order=rng.permutation(N))
+    live = [m.add_seq(int(rng.integers(0, 9))) for _ in range(4)]
+    for _ in range(2000):
+        op = rng.integers(0, 6)
+        if op == 0 and len(live) < 30:
+            live += m.fork(live[rng.integers(len(live))], 1)
+        elif op == 1 and len(live) > 2:
+            m.free_seq(live.pop(rng.integers(len(live))))
+        else:
+            s = live[rng.integers(len(live))]
+            slot = m.append_token(s)
+            if slot is None:
+                continue
+            L = m.lens[s]
+            table = m.block_table(s)
+            assert slot == table[(L - 1) // bs] * bs + (L - 1) % bs
+        m.take_copies()

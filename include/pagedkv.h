@@ -99,8 +99,8 @@ PAGEDKV_API int pagedkv_selftest_wait_timeout(unsigned int timeout_us, void *str
  *
  * where L_b = context_lens[b] counts every cached token including the one
  * written this step.  The attention reads each sequence's K/V through its block
- * table ("查询其块表…动态地找到…高效地读取", lpnh.cn/news/1824136 §2.2 item 3 and
- * §3.2 step 4; the table itself: 5688vip ch. 4 "PagedAttention：显存管理、分页机制、
+ * table (the attention looks up each block through the table while it runs:
+ * lpnh.cn/news/1824136 §2.2 item 3 and §3.2 step 4; the table itself: 5688vip ch. 4 "PagedAttention：显存管理、分页机制、
  * 块大小选择", section "分页机制：块表与物理块的组织方式"; lpnh.cn/news/2758356 §2.2).
  * Accumulation is fp32; out is rounded once to fp16 (round to nearest even).
  *

@@ -129,8 +129,8 @@ def paged_attention(q, key_cache, value_cache, block_tables, context_lens, scale
 def reshape_and_cache(key_cache, value_cache, k, v, slot_mapping, block_size):
     """Expected pools after writing token t's K/V rows to slot s = slot_mapping[t].
 
-    Slot s addresses row s % bs of physical block s // bs ("分散(Scatter)回正确的块中",
-    lpnh.cn/news/1824136 §3.1).  A slot of -1 is padding and is skipped.  Tokens are
+    Slot s addresses row s % bs of physical block s // bs (the new rows are scattered into
+    their blocks: lpnh.cn/news/1824136 §3.1).  A slot of -1 is padding and is skipped.  Tokens are
     applied in order, so a later token wins if two share a slot.  Returns new arrays.
     """
     kc = np.array(key_cache, copy=True)
@@ -152,8 +152,9 @@ def reshape_and_cache(key_cache, value_cache, k, v, slot_mapping, block_size):
 
 def copy_blocks(key_caches, value_caches, pairs):
     """Expected pools after copying whole blocks src -> dst for every (src, dst) pair,
-    in every layer, applied in pair order (the copy step of copy-on-write:
-    "分配一个新物理块把原块内容拷贝过去", lpnh.cn/news/2758356 §4.2).  Returns new lists."""
+    in every layer, applied in pair order (the copy step of copy-on-write, where a fresh
+    block receives the shared block's contents: lpnh.cn/news/2758356 §4.2).  Returns new
+    lists."""
     out_k = [np.array(x, copy=True) for x in key_caches]
     out_v = [np.array(x, copy=True) for x in value_caches]
     for src, dst in np.asarray(pairs, dtype=np.int64).reshape(-1, 2):

@@ -15,11 +15,11 @@
  *        phys = block_tables[b][i / bs] and read row i % bs of that block:
  *            K_b[i][:] = key_cache  [phys][kvh][i % bs][:]
  *            V_b[i][:] = value_cache[phys][kvh][i % bs][:]
- *        ("逻辑块 -> 物理块" via the per-sequence block table: 5688vip ch. 4
+ *        (logical block to physical block through the per-sequence table: 5688vip ch. 4
  *        "PagedAttention：显存管理、分页机制、块大小选择", section
  *        "分页机制：块表与物理块的组织方式" and its block-table figure;
- *        lpnh.cn/news/2758356 §2.2 "Block Table"; lpnh.cn/news/1824136 §2.2,
- *        item "注意力计算时动态寻址").
+ *        lpnh.cn/news/2758356 §2.2 "Block Table"; lpnh.cn/news/1824136 §2.2
+ *        item 3, addresses resolved while attention runs).
  *     2. Scores: s_i = scale * sum_d q[b][h][d] * K_b[i][d].
  *     3. Softmax with max subtraction: p_i = exp(s_i - max_j s_j) / Z,
  *        Z = sum_i exp(s_i - max_j s_j).

@@ -288,7 +288,9 @@ PAGEDKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, in
  * PAGEDKV_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory that every GPU
  * loading the library keeps until the process exits.  It allocates nothing
  * (no cudaMalloc, cudaFree or allocating library call).
- *  - A call that needs more scratch (see paged_attention_workspace_bytes)
+ *  - With partition_size 0, a split the library would choose but that needs
+ *    more scratch than the array holds falls back to a single pass.
+ *  - A call that still needs more scratch (see paged_attention_workspace_bytes)
  *    returns PAGEDKV_EWORKSPACE and enqueues nothing.
  *  - The first call on a device that needs scratch looks up the array's device
  *    address (cudaGetSymbolAddress); make that first call before any stream

@@ -74,8 +74,17 @@ extern "C" int paged_attention_decode_noalloc(
     int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
     int num_blocks, int max_context_len, int partition_size, void* stream) {
   if (num_seqs == 0) return PAGEDKV_OK;
-  const size_t need = paged_attention_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
-                                                      block_size, max_context_len, partition_size);
+  size_t need = paged_attention_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                block_size, max_context_len, partition_size);
+  if (need > kScratchBytes && partition_size == 0) {
+    // the library's own split does not fit: a single pass needs (almost) no scratch
+    const size_t single = paged_attention_workspace_bytes(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, -1);
+    if (single <= kScratchBytes) {
+      partition_size = -1;
+      need = single;
+    }
+  }
   if (need > kScratchBytes)
     return report(PAGEDKV_EWORKSPACE,
                   "this call needs %zu bytes of scratch but the built-in scratch holds "

@@ -178,6 +178,22 @@ def test_workspace_bytes(lib):
     assert pkv.paged_attention_workspace_bytes(1, 8, 3, 64, 16, 100, 0) == 0     # rejected shape
 
 
+def test_noalloc_falls_back_to_a_single_pass_for_the_automatic_plan(lib):
+    # 256 MHA sequences up to 2500 tokens: the automatic 512-token split needs ~21 MB, more
+    # than the 16 MiB built-in scratch, so the call runs a single pass instead of refusing.
+    # Without a GPU here it then fails on the device lookup, never with EWORKSPACE.
+    B, H, D, bs, maxlen = 256, 32, 128, 16, 2500
+    assert lib.paged_attention_workspace_bytes(B, H, H, D, bs, maxlen, 0) > (16 << 20)
+    fn = lib.paged_attention_decode_noalloc
+    P, I = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [P, P, P, P, P, P, ctypes.c_float] + [I] * 9 + [P]
+    fn.restype = I
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, bs, H, B, H, D, 160, 65536, maxlen)
+    st = fn(*args, 0, None)
+    assert st != nat.EWORKSPACE
+    assert fn(*args, 512, None) == nat.EWORKSPACE     # an explicit split is kept, and refused
+
+
 def test_partition_tokens(lib):
     f = pkv.paged_attention_partition_tokens
     assert f(256, 32, 32, 128, 16, 1524, -1) == 0          # single pass asked for

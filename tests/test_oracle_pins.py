@@ -11,6 +11,8 @@ import math
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 from conftest import read_golden
 
@@ -327,3 +329,24 @@ def test_copy_blocks_copies_whole_blocks_in_every_layer(oracle_mod):
         assert np.array_equal(v2[li][4], vals[li][1]) and np.array_equal(v2[li][5], vals[li][2])
         for blk in (0, 1, 2, 3):
             assert np.array_equal(k2[li][blk], layers[li][blk])
+
+
+@settings(max_examples=40, deadline=None)
+@given(seed=st.integers(0, 2 ** 20), hk=st.sampled_from([1, 2, 3]), g=st.sampled_from([1, 2, 4]),
+       d=st.sampled_from([8, 16, 24]), bs=st.sampled_from([1, 2, 4, 8]),
+       lens=st.lists(st.integers(1, 40), min_size=1, max_size=4),
+       scale=st.floats(0.0, 2.0))
+def test_attention_equals_torch_sdpa_on_random_shapes(oracle_mod, seed, hk, g, d, bs, lens,
+                                                      scale):
+    # any head grouping, head size, block size, lengths, scale and physical placement
+    H = hk * g
+    N = sum(-(-L // bs) for L in lens) + 3
+    q, kc, vc, tables, cl, denses = _random_case(seed, lens, H, hk, d, bs, N)
+    out = oracle_mod.paged_attention(q, kc, vc, tables, cl, scale, bs, hk)
+    for b, (dk, dv) in enumerate(denses):
+        qt = torch.from_numpy(q[b].astype(np.float64)).view(1, H, 1, d)
+        kt = torch.from_numpy(dk.astype(np.float64)).permute(1, 0, 2).unsqueeze(0)
+        vt = torch.from_numpy(dv.astype(np.float64)).permute(1, 0, 2).unsqueeze(0)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qt, kt, vt, scale=scale, enable_gqa=(H != hk)).view(H, d).numpy()
+        np.testing.assert_allclose(out[b], ref, rtol=1e-11, atol=1e-12)

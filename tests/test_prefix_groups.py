@@ -133,3 +133,31 @@ def test_errors_and_capacity():
     with pytest.raises(ValueError):
         prefix_groups(t, lens[:3], 16, 8)
     del P
+
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None)
+@given(seed=st.integers(0, 2 ** 20), bs=st.sampled_from([1, 2, 4, 8, 16]),
+       prompts=st.integers(1, 6), max_members=st.integers(1, 8))
+def test_random_forests_keep_the_grouping_rules(seed, bs, prompts, max_members):
+    rng = np.random.default_rng(seed)
+    N = 4000
+    bm = BlockManager(N, bs, free_order=rng.permutation(N))
+    live = []
+    for _ in range(prompts):
+        live.append(bm.add_seq(int(rng.integers(0, 60))))
+        for _ in range(int(rng.integers(0, 4))):
+            kids = bm.fork(live[int(rng.integers(len(live)))], int(rng.integers(1, 4)))
+            for k in kids:
+                for _ in range(int(rng.integers(0, 2 * bs + 2))):
+                    bm.append_token(k)
+            live += kids
+    bm.append_tokens(live)
+    bm.take_copies()
+    maxblk = max(1, max(len(bm.block_table(s)) for s in live))
+    tables, lens = bm.build_batch(live, maxblk)
+    pre, groups = prefix_groups(tables, lens, bs, max_members)
+    _check_invariants(tables, lens, bs, max_members, pre, groups, bm.refcount)

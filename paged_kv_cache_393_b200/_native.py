@@ -159,10 +159,10 @@ def _decode(name, out, q, k_new, v_new, key_cache, value_cache, block_tables, co
             tuple(q.shape), tuple(key_cache.shape), tuple(value_cache.shape), tuple(out.shape)))
     if block_tables.dim() != 2 or block_tables.shape[0] != B or tuple(context_lens.shape) != (B,):
         raise ValueError("block_tables must be [B][max_blocks] and context_lens [B]")
+    if k_new is not None and (tuple(k_new.shape) != (B, Hk, D) or tuple(v_new.shape) != (B, Hk, D)):
+        raise ValueError("k_new and v_new must be [B][Hk][D]")
     ptrs = [_cuda(out, "out", torch.float16, 3), _cuda(q, "q", torch.float16, 3)]
     if k_new is not None:
-        if tuple(k_new.shape) != (B, Hk, D) or tuple(v_new.shape) != (B, Hk, D):
-            raise ValueError("k_new and v_new must be [B][Hk][D]")
         ptrs += [_cuda(k_new, "k_new", torch.float16, 3), _cuda(v_new, "v_new", torch.float16, 3)]
     ptrs += [_cuda(key_cache, "key_cache", torch.float16, 4),
              _cuda(value_cache, "value_cache", torch.float16, 4),
@@ -284,6 +284,7 @@ def copy_blocks(key_caches, value_caches, pairs, stream=None):
     for t in list(key_caches) + list(value_caches):
         if tuple(t.shape) != shape:
             raise ValueError("every pool must have shape %s" % (shape,))
+    for t in list(key_caches) + list(value_caches):
         _cuda(t, "pool", torch.float16, 4)
     n = 0 if pairs is None else pairs.shape[0]
     if n == 0:

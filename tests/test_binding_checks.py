@@ -49,7 +49,7 @@ def test_shape_mismatches_are_refused():
         pkv.paged_attention_decode_append(out, q, q[:, :2], q[:, :2], kc, vc, tables, lens,
                                           0.125, 16)
     with pytest.raises(ValueError, match="shape mismatch"):
-        pkv.reshape_and_cache(q, q, kc, vc, torch.zeros(2, dtype=torch.int64))
+        pkv.reshape_and_cache(q[:, :2], q[:, :2], kc, vc, torch.zeros(2, dtype=torch.int64))
 
 
 def test_shared_prefix_arguments_are_checked():

@@ -22,7 +22,6 @@
 #include <mutex>
 #include <new>
 #include <string>
-#include <unordered_map>
 #include <utility>
 #include <vector>
 
@@ -30,14 +29,17 @@ struct pagedkv_block_manager {
   struct Seq {
     std::vector<int32_t> table;
     int64_t len = 0;
+    bool alive = false;
   };
   int num_blocks = 0;
   int block_size = 0;
   std::vector<int32_t> free_list;   // allocation pops the back
   std::vector<int32_t> refcount;    // per physical block
-  std::unordered_map<int, Seq> seqs;
+  // Sequence ids are handed out in order and never reused, so the id indexes
+  // this vector directly; a released sequence keeps an empty, dead entry.
+  std::vector<Seq> seqs;
+  int64_t live = 0;
   std::vector<std::pair<int64_t, int64_t>> copies;  // queued (src, dst)
-  int next_id = 0;
   std::mutex mu;
 };
 
@@ -50,6 +52,19 @@ int bm_fail(int code, const char* msg, long long a = 0) {
   snprintf(buf, sizeof(buf), msg, a);
   g_bm_error = buf;
   return code;
+}
+
+// The live sequence with this id, or NULL.
+pagedkv_block_manager::Seq* find_seq(pagedkv_block_manager* m, long long id) {
+  if (id < 0 || id >= (long long)m->seqs.size() || !m->seqs[id].alive) return nullptr;
+  return &m->seqs[id];
+}
+
+int add_live(pagedkv_block_manager* m, pagedkv_block_manager::Seq&& s) {
+  s.alive = true;
+  m->seqs.push_back(std::move(s));
+  m->live += 1;
+  return (int)m->seqs.size() - 1;
 }
 
 int32_t pop_free(pagedkv_block_manager* m) {
@@ -127,29 +142,27 @@ int bm_add_seq(pagedkv_block_manager* m, int num_tokens) {
   s.table.reserve(need);
   for (int64_t i = 0; i < need; ++i) s.table.push_back(pop_free(m));
   s.len = num_tokens;
-  const int id = m->next_id++;
-  m->seqs.emplace(id, std::move(s));
-  return id;
+  return add_live(m, std::move(s));
 }
 
 int bm_append_token(pagedkv_block_manager* m, int seq, int64_t* slot_out) {
   if (!m || !slot_out) return bm_fail(PAGEDKV_EINVAL, "NULL argument");
   std::lock_guard<std::mutex> lock(m->mu);
-  auto it = m->seqs.find(seq);
-  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
-  return append_one(m, it->second, slot_out);
+  pagedkv_block_manager::Seq* s = find_seq(m, seq);
+  if (!s) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  return append_one(m, *s, slot_out);
 }
 
 int bm_append_tokens(pagedkv_block_manager* m, const int32_t* seqs, int n, int64_t* slots_out) {
   if (!m || (n > 0 && (!seqs || !slots_out)) || n < 0) return bm_fail(PAGEDKV_EINVAL, "bad arguments");
   std::lock_guard<std::mutex> lock(m->mu);
   for (int i = 0; i < n; ++i) {
-    auto it = m->seqs.find(seqs[i]);
-    if (it == m->seqs.end()) {
+    pagedkv_block_manager::Seq* s = find_seq(m, seqs[i]);
+    if (!s) {
       bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seqs[i]);
       return i;
     }
-    if (append_one(m, it->second, &slots_out[i]) != PAGEDKV_OK) return i;
+    if (append_one(m, *s, &slots_out[i]) != PAGEDKV_OK) return i;
   }
   return n;
 }
@@ -157,14 +170,13 @@ int bm_append_tokens(pagedkv_block_manager* m, const int32_t* seqs, int n, int64
 int bm_fork(pagedkv_block_manager* m, int seq, int n, int32_t* ids_out) {
   if (!m || n < 0 || (n > 0 && !ids_out)) return bm_fail(PAGEDKV_EINVAL, "bad arguments");
   std::lock_guard<std::mutex> lock(m->mu);
-  auto it = m->seqs.find(seq);
-  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
-  const pagedkv_block_manager::Seq parent = it->second;
+  const pagedkv_block_manager::Seq* p = find_seq(m, seq);
+  if (!p) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  const pagedkv_block_manager::Seq parent = *p;  // the vector may grow below
   for (int c = 0; c < n; ++c) {
     for (int32_t b : parent.table) m->refcount[b] += 1;
-    const int id = m->next_id++;
-    m->seqs.emplace(id, parent);
-    ids_out[c] = id;
+    pagedkv_block_manager::Seq child = parent;
+    ids_out[c] = add_live(m, std::move(child));
   }
   return PAGEDKV_OK;
 }
@@ -172,33 +184,36 @@ int bm_fork(pagedkv_block_manager* m, int seq, int n, int32_t* ids_out) {
 int bm_free_seq(pagedkv_block_manager* m, int seq) {
   if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
   std::lock_guard<std::mutex> lock(m->mu);
-  auto it = m->seqs.find(seq);
-  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
-  for (int32_t b : it->second.table) {
+  pagedkv_block_manager::Seq* s = find_seq(m, seq);
+  if (!s) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  for (int32_t b : s->table) {
     if (--m->refcount[b] == 0) m->free_list.push_back(b);
   }
-  m->seqs.erase(it);
+  std::vector<int32_t>().swap(s->table);  // release its memory
+  s->len = 0;
+  s->alive = false;
+  m->live -= 1;
   return PAGEDKV_OK;
 }
 
 int bm_block_table(pagedkv_block_manager* m, int seq, int32_t* out, int cap) {
   if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
   std::lock_guard<std::mutex> lock(m->mu);
-  auto it = m->seqs.find(seq);
-  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
-  const int n = (int)it->second.table.size();
+  const pagedkv_block_manager::Seq* s = find_seq(m, seq);
+  if (!s) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  const int n = (int)s->table.size();
   if (!out) return n;
   if (cap < n) return bm_fail(PAGEDKV_ERANGE, "table of %lld entries does not fit", n);
-  if (n) memcpy(out, it->second.table.data(), n * sizeof(int32_t));
+  if (n) memcpy(out, s->table.data(), n * sizeof(int32_t));
   return n;
 }
 
 int bm_seq_len(pagedkv_block_manager* m, int seq) {
   if (!m) return bm_fail(PAGEDKV_EINVAL, "NULL manager");
   std::lock_guard<std::mutex> lock(m->mu);
-  auto it = m->seqs.find(seq);
-  if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
-  return (int)it->second.len;
+  const pagedkv_block_manager::Seq* s = find_seq(m, seq);
+  if (!s) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  return (int)s->len;
 }
 
 int bm_build_batch(pagedkv_block_manager* m, const int32_t* seqs, int n, int32_t* block_tables,
@@ -207,13 +222,13 @@ int bm_build_batch(pagedkv_block_manager* m, const int32_t* seqs, int n, int32_t
     return bm_fail(PAGEDKV_EINVAL, "bad arguments");
   std::lock_guard<std::mutex> lock(m->mu);
   for (int i = 0; i < n; ++i) {
-    auto it = m->seqs.find(seqs[i]);
-    if (it == m->seqs.end()) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seqs[i]);
-    if ((int)it->second.table.size() > max_blocks)
+    const pagedkv_block_manager::Seq* s = find_seq(m, seqs[i]);
+    if (!s) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seqs[i]);
+    if ((int)s->table.size() > max_blocks)
       return bm_fail(PAGEDKV_ERANGE, "sequence %lld has more blocks than max_blocks", seqs[i]);
   }
   for (int i = 0; i < n; ++i) {
-    const auto& s = m->seqs.find(seqs[i])->second;
+    const auto& s = *find_seq(m, seqs[i]);
     int32_t* row = block_tables + (size_t)i * max_blocks;
     const int nb = (int)s.table.size();
     for (int j = 0; j < nb; ++j) row[j] = s.table[j];
@@ -265,8 +280,8 @@ int bm_stats(pagedkv_block_manager* m, pagedkv_bm_stats* out) {
   std::lock_guard<std::mutex> lock(m->mu);
   std::vector<int32_t> fill(m->num_blocks, 0);
   int64_t logical = 0, entries = 0;
-  for (const auto& kv : m->seqs) {
-    const auto& s = kv.second;
+  for (const auto& s : m->seqs) {
+    if (!s.alive) continue;
     logical += s.len;
     entries += (int64_t)s.table.size();
     for (size_t j = 0; j < s.table.size(); ++j) {
@@ -283,7 +298,7 @@ int bm_stats(pagedkv_block_manager* m, pagedkv_bm_stats* out) {
   out->num_blocks = m->num_blocks;
   out->free_blocks = (int64_t)m->free_list.size();
   out->used_blocks = used;
-  out->num_seqs = (int64_t)m->seqs.size();
+  out->num_seqs = m->live;
   out->logical_tokens = logical;
   out->filled_slots = filled;
   out->allocated_slots = used * m->block_size;

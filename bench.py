@@ -511,6 +511,8 @@ def run_cow(args, w, dev, world, rank, local):
         need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len,
                                                    cpart)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    plain_split = pkv.paged_attention_partition_tokens(B, H, Hk, D, w.block_size,
+                                                       gb.max_context_len, cpart) > 0
     stream = torch.cuda.Stream(dev)
     n_pairs = len(steps_host[0]["pairs"])
     copy_bytes = 2 * n_pairs * 2 * Hk * w.block_size * D * 2   # K and V blocks read + written
@@ -590,7 +592,15 @@ def run_cow(args, w, dev, world, rank, local):
         if steps[j]["pairs"] is not None:
             launches += 1
         replay(j)
-        launches += {"fused": 1, "separate": 2, "shared": 3}[args.step]   # shared: prefix, suffix, merge
+        if shared:
+            # prefix pass (when there are groups), suffix pass, merge (unless every suffix
+            # fits one partition: then the suffix pass finishes the outputs)
+            pt = cpart if cpart > 0 else 512
+            launches += (1 if steps[j]["max_prefix"] > 0 else 0) + 1 + \
+                (1 if steps[j]["max_suffix"] > pt else 0)
+        else:
+            # [reshape,] attention, and the merge when the plan splits
+            launches += {"fused": 1, "separate": 2}[args.step] + (1 if plain_split else 0)
         kv_total += steps[j]["kv_bytes"]
         unique_total += steps[j].get("unique_bytes", 0)
     host_ms = (time.perf_counter() - h0) * 1e3

@@ -254,7 +254,10 @@ def run_ours(args):
     need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, part)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
-    splits = need > 0
+    # split-K (a merge kernel and partial bytes) only when the plan partitions the contexts;
+    # the tensor-core path needs a workspace word even in a single pass
+    splits = pkv.paged_attention_partition_tokens(B, H, Hk, D, w.block_size, gb.max_context_len,
+                                                  part) > 0
     fused = args.step == "fused"
     launches_per_step = (1 if fused else 2) + (1 if splits else 0)   # [reshape,] attention[, merge]
     G = H // Hk

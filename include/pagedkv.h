@@ -70,8 +70,9 @@ extern "C" {
 #define PAGEDKV_DEVERR_SLOT 4u        /* a slot beyond the pool: that token was skipped */
 #define PAGEDKV_DEVERR_TIMEOUT 8u     /* a pipeline wait gave up after ~2 s; output invalid */
 #define PAGEDKV_DEVERR_INTERNAL 16u   /* a kernel found its launch set-up inconsistent and did nothing */
-#define PAGEDKV_DEVERR_PREFIX 32u     /* a shared-prefix group or prefix length was inconsistent:
-                                         that sequence's prefix was not used (output invalid) */
+#define PAGEDKV_DEVERR_PREFIX 32u     /* a shared-prefix group or prefix length was inconsistent,
+                                         or a host bound on the prefix / suffix lengths was below
+                                         a real length: the affected outputs are invalid */
 
 /* Message of the calling thread's last failed call ("" if none). */
 PAGEDKV_API const char *pagedkv_last_error(void);

@@ -349,9 +349,9 @@ PAGEDKV_API int reshape_and_cache(const void *k, const void *v, void *key_cache,
  *   src_dst_pairs  device int64 [num_pairs][2]
  *   block_elems    fp16 values per block, a multiple of 8
  *
- * Pairs must not overlap: no dst may repeat or appear as a src (the block
- * manager never emits such pairs); overlapping pairs give unspecified block
- * contents but stay in bounds.  An id outside [0, num_blocks) skips that pair
+ * Pairs must not overlap: no dst may repeat or appear as a src (one
+ * bm_take_copies batch never does); overlapping pairs give unspecified block
+ * contents (the CTAs copy concurrently) but stay in bounds.  An id outside [0, num_blocks) skips that pair
  * and sets PAGEDKV_DEVERR_BLOCK_ID.  Bit-exact; num_pairs == 0 is a no-op.
  * Errors: EINVAL, ECUDA.
  */
@@ -377,12 +377,22 @@ PAGEDKV_API int copy_blocks(void *const *key_caches, void *const *value_caches,
  *    block.  A shared full block needs no copy (the next token starts a fresh
  *    block anyway);
  *  - release decrements every block of the sequence; blocks reaching 0 return
- *    to the free list.
+ *    to the free list;
+ *  - a queued copy has not happened yet (the pages copy the shared block
+ *    before its count drops, lpnh.cn/news/2758356 §4.2, and warn that a block
+ *    reclaimed early is handed out again and overwritten, §4.3): both blocks of
+ *    a queued pair stay off the free list until bm_take_copies hands the pair
+ *    out, even if their count reaches 0 meanwhile.  A copy-on-write of a block
+ *    that is itself still waiting for its copy is queued from that block's
+ *    source, so the pairs of one bm_take_copies never repeat a destination or
+ *    name a destination as a source (copy_blocks' requirement).
  *
  * A failed call changes nothing.  Every call locks the manager, so reference
  * counts stay consistent when several threads share one manager (the pages
  * warn that unsynchronised counts corrupt shared blocks, lpnh.cn/news/2758356
- * §4.3).  Sequence ids are small non-negative ints, never reused.
+ * §4.3).  Sequence ids are small non-negative ints; the id of a released
+ * sequence is handed out again, the most recently released first, so ids stay
+ * below the largest number of sequences alive at once.
  */
 typedef struct pagedkv_block_manager pagedkv_block_manager;
 
@@ -419,6 +429,14 @@ PAGEDKV_API int bm_block_table(pagedkv_block_manager *bm, int seq, int32_t *out,
 /* Tokens held by the sequence, or ENOENT. */
 PAGEDKV_API int bm_seq_len(pagedkv_block_manager *bm, int seq);
 
+/* Flat slots (physical block * block_size + row) of the sequence's tokens
+ * first .. first+count-1, the slots reshape_and_cache writes them to (a token
+ * at position i lies in row i % block_size of its table's block i / block_size:
+ * 5688vip ch. 4, section "分页机制：块表与物理块的组织方式").  Returns count,
+ * ENOENT, EINVAL, or ERANGE for tokens beyond the sequence's length. */
+PAGEDKV_API int bm_seq_slots(pagedkv_block_manager *bm, int seq, int first, int count,
+                             int64_t *slots_out);
+
 /* Packs the tables and lengths of seqs[0..n) into block_tables[n][max_blocks]
  * (unused entries = -1) and context_lens[n].  OK, ENOENT, ERANGE or EINVAL. */
 PAGEDKV_API int bm_build_batch(pagedkv_block_manager *bm, const int32_t *seqs, int n,
@@ -426,7 +444,10 @@ PAGEDKV_API int bm_build_batch(pagedkv_block_manager *bm, const int32_t *seqs, i
 
 /* Moves the queued copy-on-write pairs to pairs[0..2*count) as (src, dst) and
  * returns count; with pairs == NULL only returns count.  ERANGE if cap (in
- * pairs) < count, in which case nothing is moved. */
+ * pairs) < count, in which case nothing is moved.  Run copy_blocks on the pairs
+ * before any later write into their destinations (the next step's new rows);
+ * blocks that no table references any more return to the free list here, the
+ * pairs' blocks in pair order (source, then destination). */
 PAGEDKV_API int bm_take_copies(pagedkv_block_manager *bm, int64_t *pairs, int cap);
 
 /* Reference count of a block (0 = free), or EINVAL. */
@@ -452,6 +473,8 @@ typedef struct pagedkv_bm_stats {
   int64_t filled_slots;    /* physical slots holding a token */
   int64_t allocated_slots; /* used_blocks * block_size */
   int64_t table_entries;   /* sum of table lengths (= sum of refcounts) */
+  int64_t held_blocks;     /* refcount 0 but named by a queued copy pair: neither used
+                              nor free until bm_take_copies */
 } pagedkv_bm_stats;
 
 /* Fills *out.  OK or EINVAL. */

@@ -184,6 +184,17 @@ class BlockManagerModel:
       needs no copy: the next token goes to a fresh block (lpnh.cn/news/2758356 §4.2).
     * Fill of the last block is derived from the sequence length (the concept
       model's per-block token_count is ambiguous once blocks are shared).
+    * A queued copy has not happened yet: the pages copy the shared block's
+      contents first and only then drop its count (lpnh.cn/news/2758356 §4.2),
+      and a block reclaimed too early gets handed out again and overwritten
+      (§4.3).  So both ends of a queued pair stay out of the free list until
+      the pair is taken (take_copies), even when their count reaches 0 first;
+      take_copies then returns them in pair order (source, then destination).
+      A write into a block that is itself still waiting for its copy is copied
+      from that block's source, so the pairs of one take name no block twice as
+      destination and no destination as a source: applied all at once they give
+      what applying them one after another gives.
+    * Released sequence ids are reused, the most recently released first.
     """
 
     def __init__(self, num_blocks: int, block_size: int, free_order=None):
@@ -198,10 +209,13 @@ class BlockManagerModel:
             if sorted(self.free) != list(range(num_blocks)):
                 raise ValueError("free_order must be a permutation of 0..num_blocks-1")
         self.refcount = [0] * num_blocks
+        self.pinned = [0] * num_blocks      # queued copy pairs naming the block
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
         self.copies: list[tuple[int, int]] = []
+        self.copy_source: dict[int, int] = {}   # destination -> source of a queued pair
         self._next_id = 0
+        self._free_ids: list[int] = []
 
     # -- allocation ---------------------------------------------------------
     def allocate_block(self):
@@ -212,8 +226,11 @@ class BlockManagerModel:
         return blk
 
     def _new_seq(self, table, length):
-        sid = self._next_id
-        self._next_id += 1
+        if self._free_ids:
+            sid = self._free_ids.pop()
+        else:
+            sid = self._next_id
+            self._next_id += 1
         self.tables[sid] = table
         self.lens[sid] = length
         return sid
@@ -245,7 +262,11 @@ class BlockManagerModel:
                 new = self.allocate_block()
                 if new is None:
                     return None
-                self.copies.append((last, new))
+                src = self.copy_source.get(last, last)
+                self.copies.append((src, new))
+                self.copy_source[new] = src
+                self.pinned[src] += 1
+                self.pinned[new] += 1
                 self.refcount[last] -= 1
                 table[-1] = new
         slot = table[L // bs] * bs + L % bs
@@ -266,12 +287,21 @@ class BlockManagerModel:
     def free_seq(self, seq: int):
         for blk in self.tables.pop(seq):
             self.refcount[blk] -= 1
-            if self.refcount[blk] == 0:
+            if self.refcount[blk] == 0 and self.pinned[blk] == 0:
                 self.free.append(blk)
         del self.lens[seq]
+        self._free_ids.append(seq)
 
     def take_copies(self):
+        """The queued (source, destination) pairs, in queue order; their blocks are
+        released from the queue (and freed if no table references them)."""
         out, self.copies = self.copies, []
+        self.copy_source = {}
+        for pair in out:
+            for blk in pair:
+                self.pinned[blk] -= 1
+                if self.pinned[blk] == 0 and self.refcount[blk] == 0:
+                    self.free.append(blk)
         return out
 
     # -- views ----------------------------------------------------------------
@@ -291,11 +321,13 @@ class BlockManagerModel:
             for j, blk in enumerate(table):
                 fill[blk] = max(fill.get(blk, 0), min(bs, L - j * bs))
         used = sum(1 for r in self.refcount if r > 0)
+        held = sum(1 for r, p in zip(self.refcount, self.pinned) if r == 0 and p > 0)
         return {"num_blocks": self.num_blocks, "free_blocks": len(self.free),
                 "used_blocks": used, "num_seqs": len(self.tables),
                 "logical_tokens": sum(self.lens.values()), "filled_slots": sum(fill.values()),
                 "allocated_slots": used * bs,
-                "table_entries": sum(len(t) for t in self.tables.values())}
+                "table_entries": sum(len(t) for t in self.tables.values()),
+                "held_blocks": held}
 
     def slots_of(self, seq: int):
         """Flat slots of every token of the sequence, in logical order."""

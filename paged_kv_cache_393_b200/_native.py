@@ -71,6 +71,7 @@ def load_library():
             "bm_free_seq": ([P, I], I),
             "bm_block_table": ([P, I, P, I], I),
             "bm_seq_len": ([P, I], I),
+            "bm_seq_slots": ([P, I, I, I, P], I),
             "bm_build_batch": ([P, P, I, P, I, P], I),
             "bm_take_copies": ([P, P, I], I),
             "bm_refcount": ([P, I], I),
@@ -495,6 +496,15 @@ class BlockManager:
     def seq_len(self, seq: int) -> int:
         return self._chk(self._lib.bm_seq_len(self._h, int(seq)), "bm_seq_len")
 
+    def seq_slots(self, seq: int, first: int = 0, count: int = None) -> np.ndarray:
+        """Slots of the sequence's tokens first .. first+count-1 (default: to its end)."""
+        if count is None:
+            count = self.seq_len(seq) - first
+        out = np.empty(max(count, 1), np.int64)
+        self._chk(self._lib.bm_seq_slots(self._h, int(seq), int(first), int(count),
+                                         _np_ptr(out)), "bm_seq_slots")
+        return out[:count]
+
     def build_batch(self, seqs, max_blocks: int):
         s = np.ascontiguousarray(seqs, dtype=np.int32)
         tables = np.empty((s.shape[0], max_blocks), np.int32)
@@ -517,10 +527,10 @@ class BlockManager:
 
     def stats(self) -> dict:
         """Pool occupancy: see pagedkv_bm_stats in include/pagedkv.h."""
-        out = (ctypes.c_int64 * 8)()
-        self._chk(self._lib.bm_stats(self._h, out), "bm_stats")
         keys = ("num_blocks", "free_blocks", "used_blocks", "num_seqs", "logical_tokens",
-                "filled_slots", "allocated_slots", "table_entries")
+                "filled_slots", "allocated_slots", "table_entries", "held_blocks")
+        out = (ctypes.c_int64 * len(keys))()
+        self._chk(self._lib.bm_stats(self._h, out), "bm_stats")
         return dict(zip(keys, [int(x) for x in out]))
 
     def free_list(self):

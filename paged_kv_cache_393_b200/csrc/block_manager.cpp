@@ -12,7 +12,13 @@
 //  * sharing on fork and copy-on-write of a shared, not yet full block, with a
 //    shared full block needing no copy (lpnh.cn/news/2758356 §4.2);
 //  * counts updated under a lock (lpnh.cn/news/2758356 §4.3 warns that
-//    unsynchronised counts free shared blocks early).
+//    unsynchronised counts free shared blocks early);
+//  * a queued copy has not happened yet: the pages copy a shared block first
+//    and only then drop its count (§4.2), and a block reclaimed early is handed
+//    out again and overwritten (§4.3).  Both ends of a queued (src, dst) pair
+//    therefore stay off the free list until bm_take_copies hands the pair out,
+//    and a write into a block that is still waiting for its own copy is copied
+//    from that block's source, so one batch of pairs is free of overlaps.
 #include "../../include/pagedkv.h"
 
 #include <algorithm>
@@ -35,9 +41,14 @@ struct pagedkv_block_manager {
   int block_size = 0;
   std::vector<int32_t> free_list;   // allocation pops the back
   std::vector<int32_t> refcount;    // per physical block
-  // Sequence ids are handed out in order and never reused, so the id indexes
-  // this vector directly; a released sequence keeps an empty, dead entry.
+  std::vector<int32_t> pinned;      // per physical block: queued copy pairs naming it
+  std::vector<int32_t> copy_source; // per physical block: source of its queued copy, -1 = none
+  // The id indexes this vector directly.  A released sequence leaves an empty,
+  // dead entry whose id goes on free_ids; new sequences take the most recently
+  // released id first, so the vector never outgrows the most sequences alive
+  // at once.
   std::vector<Seq> seqs;
+  std::vector<int32_t> free_ids;
   int64_t live = 0;
   std::vector<std::pair<int64_t, int64_t>> copies;  // queued (src, dst)
   std::mutex mu;
@@ -62,9 +73,20 @@ pagedkv_block_manager::Seq* find_seq(pagedkv_block_manager* m, long long id) {
 
 int add_live(pagedkv_block_manager* m, pagedkv_block_manager::Seq&& s) {
   s.alive = true;
-  m->seqs.push_back(std::move(s));
   m->live += 1;
+  if (!m->free_ids.empty()) {
+    const int id = m->free_ids.back();
+    m->free_ids.pop_back();
+    m->seqs[id] = std::move(s);
+    return id;
+  }
+  m->seqs.push_back(std::move(s));
   return (int)m->seqs.size() - 1;
+}
+
+// Returns blk to the free list once no table references it and no queued copy names it.
+void release_if_unused(pagedkv_block_manager* m, int32_t blk) {
+  if (m->refcount[blk] == 0 && m->pinned[blk] == 0) m->free_list.push_back(blk);
 }
 
 int32_t pop_free(pagedkv_block_manager* m) {
@@ -90,7 +112,12 @@ int append_one(pagedkv_block_manager* m, pagedkv_block_manager::Seq& s, int64_t*
       // shared and not full: copy on write
       if (m->free_list.empty()) return bm_fail(PAGEDKV_ENOMEM, "block pool exhausted (copy on write)");
       const int32_t fresh = pop_free(m);
-      m->copies.emplace_back(last, fresh);
+      // a block still waiting for its own copy holds its source's contents
+      const int32_t src = m->copy_source[last] >= 0 ? m->copy_source[last] : last;
+      m->copies.emplace_back(src, fresh);
+      m->copy_source[fresh] = src;
+      m->pinned[src] += 1;
+      m->pinned[fresh] += 1;
       m->refcount[last] -= 1;
       s.table.back() = fresh;
     }
@@ -111,6 +138,8 @@ pagedkv_block_manager* bm_create(int num_blocks, int block_size, const int32_t* 
   m->num_blocks = num_blocks;
   m->block_size = block_size;
   m->refcount.assign(num_blocks, 0);
+  m->pinned.assign(num_blocks, 0);
+  m->copy_source.assign(num_blocks, -1);
   m->free_list.resize(num_blocks);
   if (free_order) {
     std::vector<char> seen(num_blocks, 0);
@@ -173,6 +202,8 @@ int bm_fork(pagedkv_block_manager* m, int seq, int n, int32_t* ids_out) {
   const pagedkv_block_manager::Seq* p = find_seq(m, seq);
   if (!p) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
   const pagedkv_block_manager::Seq parent = *p;  // the vector may grow below
+  if (m->seqs.size() - m->free_ids.size() + (size_t)n > (size_t)INT32_MAX)
+    return bm_fail(PAGEDKV_EINVAL, "too many sequences");
   for (int c = 0; c < n; ++c) {
     for (int32_t b : parent.table) m->refcount[b] += 1;
     pagedkv_block_manager::Seq child = parent;
@@ -187,12 +218,14 @@ int bm_free_seq(pagedkv_block_manager* m, int seq) {
   pagedkv_block_manager::Seq* s = find_seq(m, seq);
   if (!s) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
   for (int32_t b : s->table) {
-    if (--m->refcount[b] == 0) m->free_list.push_back(b);
+    --m->refcount[b];
+    release_if_unused(m, b);
   }
   std::vector<int32_t>().swap(s->table);  // release its memory
   s->len = 0;
   s->alive = false;
   m->live -= 1;
+  m->free_ids.push_back(seq);
   return PAGEDKV_OK;
 }
 
@@ -214,6 +247,22 @@ int bm_seq_len(pagedkv_block_manager* m, int seq) {
   const pagedkv_block_manager::Seq* s = find_seq(m, seq);
   if (!s) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
   return (int)s->len;
+}
+
+int bm_seq_slots(pagedkv_block_manager* m, int seq, int first, int count, int64_t* slots_out) {
+  if (!m || first < 0 || count < 0 || (count > 0 && !slots_out))
+    return bm_fail(PAGEDKV_EINVAL, "bad arguments");
+  std::lock_guard<std::mutex> lock(m->mu);
+  const pagedkv_block_manager::Seq* s = find_seq(m, seq);
+  if (!s) return bm_fail(PAGEDKV_ENOENT, "unknown sequence %lld", seq);
+  if ((int64_t)first + count > s->len)
+    return bm_fail(PAGEDKV_ERANGE, "tokens beyond the sequence's %lld", s->len);
+  const int bs = m->block_size;
+  for (int i = 0; i < count; ++i) {
+    const int64_t pos = (int64_t)first + i;
+    slots_out[i] = (int64_t)s->table[pos / bs] * bs + pos % bs;
+  }
+  return count;
 }
 
 int bm_build_batch(pagedkv_block_manager* m, const int32_t* seqs, int n, int32_t* block_tables,
@@ -247,6 +296,14 @@ int bm_take_copies(pagedkv_block_manager* m, int64_t* pairs, int cap) {
   for (int i = 0; i < n; ++i) {
     pairs[2 * i] = m->copies[i].first;
     pairs[2 * i + 1] = m->copies[i].second;
+  }
+  // the pairs are handed out: their blocks leave the queue, in pair order
+  for (const auto& pr : m->copies) {
+    for (const int64_t blk : {pr.first, pr.second}) {
+      m->pinned[blk] -= 1;
+      release_if_unused(m, (int32_t)blk);
+    }
+    m->copy_source[pr.second] = -1;
   }
   m->copies.clear();
   return n;
@@ -290,9 +347,10 @@ int bm_stats(pagedkv_block_manager* m, pagedkv_bm_stats* out) {
       if (in_block > f) f = (int32_t)in_block;
     }
   }
-  int64_t used = 0, filled = 0;
+  int64_t used = 0, filled = 0, held = 0;
   for (int b = 0; b < m->num_blocks; ++b) {
     if (m->refcount[b] > 0) ++used;
+    else if (m->pinned[b] > 0) ++held;
     filled += fill[b];
   }
   out->num_blocks = m->num_blocks;
@@ -303,6 +361,7 @@ int bm_stats(pagedkv_block_manager* m, pagedkv_bm_stats* out) {
   out->filled_slots = filled;
   out->allocated_slots = used * m->block_size;
   out->table_entries = entries;
+  out->held_blocks = held;
   return PAGEDKV_OK;
 }
 

@@ -8,11 +8,24 @@
 namespace pkv {
 namespace {
 
+// Streaming 16-byte load of data no thread of this launch writes (the new rows).
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
+  return r;
+}
+
+// Streaming 16-byte load through the coherent path: copy_blocks reads the pools
+// it writes in the same launch (another pair's destination), so the read-only
+// path is not allowed there.
+__device__ __forceinline__ uint4 ld_coherent_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p)
+               : "memory");
   return r;
 }
 
@@ -81,7 +94,7 @@ __global__ void __launch_bounds__(COPY_THREADS)
 #pragma unroll
     for (int j = 0; j < COPY_VPT; ++j) {
       const long long i = i0 + j * COPY_THREADS + threadIdx.x;
-      if (i < block_vecs) r[j] = ld_stream(s + i);
+      if (i < block_vecs) r[j] = ld_coherent_stream(s + i);
     }
 #pragma unroll
     for (int j = 0; j < COPY_VPT; ++j) {

@@ -202,3 +202,120 @@ def test_appended_slot_is_the_table_position_of_the_last_token(oracle_mod):
             table = m.block_table(s)
             assert slot == table[(L - 1) // bs] * bs + (L - 1) % bs
         m.take_copies()
+
+
+def _disjoint(pairs):
+    """No destination repeats and no destination is also a source: copy_blocks may then
+    apply the pairs in any order, or all at once, with the same result."""
+    dsts = [d for _, d in pairs]
+    return len(set(dsts)) == len(dsts) and not set(dsts) & {s for s, _ in pairs}
+
+
+def test_queued_copy_source_is_not_reclaimed_before_the_copy(oracle_mod):
+    # A and B share a partial tail T; A's write queues (T -> F); B is released before the
+    # copy is taken.  T must not go back to the free list yet: another copy-on-write in
+    # the same batch would otherwise take T as its destination (pages: the shared block
+    # is copied before its count drops, and an early-reclaimed block gets overwritten,
+    # lpnh.cn/news/2758356 §4.2-§4.3).
+    m = _model(oracle_mod, 8, 4, free_order=list(range(8)))
+    a = m.add_seq(2)
+    (b,) = m.fork(a, 1)
+    t = m.block_table(a)[0]
+    u_owner = m.add_seq(3)
+    (u_sib,) = m.fork(u_owner, 1)
+    m.append_token(a)                              # queues (t, f1)
+    m.free_seq(b)                                  # t now has no reader but the copy
+    assert m.refcount[t] == 0 and t not in m.free
+    assert m.stats()["held_blocks"] == 1
+    m.append_token(u_owner)                        # queues (u, f2) with f2 != t
+    pairs = m.take_copies()
+    assert len(pairs) == 2 and pairs[0][0] == t and pairs[1][1] != t
+    assert _disjoint(pairs)
+    assert t in m.free                             # released once its copy is handed out
+    m.free_seq(u_sib)
+
+
+def test_copy_of_a_block_still_waiting_for_its_copy_reads_the_original(oracle_mod):
+    # A writes into shared T (queues T -> F1); then A is forked and the child writes
+    # into F1 before the copies are taken: its copy comes from T (F1 does not hold
+    # T's rows yet), so the batch is (T -> F1), (T -> F2) and has no overlap
+    m = _model(oracle_mod, 8, 4, free_order=list(range(8)))
+    a = m.add_seq(1)
+    m.fork(a, 1)
+    t = m.block_table(a)[0]
+    m.append_token(a)
+    f1 = m.block_table(a)[0]
+    (c,) = m.fork(a, 1)
+    m.append_token(c)
+    f2 = m.block_table(c)[0]
+    assert m.take_copies() == [(t, f1), (t, f2)]
+
+
+def test_ids_of_released_sequences_are_reused(oracle_mod):
+    m = _model(oracle_mod, 16, 4)
+    ids = [m.add_seq(1) for _ in range(4)]
+    assert ids == [0, 1, 2, 3]
+    m.free_seq(1)
+    m.free_seq(3)
+    assert m.add_seq(1) == 3 and m.add_seq(1) == 1 and m.add_seq(1) == 4
+
+
+def test_every_sequence_reads_back_its_own_tokens(oracle_mod):
+    # A simulated device pool, run step by step the way a decode loop drives the block
+    # manager: appends (with releases and new prompts in between), then the step's
+    # copy-on-write pairs are taken and copied, then the step's new rows are written.
+    # Forks happen between steps.  After every step each live sequence, gathered through
+    # its table, must read exactly its own token history (each fork shares its parent's
+    # history, then diverges); every batch of pairs must be free of overlaps.
+    rng = np.random.default_rng(11)
+    for trial in range(40):
+        N, bs = int(rng.integers(6, 30)), int(rng.choice([1, 2, 4]))
+        m = _model(oracle_mod, N, bs, free_order=rng.permutation(N))
+        pool = [[None] * bs for _ in range(N)]
+        history = {}
+        token = [0]
+
+        def fresh():
+            token[0] += 1
+            return token[0]
+
+        def write(slot, tok):
+            pool[slot // bs][slot % bs] = tok
+
+        for step in range(60):
+            if history and rng.random() < 0.3:     # fork between steps
+                parent = list(history)[int(rng.integers(len(history)))]
+                for kid in m.fork(parent, int(rng.integers(1, 3))):
+                    history[kid] = list(history[parent])
+            pending = {}
+            for _ in range(int(rng.integers(1, 6))):
+                op = rng.random()
+                if op < 0.15 or not history:
+                    n = int(rng.integers(0, 3 * bs + 1))
+                    s = m.add_seq(n)
+                    if s is not None:
+                        history[s] = [fresh() for _ in range(n)]
+                        for i, slot in enumerate(m.slots_of(s)):
+                            write(slot, history[s][i])
+                elif op < 0.3:
+                    s = list(history)[int(rng.integers(len(history)))]
+                    m.free_seq(s)
+                    del history[s]
+                    pending.pop(s, None)
+                else:
+                    s = list(history)[int(rng.integers(len(history)))]
+                    slot = m.append_token(s)
+                    if slot is not None:
+                        tok = fresh()
+                        history[s].append(tok)
+                        pending.setdefault(s, []).append((slot, tok))
+            pairs = m.take_copies()
+            assert _disjoint(pairs), (trial, step, pairs)
+            snapshot = {s: list(pool[s]) for s, _ in pairs}
+            for src, dst in pairs:                 # all at once, as one copy_blocks launch
+                pool[dst] = list(snapshot[src])
+            for writes in pending.values():
+                for slot, tok in writes:
+                    write(slot, tok)
+            for s, hist in history.items():
+                assert [pool[x // bs][x % bs] for x in m.slots_of(s)] == hist, (trial, step, s)

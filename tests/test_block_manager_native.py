@@ -181,3 +181,62 @@ def test_block_size_trade_off_on_the_llama7b_batch():
         st = r[bs]["stats"]
         per_seq = (st["allocated_slots"] - st["filled_slots"]) / st["num_seqs"]
         assert abs(per_seq - (bs - 1) / 2) < 0.25 * bs
+
+
+def test_queued_copy_blocks_stay_allocated_until_taken(oracle_mod):
+    # the ordering that used to hand a queued copy's source out again: a write into a
+    # shared tail queues (T -> F), the other sharer is released, and another
+    # copy-on-write follows before the pairs are taken
+    native = BlockManager(8, 4, free_order=list(range(8)))
+    model = oracle_mod.BlockManagerModel(8, 4, free_order=list(range(8)))
+    ids = []
+    for bm in (native, model):
+        a = bm.add_seq(2)
+        (b,) = bm.fork(a, 1)
+        u = bm.add_seq(3)
+        (u2,) = bm.fork(u, 1)
+        bm.append_token(a)
+        bm.free_seq(b)
+        bm.append_token(u)
+        ids.append((a, u, u2))
+    assert ids[0] == ids[1]
+    t = native.block_table(ids[0][0])
+    assert native.stats() == model.stats() and native.stats()["held_blocks"] == 1
+    assert native.free_list() == model.free
+    pairs = native.take_copies().tolist()
+    assert pairs == [list(p) for p in model.take_copies()]
+    assert len(pairs) == 2 and pairs[1][1] != pairs[0][0]
+    assert native.free_list() == model.free and native.stats()["held_blocks"] == 0
+    assert t == model.block_table(ids[1][0])
+
+
+def test_seq_slots_match_the_model(oracle_mod):
+    order = np.random.default_rng(2).permutation(64)
+    native = BlockManager(64, 4, free_order=order)
+    model = oracle_mod.BlockManagerModel(64, 4, free_order=order)
+    s = native.add_seq(13)
+    assert model.add_seq(13) == s
+    for _ in range(6):
+        native.append_token(s)
+        model.append_token(s)
+    assert native.seq_slots(s).tolist() == model.slots_of(s)
+    assert native.seq_slots(s, 5, 7).tolist() == model.slots_of(s)[5:12]
+    with pytest.raises(PagedKVError):
+        native.seq_slots(s, 10, 10)               # beyond the sequence
+
+
+def test_released_ids_are_reused_so_memory_stays_bounded():
+    # 1e6 add / release cycles with at most 3 sequences alive: ids stay below 3, so the
+    # manager's per-sequence storage stays at 3 entries
+    lib = __import__("paged_kv_cache_393_b200._native", fromlist=["x"]).load_library()
+    bm = BlockManager(16, 4)
+    h = bm._h
+    live = [bm.add_seq(5), bm.add_seq(1)]
+    top = max(live)
+    for i in range(1_000_000):
+        s = lib.bm_add_seq(h, 3)
+        assert s >= 0
+        top = max(top, s)
+        assert lib.bm_free_seq(h, s) == 0
+    assert top == 2
+    assert bm.stats()["num_seqs"] == 2 and bm.num_free() == 16 - 2 - 1

@@ -76,7 +76,12 @@ class BlockManagerMachine(RuleBasedStateMachine):
 
     @rule()
     def take_copies(self):
-        assert self.native.take_copies().tolist() == [list(p) for p in self.model.take_copies()]
+        pairs = self.native.take_copies().tolist()
+        assert pairs == [list(p) for p in self.model.take_copies()]
+        # one batch is safe for a single copy_blocks launch: no destination repeats and
+        # none is also a source
+        dsts = [d for _, d in pairs]
+        assert len(set(dsts)) == len(dsts) and not set(dsts) & {s for s, _ in pairs}
 
     @invariant()
     def same_state(self):

@@ -104,22 +104,20 @@ constexpr int AUTO_PARTITION = 512;
 constexpr int SIMT_CTAS_PER_SM = 6;  // resident CUDA-core CTAs per SM at the usual 2-stage ring
 constexpr size_t MAX_SMEM = 227 * 1024;
 
-// Optional overrides of the tuning choices (for sweeps); read once.
-struct Tuning {
-  int simt_kvc = 0, simt_stage_target = 0, mma_stages = 0;
-  bool no_persistent = false;
-};
-const Tuning& tuning() {
-  static Tuning t = [] {
-    Tuning x;
-    if (const char* s = getenv("PAGEDKV_SIMT_KVC")) x.simt_kvc = atoi(s);
-    if (const char* s = getenv("PAGEDKV_SIMT_RING_BYTES")) x.simt_stage_target = atoi(s);
-    if (const char* s = getenv("PAGEDKV_MMA_STAGES")) x.mma_stages = atoi(s);
-    if (const char* s = getenv("PAGEDKV_NO_PERSISTENT")) x.no_persistent = atoi(s) != 0;
-    return x;
-  }();
-  return t;
-}
+// Tuning choices, fixed at build time (measured defaults; a sweep rebuilds the
+// library with -D overrides instead of reading the environment at run time).
+#ifndef PAGEDKV_TUNE_SIMT_KVC
+#define PAGEDKV_TUNE_SIMT_KVC 0          // 0: widest of 4/2/1 kv heads within a 16 KB stage
+#endif
+#ifndef PAGEDKV_TUNE_SIMT_RING_BYTES
+#define PAGEDKV_TUNE_SIMT_RING_BYTES 32768
+#endif
+#ifndef PAGEDKV_TUNE_MMA_STAGES
+#define PAGEDKV_TUNE_MMA_STAGES 4
+#endif
+#ifndef PAGEDKV_TUNE_PERSISTENT
+#define PAGEDKV_TUNE_PERSISTENT 1
+#endif
 
 struct Plan {
   bool mma = false;
@@ -163,7 +161,6 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
   Plan p;
   p.cascade = cascade;
   p.mma = G >= 2 && G <= 8 && block_size >= 8;
-  const Tuning& tn = tuning();
   if (!p.mma) {
     if (G == 1) {
       // widest contiguous kv-head group whose stage stays within 16 KB
@@ -175,8 +172,8 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
           break;
         }
       }
-      if (tn.simt_kvc == 1 || tn.simt_kvc == 2 || tn.simt_kvc == 4) {
-        if (num_heads % tn.simt_kvc == 0) p.kvc = tn.simt_kvc;
+      if (PAGEDKV_TUNE_SIMT_KVC == 1 || PAGEDKV_TUNE_SIMT_KVC == 2 || PAGEDKV_TUNE_SIMT_KVC == 4) {
+        if (num_heads % PAGEDKV_TUNE_SIMT_KVC == 0) p.kvc = PAGEDKV_TUNE_SIMT_KVC;
       }
       p.hpc = p.kvc;
     } else {
@@ -238,12 +235,12 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     p.num_parts = 1;
   }
   // the tensor-core path runs persistent CTAs fed by a ticket word in the workspace
-  p.persistent = p.mma && num_seqs <= PERSISTENT_MAX_SEQS && !tn.no_persistent;
+  p.persistent = p.mma && num_seqs <= PERSISTENT_MAX_SEQS && PAGEDKV_TUNE_PERSISTENT;
   if (p.persistent) p.ws_bytes = ((p.ws_bytes + 15) / 16) * 16 + 16;
   // ring depth: few stages and many CTAs per SM stream best (measured)
   if (p.mma) {
     // a multiple of the consumer warps, so every warp owns the same number of stages
-    int st = tn.mma_stages > 0 ? tn.mma_stages : 4;
+    int st = PAGEDKV_TUNE_MMA_STAGES;
     st = ((st + MMA_CONSUMER_WARPS - 1) / MMA_CONSUMER_WARPS) * MMA_CONSUMER_WARPS;
     st = st > 16 ? 16 : st;
     auto smem_of = [&](int n) {
@@ -255,7 +252,7 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     p.smem = smem_of(st);
   } else {
     const size_t stage = simt_stage_bytes(head_dim, block_size, p.kvc);
-    const size_t target = tn.simt_stage_target > 0 ? (size_t)tn.simt_stage_target : 32768;
+    const size_t target = PAGEDKV_TUNE_SIMT_RING_BYTES;
     int st = (int)(target / stage);
     st = st < 2 ? 2 : (st > 16 ? 16 : st);
     while (st > 2 && simt_smem_bytes(head_dim, block_size, p.kvc, st) > MAX_SMEM) --st;
@@ -263,7 +260,7 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     p.smem = simt_smem_bytes(head_dim, block_size, p.kvc, st);
   }
   if (cascade) {
-    int st = tn.mma_stages > 0 ? tn.mma_stages : 4;
+    int st = PAGEDKV_TUNE_MMA_STAGES;
     st = ((st + MMA_CONSUMER_WARPS - 1) / MMA_CONSUMER_WARPS) * MMA_CONSUMER_WARPS;
     st = st > 16 ? 16 : st;
     while (st > MMA_CONSUMER_WARPS && mma_smem_bytes(head_dim, block_size, st) > MAX_SMEM)

@@ -1,4 +1,5 @@
-"""Sets up a paged decode batch on a GPU from the seeded workloads.
+"""GPU-side set-up of the seeded decode batches, for the tests, the smoke check and
+the bench (a fixture, not part of the library).
 
 A batch is: K/V pools on the device (every slot pre-filled with a NaN sentinel),
 a host BlockManager seeded with the workload's shuffled free list, one sequence
@@ -17,7 +18,7 @@ import torch
 
 import workloads as wl
 
-from ._native import BlockManager, copy_blocks, reshape_and_cache
+from paged_kv_cache_393_b200 import BlockManager, copy_blocks, reshape_and_cache
 
 
 def sentinel_pools(num_blocks, num_kv_heads, block_size, head_dim, device):
@@ -26,11 +27,6 @@ def sentinel_pools(num_blocks, num_kv_heads, block_size, head_dim, device):
     kc = torch.full(shape, int(bits), dtype=torch.int16, device=device).view(torch.float16)
     vc = torch.full(shape, int(bits), dtype=torch.int16, device=device).view(torch.float16)
     return kc, vc
-
-
-def _slots(table, first, count, bs):
-    i = np.arange(first, first + count)
-    return np.asarray(table, np.int64)[i // bs] * bs + i % bs
 
 
 def _write_tokens(kc, vc, k, v, slots, device):
@@ -75,7 +71,7 @@ class PagedBatch:
                 L = int(self.lens_host[b])
                 ks.append(k[:L - 1])
                 vs.append(v[:L - 1])
-                slots.append(_slots(self.bm.block_table(self.seqs[b]), 0, L - 1, bs))
+                slots.append(self.bm.seq_slots(self.seqs[b], 0, L - 1))
                 new_k[b], new_v[b] = k[L - 1], v[L - 1]
             _write_tokens(self.key_cache, self.value_cache, np.concatenate(ks), np.concatenate(vs),
                           np.concatenate(slots), self.device)
@@ -120,8 +116,8 @@ class CowBatch:
         for p in range(w.prompts):
             s = self.bm.add_seq(w.prompt_len)
             k, v = wl.sequence_kv(w.seed, p, w.prompt_len, Hk, D)
-            _write_tokens(self.key_cache, self.value_cache, k, v,
-                          _slots(self.bm.block_table(s), 0, w.prompt_len, bs), self.device)
+            _write_tokens(self.key_cache, self.value_cache, k, v, self.bm.seq_slots(s),
+                          self.device)
             self.samples += [s] + self.bm.fork(s, w.samples - 1)
         self.step_index = 0
         self.max_context_len = w.prompt_len + w.decode_steps

@@ -241,7 +241,7 @@ def run_ours(args):
     init_dist("nccl", world, local)
     dev = torch.device("cuda", local)
     import paged_kv_cache_393_b200 as pkv
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     pkv.load_library()
     w = wl.get(args.workload)
     if w.lens == "cow":
@@ -335,26 +335,28 @@ def run_ours(args):
     # end to end through the public API: host buffers in, host result out
     e2e = None
     if args.e2e_steps > 0:
+        # paged_decode_step_host: the inputs uploaded from pinned host memory, the fused
+        # append + attention, the output downloaded, all in one C call per step
         sess = pkv.DecodeSession(gb.key_cache, gb.value_cache, B, H, gb.max_blocks,
-                                 gb.max_context_len, part, fused=fused)
+                                 gb.max_context_len, w.scale, part)
         pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
         hq, hk, hv = pin(gb.q_host), pin(gb.k_new_host), pin(gb.v_new_host)
-        hs, ht, hl = pin(gb.slots_host), pin(gb.tables_host), pin(gb.lens_host)
+        ht, hl = pin(gb.tables_host), pin(gb.lens_host)
         hout = torch.empty((B, H, D), dtype=torch.float16).pin_memory()
         for _ in range(5):
-            sess.step(hq, hk, hv, hs, ht, hl, hout, stream=stream)
+            sess.step(hq, hk, hv, ht, hl, hout, stream=stream)
         torch.cuda.synchronize(dev)
         barrier(world, local)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         E = args.e2e_steps
         e0.record(stream)
         for _ in range(E):
-            sess.step(hq, hk, hv, hs, ht, hl, hout, stream=stream)
+            sess.step(hq, hk, hv, ht, hl, hout, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms, e_bytes = aggregate(e0.elapsed_time(e1), float(kv_bytes) * E, world, dev)
         e2e = {"value": round(e_bytes / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
-               "ms_per_step": round(e_ms / E, 4),
+               "ms_per_step": round(e_ms / E, 4), "call": "paged_decode_step_host",
                "h2d_bytes_per_step": sess.h2d_bytes(), "d2h_bytes_per_step": sess.d2h_bytes()}
 
     cpu = None
@@ -400,7 +402,7 @@ def run_layers(args, w, dev, world, rank, local):
     import torch
 
     import paged_kv_cache_393_b200 as pkv
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     gb = PagedBatch(w, dev)
     Lyr = args.layers
     pool_bytes = 2 * gb.key_cache.numel() * 2
@@ -483,7 +485,7 @@ def run_cow(args, w, dev, world, rank, local):
     import torch
 
     import paged_kv_cache_393_b200 as pkv
-    from paged_kv_cache_393_b200.batch import CowBatch
+    from batches import CowBatch
     gb = CowBatch(w, dev)
     B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
     steps_host = [gb.prepare_step() for _ in range(w.decode_steps)]
@@ -626,17 +628,17 @@ def run_cow(args, w, dev, world, rank, local):
     E = min(args.e2e_steps, w.decode_steps, 50)
     if E > 0:
         sess = pkv.DecodeSession(gb.key_cache, gb.value_cache, B, H, gb.max_blocks,
-                                 gb.max_context_len, cpart, max_pairs=max(n_pairs, 1),
-                                 fused=args.step != "separate", shared_prefix=shared)
+                                 gb.max_context_len, w.scale, cpart, max_pairs=max(n_pairs, 1),
+                                 shared_prefix=shared)
         pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
-        hs = [{k: pin(steps_host[j][k]) for k in ("q", "k", "v", "slots", "tables", "lens")}
+        hs = [{k: pin(steps_host[j][k]) for k in ("q", "k", "v", "tables", "lens")}
               for j in range(E)]
         hpairs = pin(steps_host[0]["pairs"]) if n_pairs else None
         hout = torch.empty((B, H, D), dtype=torch.float16).pin_memory()
 
         def e2e_step(j):
             h = hs[j]
-            sess.step(h["q"], h["k"], h["v"], h["slots"], h["tables"], h["lens"], hout,
+            sess.step(h["q"], h["k"], h["v"], h["tables"], h["lens"], hout,
                       pairs=hpairs if j == 0 else None, stream=stream)
 
         for j in range(min(3, E)):
@@ -648,13 +650,13 @@ def run_cow(args, w, dev, world, rank, local):
         h2d = 0
         for j in range(E):
             e2e_step(j)
-            h2d += sess.h2d_bytes(n_pairs if j == 0 else 0)
+            h2d += sess.h2d_bytes()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms, e_bytes = aggregate(e0.elapsed_time(e1),
                                   float(sum(steps[j]["kv_bytes"] for j in range(E))), world, dev)
         e2e = {"value": round(e_bytes / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
-               "ms_per_step": round(e_ms / E, 4), "steps": E,
+               "ms_per_step": round(e_ms / E, 4), "steps": E, "call": "paged_decode_step_host",
                "h2d_bytes_per_step": int(h2d / E), "d2h_bytes_per_step": sess.d2h_bytes()}
     if rank == 0:
         peak, peak_kind = hbm_peak()

@@ -9,7 +9,7 @@ lengths, then one appended token per sequence per step -- and reports appended
 tokens per second, blocks allocated per 1000 appends, and the pool's tail waste
 (1 - filled / allocated slots) and table entries at the end.
 
-    python -m paged_kv_cache_393_b200.bm_bench [--steps 200] [--block-sizes 8 16 32 64]
+    python bm_bench.py [--steps 200] [--block-sizes 8 16 32 64]
 """
 from __future__ import annotations
 
@@ -21,13 +21,13 @@ import time
 
 import numpy as np
 
-_ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+_ROOT = os.path.dirname(os.path.abspath(__file__))
 if _ROOT not in sys.path:
     sys.path.insert(0, _ROOT)
 
 import workloads as wl  # noqa: E402
 
-from ._native import BlockManager  # noqa: E402
+from paged_kv_cache_393_b200 import BlockManager  # noqa: E402
 
 
 def run(block_size: int, steps: int, workload: str = "llama7b", pool_tokens: int = None) -> dict:

@@ -269,6 +269,72 @@ PAGEDKV_API int pagedkv_prefix_groups(const int32_t *block_tables, const int32_t
                            int max_members, int32_t *seq_prefix_tokens, int32_t *groups,
                            int groups_capacity);
 
+/* ---- one decode step from host buffers -----------------------------------------------
+ *
+ * The step a serving loop runs for one attention layer, driven from host
+ * memory: the block manager's tables and the step's inputs go to the GPU, the
+ * new token's K/V is written into its block and the attention gathers through
+ * the tables, and the output comes back (lpnh.cn/news/1824136 §3.2 steps 3-5;
+ * copy-on-write before the write: lpnh.cn/news/2758356 §4.2).  Enqueued on
+ * `stream`, in this order:
+ *
+ *   1. host -> device copies (one cudaMemcpyAsync per array) of block_tables,
+ *      context_lens, the copy pairs, the shared-prefix arrays, q, k_new, v_new
+ *      into the caller's staging buffer;
+ *   2. copy_blocks of the pairs (if any);
+ *   3. paged_attention_decode_append, or with seq_prefix_tokens_host given
+ *      paged_attention_decode_shared_prefix with k_new / v_new (its grid bounds
+ *      taken from the host arrays);
+ *   4. a device -> host copy of the output into out_host.
+ *
+ * The call returns once everything is enqueued; out_host is valid after the
+ * stream synchronizes.  With pinned (page-locked) host buffers every copy is
+ * asynchronous; pageable buffers work too, with copies the driver stages.
+ *
+ *   out_host          host fp16 [num_seqs][num_heads][head_dim]
+ *   q_host            host fp16 [num_seqs][num_heads][head_dim]
+ *   k_new_host,
+ *   v_new_host        host fp16 [num_seqs][num_kv_heads][head_dim]: the token each
+ *                     sequence appends, written at position L_b - 1
+ *   block_tables_host host int32 [num_seqs][max_blocks_per_seq] (bm_build_batch)
+ *   context_lens_host host int32 [num_seqs], each in [1, max_context_len]
+ *                     (checked on the host: EINVAL otherwise)
+ *   copy_pairs_host   host int64 [num_pairs][2] (bm_take_copies); num_pairs <=
+ *                     max_pairs.  Checked on the host: ids inside the pool, no
+ *                     destination repeated or used as a source (EINVAL otherwise).
+ *   seq_prefix_tokens_host, groups_host, num_groups
+ *                     NULL / NULL / 0 for the plain step; else host arrays as
+ *                     pagedkv_prefix_groups writes them (num_groups <= num_seqs / 2)
+ *   key_cache,
+ *   value_cache       device pools as for paged_attention_decode (one layer)
+ *   staging           device buffer of paged_decode_step_staging_bytes(...) bytes,
+ *                     256-byte aligned, owned by the caller: the device copies of
+ *                     the inputs, the output and the attention workspace.  Calls
+ *                     that may run at the same time need separate staging buffers.
+ *   the rest          as for paged_attention_decode_append
+ *
+ * num_seqs == 0 runs only the copies.  Errors: EINVAL, EUNSUPPORTED, EWORKSPACE
+ * (staging too small), ECUDA (part of the step may then have been enqueued).
+ */
+PAGEDKV_API int paged_decode_step_host(void *out_host, const void *q_host,
+                           const void *k_new_host, const void *v_new_host,
+                           const int32_t *block_tables_host, const int32_t *context_lens_host,
+                           const int64_t *copy_pairs_host, int num_pairs,
+                           const int32_t *seq_prefix_tokens_host, const int32_t *groups_host,
+                           int num_groups, void *key_cache, void *value_cache,
+                           float scale, int block_size, int num_kv_heads,
+                           int num_seqs, int num_heads, int head_dim,
+                           int max_blocks_per_seq, int num_blocks, int max_context_len,
+                           int partition_size, int max_pairs,
+                           void *staging, size_t staging_bytes, void *stream);
+
+/* Staging bytes paged_decode_step_host needs (shared_prefix != 0: for calls
+ * with the shared-prefix arrays).  0 for arguments it would reject. */
+PAGEDKV_API size_t paged_decode_step_staging_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                           int head_dim, int block_size, int max_blocks_per_seq,
+                           int max_context_len, int partition_size, int max_pairs,
+                           int shared_prefix);
+
 /* The partition size paged_attention_decode uses for these arguments: the tokens
  * per split-K partition, 0 for a single pass (partition_size 0 lets the library
  * choose), or a negative PAGEDKV_E* code for arguments it would reject. */

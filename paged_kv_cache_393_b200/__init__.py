@@ -11,8 +11,10 @@ Functions mirror the C names:
     written, then attended), paged_attention_decode_shared_prefix + prefix_groups
     (shared prefixes read once per group), paged_attention_workspace_bytes,
     reshape_and_cache,
-    copy_blocks, device_errors, BlockManager (bm_*), decode_step (host buffers
-    in, host result out), LayeredDecodeStep (every layer's decode as one CUDA graph).
+    copy_blocks, device_errors, BlockManager (bm_*), paged_decode_step_host and
+    DecodeSession / decode_step (one step from host buffers: inputs uploaded,
+    copy-on-write copies, fused append + attention, output downloaded),
+    LayeredDecodeStep (every layer's decode as one CUDA graph).
 """
 from ._native import (  # noqa: F401
     BlockManager,
@@ -29,6 +31,8 @@ from ._native import (  # noqa: F401
     paged_attention_partition_tokens,
     paged_attention_shared_prefix_workspace_bytes,
     paged_attention_workspace_bytes,
+    paged_decode_step_host,
+    paged_decode_step_staging_bytes,
     prefix_groups,
     reshape_and_cache,
     selftest_wait_timeout,

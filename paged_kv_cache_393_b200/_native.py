@@ -60,6 +60,10 @@ def load_library():
                 [P, P, P, P, P, P, P, P, P, P, I, I, I, F, I, I, I, I, I, I, I, I, I, P, Z, P], I),
             "paged_attention_shared_prefix_workspace_bytes": ([I, I, I, I, I, I, I], Z),
             "pagedkv_prefix_groups": ([P, P, I, I, I, I, P, P, I], I),
+            "paged_decode_step_host": (
+                [P, P, P, P, P, P, P, I, P, P, I, P, P, F, I, I, I, I, I, I, I, I, I, I, P, Z, P],
+                I),
+            "paged_decode_step_staging_bytes": ([I, I, I, I, I, I, I, I, I, I], Z),
             "reshape_and_cache": ([P, P, P, P, P, I, I, I, I, I, P], I),
             "copy_blocks": ([P, P, P, I, I, Z, I, P], I),
             "bm_create": ([I, I, P], P),
@@ -318,106 +322,132 @@ def device_errors(clear: bool = True) -> int:
     return int(flags.value)
 
 
+def _host(a, name, dtype, shape):
+    """Pointer of a contiguous host array (torch CPU tensor, pinned or not, or numpy)."""
+    if isinstance(a, torch.Tensor):
+        if a.is_cuda:
+            raise ValueError("%s must be in host memory" % name)
+        if a.dtype != dtype:
+            raise TypeError("%s must be %s, got %s" % (name, dtype, a.dtype))
+        if not a.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
+        got, ptr = tuple(a.shape), a.data_ptr()
+    else:
+        npd = {torch.float16: np.float16, torch.int32: np.int32, torch.int64: np.int64}[dtype]
+        if not isinstance(a, np.ndarray) or a.dtype != npd or not a.flags.c_contiguous:
+            raise TypeError("%s must be a contiguous %s array" % (name, np.dtype(npd).name))
+        got, ptr = a.shape, a.ctypes.data
+    if tuple(got) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(got)))
+    return ptr
+
+
+def paged_decode_step_staging_bytes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                    max_blocks_per_seq, max_context_len, partition_size=0,
+                                    max_pairs=0, shared_prefix=False) -> int:
+    return int(load_library().paged_decode_step_staging_bytes(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+        max_context_len, partition_size, max_pairs, int(bool(shared_prefix))))
+
+
+def paged_decode_step_host(out_host, q, k_new, v_new, block_tables, context_lens, key_cache,
+                           value_cache, scale, max_context_len, staging, partition_size=0,
+                           pairs=None, max_pairs=0, seq_prefix_tokens=None, groups=None,
+                           stream=None):
+    """One decode step from host buffers (paged_decode_step_host in include/pagedkv.h): the
+    inputs are uploaded into ``staging`` (a device uint8 tensor of
+    paged_decode_step_staging_bytes), copy-on-write pairs are copied, the fused append +
+    attention (or the shared-prefix form, given seq_prefix_tokens and groups) runs, and the
+    output is copied into out_host.  Returns out_host; it is valid once the stream
+    synchronizes."""
+    lib = load_library()
+    N, Hk, bs, D = key_cache.shape
+    B, H = q.shape[0], q.shape[1]
+    maxblk = block_tables.shape[1]
+    npairs = 0 if pairs is None else int(pairs.shape[0])
+    shared = seq_prefix_tokens is not None
+    ng = 0 if groups is None else int(groups.shape[0])
+    if tuple(value_cache.shape) != tuple(key_cache.shape):
+        raise ValueError("the pools must have the same shape")
+    ptrs = [_host(out_host, "out_host", torch.float16, (B, H, D)),
+            _host(q, "q", torch.float16, (B, H, D)),
+            _host(k_new, "k_new", torch.float16, (B, Hk, D)),
+            _host(v_new, "v_new", torch.float16, (B, Hk, D)),
+            _host(block_tables, "block_tables", torch.int32, (B, maxblk)),
+            _host(context_lens, "context_lens", torch.int32, (B,)),
+            _host(pairs, "pairs", torch.int64, (npairs, 2)) if npairs else None, npairs,
+            _host(seq_prefix_tokens, "seq_prefix_tokens", torch.int32, (B,)) if shared else None,
+            _host(groups, "groups", torch.int32, (ng, GROUP_WIDTH)) if ng else None, ng]
+    st = lib.paged_decode_step_host(
+        *ptrs, _cuda(key_cache, "key_cache", torch.float16, 4),
+        _cuda(value_cache, "value_cache", torch.float16, 4), float(scale), bs, Hk, B, H, D,
+        maxblk, N, int(max_context_len), int(partition_size), int(max_pairs),
+        _cuda(staging, "staging", torch.uint8), staging.numel(), _stream(stream, key_cache.device))
+    _check(st, "paged_decode_step_host")
+    return out_host
+
+
 class DecodeSession:
     """A decode step driven from host buffers: the call a serving loop makes.
 
-    Holds device staging buffers for one batch shape.  ``step`` copies the
-    step's inputs from (pinned) host memory, runs copy_blocks for pending
-    copy-on-write pairs, then either reshape_and_cache for the new tokens and
-    paged_attention_decode, or (fused=True) paged_attention_decode_append, which
-    writes the new tokens at position L-1 through the tables itself and needs no
-    slots, or (shared_prefix=True, fused as well) groups the batch by shared table
-    prefixes on the host (prefix_groups) and calls
-    paged_attention_decode_shared_prefix; finally it copies the output back into a
-    host tensor.
+    Holds the device staging buffer for one batch shape.  ``step`` hands the step's
+    host inputs to paged_decode_step_host, which uploads them, runs copy_blocks for
+    pending copy-on-write pairs, writes every sequence's new token at position L-1
+    through the tables and attends (paged_attention_decode_append), and copies the
+    output back into a host tensor.  With shared_prefix=True the batch is grouped
+    by shared table prefixes on the host each step (pagedkv_prefix_groups) and the
+    shared-prefix call runs instead.
     """
 
     def __init__(self, key_cache, value_cache, num_seqs, num_heads, max_blocks, max_context_len,
-                 partition_size=0, max_pairs=0, fused=False, shared_prefix=False):
-        dev = key_cache.device
+                 scale=None, partition_size=0, max_pairs=0, shared_prefix=False):
         N, Hk, bs, D = key_cache.shape
         self.key_cache, self.value_cache = key_cache, value_cache
+        self.num_seqs, self.num_heads, self.max_blocks = num_seqs, num_heads, max_blocks
         self.max_context_len = int(max_context_len)
+        self.scale = 1.0 / D ** 0.5 if scale is None else float(scale)
         self.partition_size = partition_size
+        self.max_pairs = int(max_pairs)
         self.shared_prefix = bool(shared_prefix)
-        self.fused = bool(fused) or self.shared_prefix
         self.block_size = bs
         self.max_members = max(1, 8 // (num_heads // Hk))
-        self.q = torch.empty((num_seqs, num_heads, D), dtype=torch.float16, device=dev)
-        self.k = torch.empty((num_seqs, Hk, D), dtype=torch.float16, device=dev)
-        self.v = torch.empty_like(self.k)
-        self.slots = torch.empty(num_seqs, dtype=torch.int64, device=dev)
-        self.tables = torch.empty((num_seqs, max_blocks), dtype=torch.int32, device=dev)
-        self.lens = torch.empty(num_seqs, dtype=torch.int32, device=dev)
-        self.out = torch.empty((num_seqs, num_heads, D), dtype=torch.float16, device=dev)
-        self.pairs = torch.empty((max(max_pairs, 1), 2), dtype=torch.int64, device=dev)
-        if self.shared_prefix:
-            self.prefix = torch.zeros(num_seqs, dtype=torch.int32, device=dev)
-            self.groups = torch.zeros((max(num_seqs // 2, 1), GROUP_WIDTH), dtype=torch.int32,
-                                      device=dev)
-            need = paged_attention_shared_prefix_workspace_bytes(num_seqs, num_heads, Hk, D, bs,
-                                                                 max_context_len, partition_size)
-        else:
-            need = paged_attention_workspace_bytes(num_seqs, num_heads, Hk, D, bs,
-                                                   max_context_len, partition_size)
-        self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        need = paged_decode_step_staging_bytes(num_seqs, num_heads, Hk, D, bs, max_blocks,
+                                               max_context_len, partition_size, max_pairs,
+                                               shared_prefix)
+        if need == 0:
+            _check(EINVAL, "paged_decode_step_staging_bytes")
+        self.staging = torch.zeros(need, dtype=torch.uint8, device=key_cache.device)
         self._last_groups = 0
+        self._last_pairs = 0
 
-    def h2d_bytes(self, num_pairs=0) -> int:
-        ts = (self.q, self.k, self.v, self.tables, self.lens) + (() if self.fused else (self.slots,))
-        n = sum(t.numel() * t.element_size() for t in ts) + num_pairs * 16
-        if self.shared_prefix:   # prefix lengths and the step's groups
-            n += self.prefix.numel() * 4 + self._last_groups * GROUP_WIDTH * 4
+    def h2d_bytes(self) -> int:
+        """Host-to-device bytes of the last step."""
+        B, H, D = self.num_seqs, self.num_heads, self.key_cache.shape[3]
+        Hk = self.key_cache.shape[1]
+        n = B * H * D * 2 + 2 * B * Hk * D * 2 + B * self.max_blocks * 4 + B * 4
+        n += self._last_pairs * 16
+        if self.shared_prefix:
+            n += B * 4 + self._last_groups * GROUP_WIDTH * 4
         return n
 
     def d2h_bytes(self) -> int:
-        return self.out.numel() * self.out.element_size()
+        return self.num_seqs * self.num_heads * self.key_cache.shape[3] * 2
 
-    def step(self, q, k, v, slots, tables, lens, out_host, pairs=None, stream=None):
-        """slots may be None when the session is fused."""
-        s = torch.cuda.current_stream(self.q.device) if stream is None else stream
-        scale = 1.0 / (self.q.shape[2] ** 0.5)
-        with torch.cuda.stream(s):
-            self.q.copy_(q, non_blocking=True)
-            self.k.copy_(k, non_blocking=True)
-            self.v.copy_(v, non_blocking=True)
-            if not self.fused:
-                self.slots.copy_(slots, non_blocking=True)
-            self.tables.copy_(tables, non_blocking=True)
-            self.lens.copy_(lens, non_blocking=True)
-            if pairs is not None and len(pairs):
-                n = pairs.shape[0]
-                self.pairs[:n].copy_(pairs, non_blocking=True)
-                copy_blocks([self.key_cache], [self.value_cache], self.pairs[:n], stream=s)
-            if self.shared_prefix:
-                t_host = tables.numpy() if isinstance(tables, torch.Tensor) else np.asarray(tables)
-                l_host = lens.numpy() if isinstance(lens, torch.Tensor) else np.asarray(lens)
-                pre, groups = prefix_groups(t_host, l_host, self.block_size, self.max_members)
-                n = groups.shape[0]
-                self._last_groups = n
-                self.prefix.copy_(torch.from_numpy(pre), non_blocking=False)
-                if n:
-                    self.groups[:n].copy_(torch.from_numpy(groups), non_blocking=False)
-                max_prefix = int(groups[:, 0].max()) * self.block_size if n else 0
-                max_suffix = int((l_host - pre).max()) if len(l_host) else 0
-                paged_attention_decode_shared_prefix(
-                    self.out, self.q, self.key_cache, self.value_cache, self.tables, self.lens,
-                    self.prefix, self.groups[:n], scale, self.max_context_len,
-                    self.partition_size, self.workspace, k_new=self.k, v_new=self.v, stream=s,
-                    max_prefix_tokens=max_prefix, max_suffix_tokens=max_suffix)
-            elif self.fused:
-                paged_attention_decode_append(self.out, self.q, self.k, self.v, self.key_cache,
-                                              self.value_cache, self.tables, self.lens, scale,
-                                              self.max_context_len, self.partition_size,
-                                              self.workspace, stream=s)
-            else:
-                reshape_and_cache(self.k, self.v, self.key_cache, self.value_cache, self.slots,
-                                  stream=s)
-                paged_attention_decode(self.out, self.q, self.key_cache, self.value_cache,
-                                       self.tables, self.lens, scale, self.max_context_len,
-                                       self.partition_size, self.workspace, stream=s)
-            out_host.copy_(self.out, non_blocking=True)
-        return out_host
+    def step(self, q, k, v, tables, lens, out_host, pairs=None, stream=None):
+        """q [B][H][D], k/v [B][Hk][D] fp16, tables [B][max_blocks] and lens [B] int32, pairs
+        [n][2] int64 or None: host arrays (pinned for asynchronous copies).  Returns out_host
+        (valid once the stream synchronizes)."""
+        pre = groups = None
+        if self.shared_prefix:
+            t_host = tables.numpy() if isinstance(tables, torch.Tensor) else np.asarray(tables)
+            l_host = lens.numpy() if isinstance(lens, torch.Tensor) else np.asarray(lens)
+            pre, groups = prefix_groups(t_host, l_host, self.block_size, self.max_members)
+            self._last_groups = groups.shape[0]
+        self._last_pairs = 0 if pairs is None else int(pairs.shape[0])
+        return paged_decode_step_host(
+            out_host, q, k, v, tables, lens, self.key_cache, self.value_cache, self.scale,
+            self.max_context_len, self.staging, self.partition_size,
+            pairs if self._last_pairs else None, self.max_pairs, pre, groups, stream)
 
 
 def decode_step(session: DecodeSession, *args, **kwargs):

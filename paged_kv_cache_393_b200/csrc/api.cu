@@ -14,6 +14,8 @@
 #include <cstdlib>
 #include <mutex>
 #include <string>
+#include <vector>
+#include <algorithm>
 
 namespace pkv {
 namespace {
@@ -598,6 +600,207 @@ int copy_blocks(void* const* key_caches, void* const* value_caches, const int64_
   cudaError_t e = launch_copy_blocks(key_caches, value_caches, src_dst_pairs, num_pairs, num_layers,
                                      block_elems, num_blocks, err, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "copy_blocks launch");
+  return PAGEDKV_OK;
+}
+
+}  // extern "C"
+
+// ---- one decode step from host buffers ---------------------------------------------
+
+namespace pkv {
+namespace {
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Offsets of the regions of the caller's staging buffer (each 256-byte aligned).
+struct StepLayout {
+  size_t q, k, v, tables, lens, pairs, out, prefix, groups, ws;
+  size_t ws_bytes, total;
+};
+
+int step_layout(StepLayout* lay, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                int block_size, int max_blocks_per_seq, int max_context_len, int partition_size,
+                int max_pairs, bool shared_prefix) {
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_pairs < 0)
+    return fail(PAGEDKV_EINVAL, "num_seqs, max_blocks_per_seq and max_pairs must be >= 0 (> 0)");
+  Plan plan;
+  const int st = make_plan(&plan, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                           max_context_len, partition_size, shared_prefix);
+  if (st != PAGEDKV_OK) return st;
+  const size_t B = (size_t)num_seqs, H = (size_t)num_heads, Hk = (size_t)num_kv_heads,
+               D = (size_t)head_dim;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  lay->q = take(B * H * D * 2);
+  lay->k = take(B * Hk * D * 2);
+  lay->v = take(B * Hk * D * 2);
+  lay->tables = take(B * (size_t)max_blocks_per_seq * 4);
+  lay->lens = take(B * 4);
+  lay->pairs = take((size_t)max_pairs * 16);
+  lay->out = take(B * H * D * 2);
+  lay->prefix = shared_prefix ? take(B * 4) : 0;
+  lay->groups = shared_prefix ? take((B / 2 > 0 ? B / 2 : 1) * GROUP_WIDTH * 4) : 0;
+  lay->ws = take(plan.ws_bytes);
+  lay->ws_bytes = plan.ws_bytes;
+  lay->total = off;
+  return PAGEDKV_OK;
+}
+
+// Copy-on-write pairs that one copy_blocks launch may apply in any order: ids in
+// range, no destination repeated, no destination also a source.
+int check_pairs(const int64_t* pairs, int n, int num_blocks) {
+  std::vector<char> role((size_t)num_blocks, 0);  // 1 = source, 2 = destination
+  for (int i = 0; i < n; ++i) {
+    const int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks)
+      return fail(PAGEDKV_EINVAL, "copy pair %d (%lld, %lld) outside the pool", i, (long long)s,
+                  (long long)d);
+    if (role[(size_t)s] == 2 || role[(size_t)d] != 0)
+      return fail(PAGEDKV_EINVAL, "copy pair %d (%lld, %lld) overlaps an earlier pair", i,
+                  (long long)s, (long long)d);
+    role[(size_t)s] = 1;
+    role[(size_t)d] = 2;
+  }
+  return PAGEDKV_OK;
+}
+
+int h2d(void* dst, const void* src, size_t bytes, cudaStream_t s, const char* what) {
+  if (bytes == 0) return PAGEDKV_OK;
+  const cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s);
+  return e == cudaSuccess ? PAGEDKV_OK : cuda_fail(e, what);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+size_t paged_decode_step_staging_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_dim, int block_size, int max_blocks_per_seq,
+                                       int max_context_len, int partition_size, int max_pairs,
+                                       int shared_prefix) {
+  StepLayout lay;
+  if (step_layout(&lay, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                  max_blocks_per_seq, max_context_len, partition_size, max_pairs,
+                  shared_prefix != 0) != PAGEDKV_OK)
+    return 0;
+  return lay.total;
+}
+
+int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new_host,
+                           const void* v_new_host, const int32_t* block_tables_host,
+                           const int32_t* context_lens_host, const int64_t* copy_pairs_host,
+                           int num_pairs, const int32_t* seq_prefix_tokens_host,
+                           const int32_t* groups_host, int num_groups, void* key_cache,
+                           void* value_cache, float scale, int block_size, int num_kv_heads,
+                           int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+                           int num_blocks, int max_context_len, int partition_size, int max_pairs,
+                           void* staging, size_t staging_bytes, void* stream) {
+  if (num_seqs < 0) return fail(PAGEDKV_EINVAL, "num_seqs must be >= 0");
+  if (num_pairs < 0 || num_pairs > max_pairs)
+    return fail(PAGEDKV_EINVAL, "num_pairs %d outside [0, max_pairs = %d]", num_pairs, max_pairs);
+  if (num_seqs == 0 && num_pairs == 0) return PAGEDKV_OK;
+  const bool shared = seq_prefix_tokens_host != nullptr;
+  if (!key_cache || !value_cache || !staging ||
+      (num_seqs > 0 && (!out_host || !q_host || !k_new_host || !v_new_host ||
+                        !block_tables_host || !context_lens_host)) ||
+      (num_pairs > 0 && !copy_pairs_host) || (shared && num_groups > 0 && !groups_host))
+    return fail(PAGEDKV_EINVAL, "a required pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(staging) & 255u) != 0)
+    return fail(PAGEDKV_EINVAL, "staging must be 256-byte aligned");
+  if (num_blocks <= 0) return fail(PAGEDKV_EINVAL, "num_blocks must be positive");
+  StepLayout lay;
+  int st = step_layout(&lay, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                       max_blocks_per_seq, max_context_len, partition_size, max_pairs, shared);
+  if (st != PAGEDKV_OK) return st;
+  if (staging_bytes < lay.total)
+    return fail(PAGEDKV_EWORKSPACE, "staging of %zu bytes required, %zu given", lay.total,
+                staging_bytes);
+  // host-side checks of what the host already holds
+  for (int b = 0; b < num_seqs; ++b) {
+    const int L = context_lens_host[b];
+    if (L < 1 || L > max_context_len)
+      return fail(PAGEDKV_EINVAL, "context_lens[%d] = %d outside [1, max_context_len = %d]", b, L,
+                  max_context_len);
+  }
+  st = check_pairs(copy_pairs_host, num_pairs, num_blocks);
+  if (st != PAGEDKV_OK) return st;
+  int max_prefix = 0, max_suffix = 0;
+  if (shared) {
+    if (num_groups < 0 || num_groups > (num_seqs / 2 > 0 ? num_seqs / 2 : 1))
+      return fail(PAGEDKV_EINVAL, "num_groups %d outside [0, num_seqs / 2]", num_groups);
+    for (int g = 0; g < num_groups; ++g) {
+      const int pb = groups_host[(size_t)g * GROUP_WIDTH];
+      if (pb > 0 && (long long)pb * block_size > max_prefix)
+        max_prefix = (int)std::min<long long>((long long)pb * block_size, max_context_len);
+    }
+    for (int b = 0; b < num_seqs; ++b) {
+      const int P = seq_prefix_tokens_host[b];
+      const int L = context_lens_host[b];
+      // a prefix length the kernels reject counts as 0 (they flag it)
+      const int rest = (P > 0 && P % block_size == 0 && P <= L - 1) ? L - P : L;
+      max_suffix = rest > max_suffix ? rest : max_suffix;
+    }
+  }
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(staging);
+  const size_t B = (size_t)num_seqs, H = (size_t)num_heads, Hk = (size_t)num_kv_heads,
+               D = (size_t)head_dim;
+  // 1. the step's inputs, host to device (small arrays first)
+  if ((st = h2d(base + lay.tables, block_tables_host, B * max_blocks_per_seq * 4, s,
+                "block table upload")) != PAGEDKV_OK ||
+      (st = h2d(base + lay.lens, context_lens_host, B * 4, s, "context length upload")) !=
+          PAGEDKV_OK ||
+      (st = h2d(base + lay.pairs, copy_pairs_host, (size_t)num_pairs * 16, s, "pair upload")) !=
+          PAGEDKV_OK)
+    return st;
+  if (shared &&
+      ((st = h2d(base + lay.prefix, seq_prefix_tokens_host, B * 4, s, "prefix upload")) !=
+           PAGEDKV_OK ||
+       (st = h2d(base + lay.groups, groups_host, (size_t)num_groups * GROUP_WIDTH * 4, s,
+                 "group upload")) != PAGEDKV_OK))
+    return st;
+  if ((st = h2d(base + lay.q, q_host, B * H * D * 2, s, "query upload")) != PAGEDKV_OK ||
+      (st = h2d(base + lay.k, k_new_host, B * Hk * D * 2, s, "new K upload")) != PAGEDKV_OK ||
+      (st = h2d(base + lay.v, v_new_host, B * Hk * D * 2, s, "new V upload")) != PAGEDKV_OK)
+    return st;
+  // 2. copy-on-write copies before any write into their destinations
+  if (num_pairs > 0) {
+    void* kc[1] = {key_cache};
+    void* vc[1] = {value_cache};
+    st = copy_blocks(kc, vc, reinterpret_cast<const int64_t*>(base + lay.pairs), num_pairs, 1,
+                     (size_t)num_kv_heads * block_size * head_dim, num_blocks, stream);
+    if (st != PAGEDKV_OK) return st;
+  }
+  if (num_seqs == 0) return PAGEDKV_OK;
+  // 3. new rows written at position L - 1, then the attention over the updated cache
+  void* ws = lay.ws_bytes ? base + lay.ws : nullptr;
+  const int32_t* tables = reinterpret_cast<const int32_t*>(base + lay.tables);
+  const int32_t* lens = reinterpret_cast<const int32_t*>(base + lay.lens);
+  if (shared) {
+    st = paged_attention_decode_shared_prefix(
+        base + lay.out, base + lay.q, base + lay.k, base + lay.v, key_cache, value_cache, tables,
+        lens, reinterpret_cast<const int32_t*>(base + lay.prefix),
+        num_groups ? reinterpret_cast<const int32_t*>(base + lay.groups) : nullptr, num_groups,
+        max_prefix, max_suffix, scale, block_size, num_kv_heads, num_seqs, num_heads, head_dim,
+        max_blocks_per_seq, num_blocks, max_context_len, partition_size, ws, lay.ws_bytes, stream);
+  } else {
+    st = paged_attention_decode_append(base + lay.out, base + lay.q, base + lay.k, base + lay.v,
+                                       key_cache, value_cache, tables, lens, scale, block_size,
+                                       num_kv_heads, num_seqs, num_heads, head_dim,
+                                       max_blocks_per_seq, num_blocks, max_context_len,
+                                       partition_size, ws, lay.ws_bytes, stream);
+  }
+  if (st != PAGEDKV_OK) return st;
+  // 4. the output back to the host
+  const cudaError_t e =
+      cudaMemcpyAsync(out_host, base + lay.out, B * H * D * 2, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "output download");
   return PAGEDKV_OK;
 }
 

@@ -45,6 +45,7 @@ class LayeredDecodeStep:
         # the layers run in order on one stream, so they share one workspace
         self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.graph = None
+        self._inputs_set = False
 
     def _layers(self):
         for l in range(self.num_layers):
@@ -55,7 +56,10 @@ class LayeredDecodeStep:
 
     def capture(self):
         """Captures the per-layer launches (after one eager run that sets up the kernels).
-        The eager run writes the current inputs' new rows, as a replay would."""
+        The eager run writes the current inputs' new rows, as a replay would, so the
+        inputs must be set first (set_inputs): the placeholder tables hold no blocks."""
+        if not self._inputs_set:
+            raise RuntimeError("set_inputs() before capture(): the set-up run reads the tables")
         self._layers()
         self.stream.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -70,6 +74,8 @@ class LayeredDecodeStep:
                              (self.block_tables, block_tables), (self.context_lens, context_lens)):
                 if src is not None:
                     dst.copy_(src, non_blocking=True)
+        if block_tables is not None and context_lens is not None:
+            self._inputs_set = True
 
     def replay(self, pairs=None):
         """One decode step: copy-on-write copies (pairs [n][2] int64, device or None) over every

@@ -223,3 +223,54 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(nat, "library_path", lambda: str(tmp_path / "libpagedkv.so"))
     with pytest.raises(nat.PagedKVError, match="no CPU fallback"):
         nat.load_library()
+
+
+def _host_step(lib, lens, pairs=None, staging_bytes=None, staging=FAKE, maxlen=100, max_pairs=4,
+               pre=None, groups=None, ng=0, B=None):
+    """paged_decode_step_host with real host arrays and fake device pointers: every refusal
+    below happens on the host, before any CUDA call."""
+    import numpy as np
+    lens = np.ascontiguousarray(lens, np.int32)
+    B = len(lens) if B is None else B
+    H, Hk, D, bs, maxblk, N = 8, 8, 64, 16, 8, 64
+    tables = np.zeros((max(B, 1), maxblk), np.int32)
+    pr = np.ascontiguousarray(pairs if pairs is not None else np.zeros((0, 2)), np.int64)
+    need = lib.paged_decode_step_staging_bytes(B, H, Hk, D, bs, maxblk, maxlen, 0, max_pairs,
+                                               int(pre is not None))
+    return lib.paged_decode_step_host(
+        FAKE, FAKE, FAKE, FAKE, tables.ctypes.data, lens.ctypes.data,
+        pr.ctypes.data if len(pr) else None, len(pr),
+        None if pre is None else np.ascontiguousarray(pre, np.int32).ctypes.data,
+        None if groups is None else np.ascontiguousarray(groups, np.int32).ctypes.data, ng,
+        FAKE, FAKE, 0.125, bs, Hk, B, H, D, maxblk, N, maxlen, 0, max_pairs, staging,
+        need if staging_bytes is None else staging_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(lens=[5, 0]), nat.EINVAL),                          # a context length below 1
+    (dict(lens=[5, 101]), nat.EINVAL),                        # beyond max_context_len
+    (dict(lens=[5, 7], pairs=[[1, 2], [3, 1]]), nat.EINVAL),  # a destination used as a source
+    (dict(lens=[5, 7], pairs=[[1, 2], [3, 2]]), nat.EINVAL),  # a destination repeated
+    (dict(lens=[5, 7], pairs=[[1, 64]]), nat.EINVAL),         # outside the pool
+    (dict(lens=[5, 7], pairs=[[1, 2]] * 5), nat.EINVAL),      # more than max_pairs
+    (dict(lens=[5, 7], staging_bytes=1024), nat.EWORKSPACE),
+    (dict(lens=[5, 7], staging=FAKE + 16), nat.EINVAL),       # staging not 256-byte aligned
+    (dict(lens=[5, 7], pre=[0, 0], ng=3), nat.EINVAL),        # more groups than num_seqs / 2
+])
+def test_host_step_rejects_bad_host_inputs(lib, kw, code):
+    assert _host_step(lib, **kw) == code
+    assert lib.pagedkv_last_error().decode()
+
+
+def test_host_step_staging_bytes(lib):
+    f = lib.paged_decode_step_staging_bytes
+    r = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    B, H, Hk, D, bs, maxblk, maxlen = 256, 32, 32, 128, 16, 96, 1524
+    ws = lib.paged_attention_workspace_bytes(B, H, Hk, D, bs, maxlen, 0)
+    want = (r(B * H * D * 2) * 2 + r(B * Hk * D * 2) * 2 + r(B * maxblk * 4) + r(B * 4) +
+            r(224 * 16) + r(ws))
+    assert f(B, H, Hk, D, bs, maxblk, maxlen, 0, 224, 0) == want
+    ws2 = lib.paged_attention_shared_prefix_workspace_bytes(B, H, Hk, D, bs, maxlen, 0)
+    assert f(B, H, Hk, D, bs, maxblk, maxlen, 0, 224, 1) == \
+        want - r(ws) + r(B * 4) + r(B // 2 * 9 * 4) + r(ws2)
+    assert f(B, H, Hk, 96, bs, maxblk, maxlen, 0, 0, 0) == 0    # rejected head_dim

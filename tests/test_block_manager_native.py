@@ -169,7 +169,7 @@ def test_concurrent_callers_keep_counts_consistent():
 
 def test_block_size_trade_off_on_the_llama7b_batch():
     # smaller blocks: less tail waste, longer tables, more allocations per append
-    from paged_kv_cache_393_b200 import bm_bench
+    import bm_bench
     r = {bs: bm_bench.run(bs, steps=20) for bs in (8, 16, 32, 64)}
     waste = [r[bs]["tail_waste"] for bs in (8, 16, 32, 64)]
     entries = [r[bs]["table_entries"] for bs in (8, 16, 32, 64)]

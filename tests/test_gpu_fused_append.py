@@ -62,7 +62,7 @@ def test_query_groups_split_over_ctas_write_one_row(pkv):
 
 
 def _edge_batch(H=4, Hk=4):
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     return PagedBatch(_fixed("edge_fused", H, Hk, 64, 16, [5, 40, 17]), DEV)
 
 
@@ -105,7 +105,7 @@ def test_fused_arguments_are_checked(pkv):
 def test_cow_workload_fused(pkv):
     # copy-on-write step then the fused call, for all decode steps; afterwards the cache
     # rows of chosen samples and their attention match the oracle
-    from paged_kv_cache_393_b200.batch import CowBatch
+    from batches import CowBatch
     from oracle_side import compact_pools
     w = wl.get("cow")
     Hk, D, bs, N = w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks

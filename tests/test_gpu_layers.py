@@ -34,7 +34,7 @@ def _layer_seed(w, l):
 
 
 def _build(pkv, w, layers):
-    from paged_kv_cache_393_b200.batch import PagedBatch, sentinel_pools
+    from batches import PagedBatch, sentinel_pools
     gb = PagedBatch(w, DEV)                       # tables, lengths and layer 0's pools
     lens = gb.lens_host
     kcs, vcs = [gb.key_cache], [gb.value_cache]
@@ -121,3 +121,16 @@ def test_copy_on_write_pairs_reach_every_layer(pkv):
         # the copied block equals the oracle's; the step's new rows are written elsewhere
         assert np.array_equal(got_k[dst], ek[0].view(np.uint16)[dst])
         assert np.array_equal(got_v[dst], ev[0].view(np.uint16)[dst])
+
+
+def test_capture_needs_the_inputs_first(pkv):
+    # the capture's set-up run reads the tables: with the placeholders it would raise
+    # device error bits the caller never caused, so capture() refuses instead
+    w = _fixed("layers_capture", 4, 4, 64, 16, [40, 70], slack=8)
+    gb, kcs, vcs = _build(pkv, w, 2)
+    step = pkv.LayeredDecodeStep(kcs, vcs, w.num_seqs, w.num_heads, gb.max_blocks,
+                                 gb.max_context_len, w.scale)
+    with pytest.raises(RuntimeError, match="set_inputs"):
+        step.capture()
+    torch.cuda.synchronize()
+    assert pkv.device_errors() == 0

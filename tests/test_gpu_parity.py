@@ -40,7 +40,7 @@ def _bits(t):
 
 
 def _run_and_compare(pkv, w, partition_size=0, sample=None, check_pool=True, fused=False):
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     gb = PagedBatch(w, DEV)
     ob = OracleBatch(w, sample)
     # the product block manager and the oracle's model agree exactly
@@ -130,7 +130,7 @@ def test_small_cases(pkv, w, part):
 
 def test_single_pass_and_split_agree(pkv):
     w = _fixed("agree", 8, 2, 128, 16, [100, 1000, 2049])
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     gb = PagedBatch(w, DEV)
     pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
     outs = []
@@ -144,7 +144,7 @@ def test_single_pass_and_split_agree(pkv):
 
 def test_deterministic(pkv):
     w = _fixed("det", 8, 8, 128, 16, [33, 400])
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     gb = PagedBatch(w, DEV)
     pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
     res = []
@@ -168,7 +168,7 @@ def test_block_table_figure_on_the_gpu(pkv):
     kc_h, vc_h = oracle.reshape_and_cache(wl.sentinel_pool(N, 1, bs, D), wl.sentinel_pool(N, 1, bs, D),
                                           k, v, slots, bs)
     ref = oracle.paged_attention(q, kc_h, vc_h, [table], [12], 0.125, bs, 1)
-    from paged_kv_cache_393_b200.batch import sentinel_pools
+    from batches import sentinel_pools
     kc, vc = sentinel_pools(N, 1, bs, D, DEV)
     pkv.reshape_and_cache(torch.from_numpy(k).to(DEV), torch.from_numpy(v).to(DEV), kc, vc,
                           torch.from_numpy(slots).to(DEV))
@@ -182,7 +182,7 @@ def test_block_table_figure_on_the_gpu(pkv):
 
 def test_context_of_one_is_exactly_v(pkv):
     w = _fixed("len1", 8, 2, 128, 16, [1, 1, 1])
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     gb = PagedBatch(w, DEV)
     pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
     pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
@@ -223,7 +223,7 @@ def test_gqa_full_size_automatic_split(pkv):
 # ---- copy-on-write workload ---------------------------------------------------------
 
 def test_cow_workload(pkv):
-    from paged_kv_cache_393_b200.batch import CowBatch
+    from batches import CowBatch
     w = wl.get("cow")
     Hk, D, bs, N = w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks
     gb = CowBatch(w, DEV)
@@ -311,7 +311,7 @@ def test_cow_workload(pkv):
 # ---- edge cases and device-side checks ----------------------------------------------
 
 def _tiny_batch():
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     import paged_kv_cache_393_b200 as m
     gb = PagedBatch(_fixed("edge", 4, 4, 64, 16, [5, 40, 17]), DEV)
     m.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
@@ -352,7 +352,7 @@ def test_bad_block_id_is_flagged_not_faulted(pkv):
                                gb.context_lens, 0.125, gb.max_context_len)
     assert pkv.device_errors() & pkv.DEVERR_BLOCK_ID
     # the mma kernel's producer checks the same way
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     g2 = PagedBatch(_fixed("edge_gqa", 8, 2, 64, 16, [20, 40]), DEV)
     t2 = g2.block_tables.clone()
     t2[0, 1] = 1 << 30

@@ -36,7 +36,7 @@ class ForkBatch:
 
     def __init__(self, pkv, H, Hk, D, bs, prompts, samples, extra, seed=3000):
         from paged_kv_cache_393_b200 import BlockManager
-        from paged_kv_cache_393_b200.batch import sentinel_pools
+        from batches import sentinel_pools
         self.H, self.Hk, self.D, self.bs = H, Hk, D, bs
         total = len(prompts) * samples
         N = sum(-(-L // bs) for L in prompts) + total * (max(extra(i) for i in range(total)) // bs + 3)
@@ -247,7 +247,7 @@ def test_inconsistent_groups_are_flagged_not_faulted(pkv):
 def test_cow_workload_shared_prefix(pkv):
     # all 200 decode steps of the copy-on-write workload through the fused shared-prefix
     # call; afterwards the chosen samples' cache rows and attention match the oracle
-    from paged_kv_cache_393_b200.batch import CowBatch
+    from batches import CowBatch
     w = wl.get("cow")
     Hk, D, bs, N = w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks
     gb = CowBatch(w, DEV)
@@ -300,12 +300,12 @@ def test_decode_session_with_shared_prefixes(pkv, H, Hk):
     # the host-buffer call: inputs from pinned host memory, groups built on the host per step
     fb = ForkBatch(pkv, H, Hk, 128, 16, [700, 90], 4, lambda i: (11 * i) % 30)
     sess = pkv.DecodeSession(fb.kc, fb.vc, len(fb.seqs), H, fb.max_blocks, fb.max_context_len,
-                             shared_prefix=True)
+                             scale=1.0 / 128 ** 0.5, shared_prefix=True)
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
     out = torch.empty((len(fb.seqs), H, 128), dtype=torch.float16).pin_memory()
     kn = np.stack([a for a, _ in fb.new])
     vn = np.stack([b for _, b in fb.new])
-    sess.step(pin(fb.q_host), pin(kn), pin(vn), None, pin(fb.tables_host), pin(fb.lens_host), out)
+    sess.step(pin(fb.q_host), pin(kn), pin(vn), pin(fb.tables_host), pin(fb.lens_host), out)
     torch.cuda.synchronize()
     assert pkv.device_errors() == 0
     # 4 samples per prompt: one group each with MHA, two of 2 members with 4 heads per kv head

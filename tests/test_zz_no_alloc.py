@@ -55,7 +55,7 @@ CASES = [
 @pytest.mark.parametrize("w,part", CASES, ids=[c[0].name for c in CASES])
 def test_matches_the_regular_entry_point_twice(lib, w, part):
     import paged_kv_cache_393_b200 as pkv
-    from paged_kv_cache_393_b200.batch import PagedBatch
+    from batches import PagedBatch
     gb = PagedBatch(w, DEV)
     pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
     ref = torch.empty_like(gb.out)

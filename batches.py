@@ -39,11 +39,10 @@ def _write_tokens(kc, vc, k, v, slots, device):
 class PagedBatch:
     """One decode step of a fixed-length workload (tiny, llama7b, bs_sweep_*, gqa)."""
 
-    def __init__(self, w: wl.Workload, device, prefill_chunk_tokens: int = 1 << 17):
+    def __init__(self, w: wl.Workload, device, prefill_chunk_tokens: int = 1 << 17, _defer=False):
         self.w = w
         self.device = torch.device(device)
-        B, H, Hk, D, bs, N = (w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
-                              w.num_blocks)
+        B, Hk, D, bs, N = w.num_seqs, w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks
         self.lens_host = wl.context_lens(w)
         self.max_context_len = int(self.lens_host.max())
         self.max_blocks = -(-self.max_context_len // bs)
@@ -55,42 +54,75 @@ class PagedBatch:
             if s is None:
                 raise MemoryError("pool of %d blocks too small for the workload" % N)
             self.seqs.append(s)
-        # prefill the prompts (every token but the last) in chunks of sequences
-        new_k = np.empty((B, Hk, D), np.float16)
-        new_v = np.empty((B, Hk, D), np.float16)
-        b0 = 0
-        while b0 < B:
-            b1, tok = b0, 0
-            while b1 < B and (b1 == b0 or tok + int(self.lens_host[b1]) <= prefill_chunk_tokens):
-                tok += int(self.lens_host[b1])
-                b1 += 1
-            kvs = wl.sequences_kv(w.seed, range(b0, b1), self.lens_host[b0:b1], Hk, D)
-            ks, vs, slots = [], [], []
-            for j, b in enumerate(range(b0, b1)):
-                k, v = kvs[j]
-                L = int(self.lens_host[b])
-                ks.append(k[:L - 1])
-                vs.append(v[:L - 1])
-                slots.append(self.bm.seq_slots(self.seqs[b], 0, L - 1))
-                new_k[b], new_v[b] = k[L - 1], v[L - 1]
-            _write_tokens(self.key_cache, self.value_cache, np.concatenate(ks), np.concatenate(vs),
-                          np.concatenate(slots), self.device)
-            b0 = b1
-        # the decode step: one new token per sequence
+        self.k_new_host = np.empty((B, Hk, D), np.float16)
+        self.v_new_host = np.empty((B, Hk, D), np.float16)
+        if not _defer:
+            _prefill([self], prefill_chunk_tokens)
+            self._finish()
+
+    def _write_prompts(self, b0, kvs):
+        """Writes every token but the last of sequences b0, b0+1, ... (K/V rows kvs)."""
+        ks, vs, slots = [], [], []
+        for j, (k, v) in enumerate(kvs):
+            b = b0 + j
+            L = int(self.lens_host[b])
+            ks.append(k[:L - 1])
+            vs.append(v[:L - 1])
+            slots.append(self.bm.seq_slots(self.seqs[b], 0, L - 1))
+            self.k_new_host[b], self.v_new_host[b] = k[L - 1], v[L - 1]
+        _write_tokens(self.key_cache, self.value_cache, np.concatenate(ks), np.concatenate(vs),
+                      np.concatenate(slots), self.device)
+
+    def _finish(self):
+        """The decode step: one new token per sequence."""
+        w, dev = self.w, self.device
+        B = w.num_seqs
         self.slots_host = self.bm.append_tokens(self.seqs)
         assert len(self.slots_host) == B
         self.tables_host, lens = self.bm.build_batch(self.seqs, self.max_blocks)
         assert np.array_equal(lens, self.lens_host)
-        self.q_host = wl.decode_q(w.seed, 0, B, H, D)
-        self.k_new_host, self.v_new_host = new_k, new_v
-        dev = self.device
+        self.q_host = wl.decode_q(w.seed, 0, B, w.num_heads, w.head_dim)
         self.q = torch.from_numpy(self.q_host).to(dev)
-        self.k_new = torch.from_numpy(new_k).to(dev)
-        self.v_new = torch.from_numpy(new_v).to(dev)
+        self.k_new = torch.from_numpy(self.k_new_host).to(dev)
+        self.v_new = torch.from_numpy(self.v_new_host).to(dev)
         self.slots = torch.from_numpy(self.slots_host).to(dev)
         self.block_tables = torch.from_numpy(self.tables_host).to(dev)
         self.context_lens = torch.from_numpy(self.lens_host).to(dev)
-        self.out = torch.empty((B, H, D), dtype=torch.float16, device=dev)
+        self.out = torch.empty((B, w.num_heads, w.head_dim), dtype=torch.float16, device=dev)
+
+
+def _prefill(batches, chunk_tokens):
+    """Writes the prompts of every batch, drawing each sequence's K/V values once (the
+    batches differ only in block size and pool)."""
+    w = batches[0].w
+    lens = batches[0].lens_host
+    B = w.num_seqs
+    b0 = 0
+    while b0 < B:
+        b1, tok = b0, 0
+        while b1 < B and (b1 == b0 or tok + int(lens[b1]) <= chunk_tokens):
+            tok += int(lens[b1])
+            b1 += 1
+        kvs = wl.sequences_kv(w.seed, range(b0, b1), lens[b0:b1], w.num_kv_heads, w.head_dim)
+        for gb in batches:
+            gb._write_prompts(b0, kvs)
+        b0 = b1
+
+
+def paged_batches(ws, device, prefill_chunk_tokens: int = 1 << 17):
+    """PagedBatch of several workloads that differ only in block size and pool size (the
+    block-size sweep: the same tokens, K/V values and lengths), from one draw of the values."""
+    ref = ws[0]
+    for w in ws:
+        if (w.seed, w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.lens, w.len_lo,
+                w.len_hi) != (ref.seed, ref.num_seqs, ref.num_heads, ref.num_kv_heads,
+                              ref.head_dim, ref.lens, ref.len_lo, ref.len_hi):
+            raise ValueError("paged_batches needs workloads that differ only in block size")
+    out = [PagedBatch(w, device, _defer=True) for w in ws]
+    _prefill(out, prefill_chunk_tokens)
+    for gb in out:
+        gb._finish()
+    return out
 
     @property
     def scale(self) -> float:

@@ -40,6 +40,9 @@ import workloads as wl  # noqa: E402
 METRIC = "paged decode attention KV GB/s (% of B200 HBM peak) and decode tokens/s"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+# The nominal B200 HBM3e bandwidth (~8 TB/s) the target is stated against; the roofline
+# fractions use the measured copy bandwidth instead (a read-only stream can exceed a copy).
+NOMINAL_HBM_GBS = 8000.0
 
 
 def parse_args(argv=None):
@@ -62,6 +65,11 @@ def parse_args(argv=None):
                          "the workload's), run as one CUDA graph (LayeredDecodeStep)")
     ap.add_argument("--partition-size", type=int, default=None,
                     help="split-K partition size (default: the workload's)")
+    ap.add_argument("--no-sub-results", action="store_true",
+                    help="default llama7b run: skip the other workloads' lines (block-size sweep, "
+                         "gqa, cow shared-prefix step)")
+    ap.add_argument("--sub-steps", type=int, default=300,
+                    help="timed steps of each sub-result workload")
     ap.add_argument("--eager", action="store_true",
                     help="cow workload: launch every step from Python instead of replaying "
                          "one CUDA graph per step")
@@ -233,33 +241,23 @@ def recorded_traffic(kernel_file: str, workload: str):
 
 # ---- the CUDA arm ------------------------------------------------------------------------
 
-def run_ours(args):
+def time_decode(gb, part, step_kind, K, warmup, dev, stream, world, local):
+    """Times K decode steps of a PagedBatch on `stream`: the fused append + attention call
+    (step_kind "fused"), or reshape_and_cache then paged_attention_decode ("separate"),
+    plus the split-K merge when the plan splits.  CUDA events bracket the attention call
+    of every step; clocks are sampled over the timed region."""
     import torch
 
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    init_dist("nccl", world, local)
-    dev = torch.device("cuda", local)
     import paged_kv_cache_393_b200 as pkv
-    from batches import PagedBatch
-    pkv.load_library()
-    w = wl.get(args.workload)
-    if w.lens == "cow":
-        return run_cow(args, w, dev, world, rank, local)
-    if args.layers > 1:
-        return run_layers(args, w, dev, world, rank, local)
-    gb = PagedBatch(w, dev)
-    part = w.partition_size if args.partition_size is None else args.partition_size
+    w = gb.w
     B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
     need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len, part)
-    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.Stream(dev)
+    ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
     # split-K (a merge kernel and partial bytes) only when the plan partitions the contexts;
     # the tensor-core path needs a workspace word even in a single pass
-    splits = pkv.paged_attention_partition_tokens(B, H, Hk, D, w.block_size, gb.max_context_len,
-                                                  part) > 0
-    fused = args.step == "fused"
-    launches_per_step = (1 if fused else 2) + (1 if splits else 0)   # [reshape,] attention[, merge]
+    pt = pkv.paged_attention_partition_tokens(B, H, Hk, D, w.block_size, gb.max_context_len, part)
+    fused = step_kind == "fused"
+    launches_per_step = (1 if fused else 2) + (1 if pt > 0 else 0)   # [reshape,] attention[, merge]
     G = H // Hk
     kernel_file = "attention_mma.cu" if (2 <= G <= 8 and w.block_size >= 8) else "attention_simt.cu"
 
@@ -278,13 +276,12 @@ def run_ours(args):
             pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots,
                                   stream=stream)
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         cache_update()
         attention()
     torch.cuda.synchronize(dev)
     pkv.device_errors(clear=True)
 
-    K = args.steps
     ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -308,29 +305,92 @@ def run_ours(args):
     clocks = sampler.stop()
     flags = pkv.device_errors(clear=True)
     if flags:
-        raise SystemExit("device error flags %#x during the timed steps" % flags)
+        raise SystemExit("device error flags %#x during the timed steps (%s)" % (flags, w.name))
 
-    ms_total = t0.elapsed_time(t1)
     attn_ms = sum(a.elapsed_time(b) for a, b in ev_a) / K
     kv_bytes = gb.kv_bytes()
-    ms_max, kv_all = aggregate(ms_total, float(kv_bytes) * K, world, dev)
+    # the attention call's algorithmic bytes per launch: K+V rows read, q read, out
+    # written, table entries and lengths read, new rows, split partials written and read
+    nblk = (gb.lens_host + w.block_size - 1) // w.block_size
+    attn_bytes = kv_bytes + 2 * B * H * D * 2 + int(nblk.sum()) * 4 + B * 4
+    if fused:
+        attn_bytes += 2 * B * Hk * D * 2 * 2
+    # (the split-K partials are the implementation's own traffic, not the method's: they
+    # are reported apart and left out of the algorithmic bytes)
+    partial_bytes = 0
+    if pt > 0:
+        parts = (gb.lens_host + pt - 1) // pt
+        partial_bytes = int(parts[parts > 1].sum()) * H * (D + 2) * 4 * 2
+    return {"ms_total": t0.elapsed_time(t1), "K": K, "attn_ms": attn_ms, "kv_bytes": kv_bytes,
+            "attn_bytes": attn_bytes, "partial_bytes": partial_bytes,
+            "launches": K * launches_per_step, "clocks": clocks, "kernel_file": kernel_file,
+            "partition_tokens": pt}
+
+
+def roofline_of(res, workload):
+    peak, peak_kind = hbm_peak()
+    achieved = res["attn_bytes"] / (res["attn_ms"] / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": res["kernel_file"].replace(".cu", ""),
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+            "traffic": recorded_traffic(res["kernel_file"], workload),
+            "algorithmic_bytes": res["attn_bytes"], "split_partial_bytes": res["partial_bytes"],
+            "avg_launch_ms": round(res["attn_ms"], 5)}
+
+
+def sub_entry(w, res, step_kind):
+    """One sub-result: a workload's own device-timed line (K+V GB/s, its roofline, clocks)."""
+    ms = res["ms_total"] / res["K"]
+    return {"workload": describe(w), "step": step_kind, "steps": res["K"],
+            "ms_per_step": round(ms, 5),
+            "value": round(res["kv_bytes"] / (ms / 1e3) / 1e9, 2), "unit": UNIT,
+            "tokens_per_s": round(w.num_seqs / (ms / 1e3), 1),
+            "pct_of_hbm_peak": round(100 * res["kv_bytes"] / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS, 2),
+            "partition_tokens": res["partition_tokens"],
+            "roofline": roofline_of(res, w.name), "gpu_launches": res["launches"],
+            "clocks": res["clocks"]}
+
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    init_dist("nccl", world, local)
+    dev = torch.device("cuda", local)
+    import paged_kv_cache_393_b200 as pkv
+    from batches import PagedBatch, paged_batches
+    pkv.load_library()
+    w = wl.get(args.workload)
+    if w.lens == "cow":
+        line = measure_cow(args, w, dev, world, rank, local, args.step, args.steps,
+                           min(args.e2e_steps, w.decode_steps, 50))
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    if args.layers > 1:
+        return run_layers(args, w, dev, world, rank, local)
+    # the default run also reports the other workloads (sub_results) on one GPU
+    subs = args.workload == "llama7b" and world == 1 and not args.no_sub_results
+    if subs:
+        # block-size sweep: the llama7b tokens and values at block sizes 8/16/32/64, drawn once
+        sweep = paged_batches([wl.bs_sweep(8), w, wl.bs_sweep(32), wl.bs_sweep(64)], dev)
+        gb = sweep[1]
+    else:
+        sweep = []
+        gb = PagedBatch(w, dev)
+    part = w.partition_size if args.partition_size is None else args.partition_size
+    B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
+    stream = torch.cuda.Stream(dev)
+    K = args.steps
+    res = time_decode(gb, part, args.step, K, args.warmup, dev, stream, world, local)
+    kv_bytes = res["kv_bytes"]
+    ms_max, kv_all = aggregate(res["ms_total"], float(kv_bytes) * K, world, dev)
     ms_per_step = ms_max / K
     value = kv_all / (ms_max / 1e3) / 1e9
-
-    # roofline of the attention kernel: its algorithmic bytes per launch
-    # (K+V rows read, q read, out written, table entries and lengths read)
-    nblk = (gb.lens_host + w.block_size - 1) // w.block_size
-    attn_bytes = (kv_bytes + 2 * B * H * D * 2 + int(nblk.sum()) * 4 + B * 4)
-    if fused:
-        attn_bytes += 2 * B * Hk * D * 2 * 2    # new K/V rows read and written
-    if splits:
-        pt = pkv.paged_attention_partition_tokens(B, H, Hk, D, w.block_size, gb.max_context_len,
-                                                  part)
-        parts = (gb.lens_host + pt - 1) // pt
-        attn_bytes += int(parts.sum()) * H * (D + 2) * 4 * 2    # partials written + read
-    peak, peak_kind = hbm_peak()
-    achieved = attn_bytes / (attn_ms / 1e3) / 1e9
-    traffic = recorded_traffic(kernel_file, args.workload)
 
     # end to end through the public API: host buffers in, host result out
     e2e = None
@@ -358,12 +418,37 @@ def run_ours(args):
         e2e = {"value": round(e_bytes / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
                "ms_per_step": round(e_ms / E, 4), "call": "paged_decode_step_host",
                "h2d_bytes_per_step": sess.h2d_bytes(), "d2h_bytes_per_step": sess.d2h_bytes()}
+        del sess
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
+    sub_results = None
+    if subs:
+        KS = max(args.sub_steps, 3)
+        sub_results = []
+        for g in sweep:
+            r = res if g is gb and K >= KS else time_decode(g, part, args.step, KS, args.warmup,
+                                                              dev, stream, world, local)
+            sub_results.append(sub_entry(g.w, r, args.step))
+        del g, sweep, gb
+        torch.cuda.empty_cache()
+        gq = PagedBatch(wl.get("gqa"), dev)
+        r = time_decode(gq, gq.w.partition_size, args.step, KS, args.warmup, dev, stream, world,
+                        local)
+        sub_results.append(sub_entry(gq.w, r, args.step))
+        del gq, r
+        torch.cuda.empty_cache()
+        cow = measure_cow(args, wl.get("cow"), dev, world, rank, local, "shared",
+                          max(KS, 200), 0)
+        sub_results.append({k: cow[k] for k in (
+            "workload", "step", "steps", "ms_per_step", "value", "unit", "tokens_per_s",
+            "unique_kv_GB_per_s", "roofline", "copy_blocks", "gpu_launches", "clocks")})
+        torch.cuda.empty_cache()
+
     if rank == 0:
+        peak, _ = hbm_peak()
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
@@ -378,16 +463,15 @@ def run_ours(args):
                 "parallelism": "replicas x%d" % world},
             "tokens_per_s": round(B * world / (ms_per_step / 1e3), 1),
             "steps_per_s": round(1e3 / ms_per_step, 2),
-            "roofline": {"bound": "hbm", "kernel": kernel_file.replace(".cu", ""),
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                         "traffic": traffic, "algorithmic_bytes": attn_bytes,
-                         "avg_launch_ms": round(attn_ms, 5)},
-            "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-            "gpu_launches": K * launches_per_step,
-            "clocks": clocks,
+            "roofline": roofline_of(res, args.workload),
+            "pct_of_hbm_peak": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+            "hbm_peak_nominal_gbs": NOMINAL_HBM_GBS,
+            "pct_of_measured_copy_peak": round(100 * value / world / peak, 2),
+            "gpu_launches": res["launches"],
+            "clocks": res["clocks"],
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "sub_results": sub_results,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -474,13 +558,13 @@ def run_layers(args, w, dev, world, rank, local):
         dist.destroy_process_group()
 
 
-def run_cow(args, w, dev, world, rank, local):
+def measure_cow(args, w, dev, world, rank, local, step_kind, K, e2e_steps):
     """The copy-on-write workload: 32 prompts of 1000 tokens forked into 8 samples,
     then decode steps.  Step 0 copies the 224 shared partial tail blocks
     (copy_blocks) before its scatter and attention; the steps are replayed in
     order.  Replays do the same work; their cache contents may differ (a replayed
     step-0 copy overwrites later rows of the copied blocks), which the timing
-    does not depend on."""
+    does not depend on.  Returns the workload's JSON line (a dict)."""
     import numpy as np
     import torch
 
@@ -490,7 +574,7 @@ def run_cow(args, w, dev, world, rank, local):
     B, H, Hk, D = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim
     steps_host = [gb.prepare_step() for _ in range(w.decode_steps)]
     up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
-    shared = args.step == "shared"
+    shared = step_kind == "shared"
     steps = []
     unique_total = 0
     for h in steps_host:
@@ -536,7 +620,7 @@ def run_cow(args, w, dev, world, rank, local):
                 st["groups"], w.scale, gb.max_context_len, cpart, ws, k_new=st["k"], v_new=st["v"],
                 stream=stream, max_prefix_tokens=st["max_prefix"],
                 max_suffix_tokens=st["max_suffix"])
-        elif args.step == "fused":
+        elif step_kind == "fused":
             pkv.paged_attention_decode_append(out, st["q"], st["k"], st["v"], gb.key_cache,
                                               gb.value_cache, st["tables"], st["lens"], w.scale,
                                               gb.max_context_len, cpart, ws, stream=stream)
@@ -572,7 +656,6 @@ def run_cow(args, w, dev, world, rank, local):
                 run_step(j)
             graphs.append(g)
         torch.cuda.synchronize(dev)
-    K = args.steps
     sampler = ClockSampler(gpu_id_for(local))
     sampler.start()
 
@@ -591,11 +674,13 @@ def run_cow(args, w, dev, world, rank, local):
     t0.record(stream)
     kv_total = 0
     launches = 0
+    copies_total = 0
     h0 = time.perf_counter()
     for i in range(K):
         j = i % w.decode_steps
         if steps[j]["pairs"] is not None:
             launches += 1
+            copies_total += copy_bytes
         replay(j)
         if shared:
             # prefix pass (when there are groups), suffix pass, merge (unless every suffix
@@ -605,7 +690,7 @@ def run_cow(args, w, dev, world, rank, local):
                 (1 if steps[j]["max_suffix"] > pt else 0)
         else:
             # [reshape,] attention, and the merge when the plan splits
-            launches += {"fused": 1, "separate": 2}[args.step] + (1 if plain_split else 0)
+            launches += {"fused": 1, "separate": 2}[step_kind] + (1 if plain_split else 0)
         kv_total += steps[j]["kv_bytes"]
         unique_total += steps[j].get("unique_bytes", 0)
     host_ms = (time.perf_counter() - h0) * 1e3
@@ -625,7 +710,7 @@ def run_cow(args, w, dev, world, rank, local):
     # from the start (copy-on-write pairs at step 0); the host grouping of the shared-prefix
     # step is inside the timed region
     e2e = None
-    E = min(args.e2e_steps, w.decode_steps, 50)
+    E = min(e2e_steps, w.decode_steps)
     if E > 0:
         sess = pkv.DecodeSession(gb.key_cache, gb.value_cache, B, H, gb.max_blocks,
                                  gb.max_context_len, w.scale, cpart, max_pairs=max(n_pairs, 1),
@@ -658,9 +743,12 @@ def run_cow(args, w, dev, world, rank, local):
         e2e = {"value": round(e_bytes / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
                "ms_per_step": round(e_ms / E, 4), "steps": E, "call": "paged_decode_step_host",
                "h2d_bytes_per_step": int(h2d / E), "d2h_bytes_per_step": sess.d2h_bytes()}
-    if rank == 0:
-        peak, peak_kind = hbm_peak()
-        print(json.dumps({
+    peak, peak_kind = hbm_peak()
+    # roofline of the step: the K/V bytes it must read (with shared prefixes: each group's
+    # prefix once) plus the copy-on-write copies, over the device time
+    alg = (unique_total if shared else kv_total) + copies_total
+    achieved = alg * world / (ms_max / 1e3) / 1e9
+    return {
             "metric": METRIC, "value": round(kv_all / (ms_max / 1e3) / 1e9, 2), "unit": UNIT,
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
@@ -669,7 +757,7 @@ def run_cow(args, w, dev, world, rank, local):
                                    "steps replayed in order; K/V bytes counted per sample "
                                    "(shared prefix blocks counted once per reader)" % (
                                        w.prompts, w.prompt_len, w.samples, w.decode_steps),
-                       "seed": w.seed, "step": args.step, "partition_size": cpart,
+                       "seed": w.seed, "step": step_kind, "partition_size": cpart,
                        "l2": "no flush; shared prefix blocks (%d x 128 KiB x 2) "
                              "can hit in L2" % prefix_blocks,
                        "parallelism": "replicas x%d" % world},
@@ -679,13 +767,19 @@ def run_cow(args, w, dev, world, rank, local):
             "copy_blocks": {"pairs": n_pairs, "bytes": copy_bytes, "avg_us": copy_us,
                             "GB_per_s": round(copy_bytes / (copy_us / 1e6) / 1e9, 1) if copy_us else None,
                             "peak": peak, "peak_kind": peak_kind},
+            "roofline": {"bound": "hbm",
+                         "kernel": "mma_prefix + suffix pass" if shared else "attention_simt",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                         "traffic": None, "algorithmic_bytes": int(alg / K),
+                         "scope": "whole step (device time per step), K/V bytes read once "
+                                  "per group prefix plus the copy-on-write copies"},
+            "step": step_kind, "workload": "cow (%d prompts x %d tokens, %d samples each)" % (
+                w.prompts, w.prompt_len, w.samples),
             "gpu_launches": launches, "clocks": clocks, "e2e": e2e, "cpu_baseline": None,
             "launch": "eager" if graphs is None else "one CUDA graph per step",
             "host_issue_ms_per_step": round(host_ms / K, 4),
-        }), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    }
 
 
 # ---- the oracle: cpu_baseline leg and reference arm ---------------------------------------

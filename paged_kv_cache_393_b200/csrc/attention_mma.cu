@@ -19,10 +19,14 @@
 // boxes of the pools viewed as a [N*Hk*bs][D] matrix into a ring of stages of
 // 16 tokens: 16 rows of one block (bs >= 16) or two whole blocks (bs 8).
 // ldmatrix reads the swizzled tiles without bank conflicts (K plain for the A
-// operand of QK^T, V transposed for the A operand of PV).  Each stage has ONE
-// owner warp, (stage index) mod (consumer warps), which consumes every fill of that stage in
-// order; a warp therefore never waits on a barrier phase that a slower warp
-// has not reached yet (parity waits cannot tell phase k from phase k+2).
+// operand of QK^T, V transposed for the A operand of PV).  The ring is split
+// into one sub-ring per consumer warp (stages w, w + NW, w + 2 NW, ... belong
+// to warp w), and chunk j of every work item goes to warp j mod NW: a warp
+// consumes the fills of its own stages in order, so it never waits on a
+// barrier phase that a slower warp has not reached yet (parity waits cannot
+// tell phase k from phase k+2), and which warp sums which chunk -- the fp32
+// summation order -- does not depend on how items are handed out, so results
+// are reproducible run to run.
 // The consumer warps (two: small CTAs, more of them per SM, measured best),
 // each with its own online softmax, merge through shared
 // memory.  Rows past the context are masked out of the scores, and the
@@ -125,27 +129,47 @@ __device__ __forceinline__ void issue_stage(uint32_t kdst, uint32_t full, const 
   }
 }
 
+// Fill counts of the consumer warps' sub-rings: stage (k mod SPW) * NW + w
+// takes warp w's k-th fill, SPW = stages / NW.
+struct RingFills {
+  int n[NW];
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int w = 0; w < NW; ++w) n[w] = 0;
+  }
+  // after an item of nchunks chunks (chunk j went to warp j mod NW)
+  __device__ __forceinline__ void advance(int nchunks) {
+#pragma unroll
+    for (int w = 0; w < NW; ++w) n[w] += (nchunks - w + NW - 1) / NW;
+  }
+};
+
+__device__ __forceinline__ int ring_stage(int k, int warp, int spw) { return (k % spw) * NW + warp; }
+
 // Streams the nchunks chunks of one item (its table row starts at `row`) into
-// the ring, the item's first chunk having global chunk index gc0.  Run by the
-// whole producer warp; lane 0 issues.  With a fused append (new_tok >= 0: the
-// item ends its context, and its token new_tok is the new one) the warp writes
-// the new K/V rows of sequence b, kv head kvh, into their slot before it issues
-// the chunk that reads them.  Returns false (warp-uniform) when it
-// gave up; *issued_end is one past the last global chunk issued.
+// the ring: chunk c goes to warp c mod NW's sub-ring, as that warp's fill
+// base.n[w] + c / NW.  Run by the whole producer warp; lane 0 issues.  With a
+// fused append (new_tok >= 0: the item ends its context, and its token new_tok
+// is the new one) the warp writes the new K/V rows of sequence b, kv head kvh,
+// into their slot before it issues the chunk that reads them.  Returns false
+// (warp-uniform) when it gave up; lane 0's issued.n[w] counts the fills issued
+// to warp w so far.
 template <int D, int BS>
-__device__ bool produce_item(const int32_t* row, int nblk, int nchunks, int gc0, int kvh, int b,
-                             int new_tok, const DecodeParams& p, int* s_ids, uint64_t* bars,
-                             int stages, uint32_t ring, const CUtensorMap* km,
+__device__ bool produce_item(const int32_t* row, int nblk, int nchunks, const RingFills& base,
+                             int kvh, int b, int new_tok, const DecodeParams& p, int* s_ids,
+                             uint64_t* bars, int stages, uint32_t ring, const CUtensorMap* km,
                              const CUtensorMap* vm, uint64_t policy, volatile int* abort_flag,
-                             int lane, int* issued_end) {
+                             int lane, RingFills& issued) {
   using Geo = StageGeom<D>;
   NewRows<D, 1> fresh;
   if (new_tok >= 0) fresh.load(p.k_new, p.v_new, b, p.num_kv_heads, kvh, lane);
+  const int spw = stages / NW;
   // issues chunk c (lane 0 only); false when the wait for a free stage gave up
   auto issue = [&](int c, int w0) -> bool {
-    const int gc = gc0 + c;
-    const int st = gc % stages;
-    const int round = gc / stages;
+    const int w = c % NW;
+    const int k = base.n[w] + c / NW;
+    const int st = ring_stage(k, w, spw);
+    const int round = k / spw;
     if (round > 0 && !mbar_wait(smem_u32(&bars[stages + st]), (round - 1) & 1)) {
       *abort_flag = 1;
       flag_error(p.err, ERR_TIMEOUT);
@@ -153,7 +177,7 @@ __device__ bool produce_item(const int32_t* row, int nblk, int nchunks, int gc0,
     }
     issue_stage<D, BS>(ring + (uint32_t)st * 2 * Geo::TILE_BYTES, smem_u32(&bars[st]), s_ids, w0,
                        c, nblk, kvh, p.num_kv_heads, km, vm, policy);
-    *issued_end = gc + 1;
+    issued.n[w] = k + 1;
     return true;
   };
   bool ok = true;
@@ -197,11 +221,14 @@ __device__ bool produce_item(const int32_t* row, int nblk, int nchunks, int gc0,
   return ok;
 }
 
-// After an abort only the last `stages` fills can still be in flight: let them
-// land before this CTA's shared memory can be handed to another CTA.
-__device__ __forceinline__ void drain_ring(uint64_t* bars, int stages, int issued_end) {
-  for (int c = max(0, issued_end - stages); c < issued_end; ++c)
-    mbar_wait(smem_u32(&bars[c % stages]), (c / stages) & 1);
+// After an abort only the last SPW fills of each sub-ring can still be in
+// flight: let them land before this CTA's shared memory can be handed to
+// another CTA.
+__device__ __forceinline__ void drain_ring(uint64_t* bars, int stages, const RingFills& issued) {
+  const int spw = stages / NW;
+  for (int w = 0; w < NW; ++w)
+    for (int k = max(0, issued.n[w] - spw); k < issued.n[w]; ++k)
+      mbar_wait(smem_u32(&bars[ring_stage(k, w, spw)]), (k / spw) & 1);
 }
 
 // ---- consumer side ---------------------------------------------------------------
@@ -505,10 +532,12 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     const int32_t* row = p.block_tables + (size_t)b * p.max_blocks + tok0 / BS;
     const int new_tok =
         (p.k_new && tok0 + ntok == L && p.context_lens[b] == L) ? ntok - 1 : -1;
-    int issued_end = 0;
-    produce_item<D, BS>(row, nblk, nchunks, 0, kvh, b, new_tok, p, s_ids, bars, stages, ring,
-                        &k_map, &v_map, l2_evict_first_policy(), abort_flag, lane, &issued_end);
-    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued_end);
+    RingFills base, issued;
+    base.reset();
+    issued.reset();
+    produce_item<D, BS>(row, nblk, nchunks, base, kvh, b, new_tok, p, s_ids, bars, stages, ring,
+                        &k_map, &v_map, l2_evict_first_policy(), abort_flag, lane, issued);
+    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued);
     return;
   }
 
@@ -660,10 +689,12 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       prefetch_tensor_map(&k_map);
       prefetch_tensor_map(&v_map);
     }
-    int issued_end = 0;
-    produce_item<D, BS>(ref_row, nblk, nchunks, 0, kvh, first, -1, p, s_ids, bars, stages, ring,
-                        &k_map, &v_map, l2_evict_first_policy(), abort_flag, lane, &issued_end);
-    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued_end);
+    RingFills base, issued;
+    base.reset();
+    issued.reset();
+    produce_item<D, BS>(ref_row, nblk, nchunks, base, kvh, first, -1, p, s_ids, bars, stages,
+                        ring, &k_map, &v_map, l2_evict_first_policy(), abort_flag, lane, issued);
+    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued);
     return;
   }
 
@@ -893,8 +924,9 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       prefetch_tensor_map(&v_map);
     }
     const uint64_t policy = l2_evict_first_policy();
-    int gc = 0;          // global index of the next chunk
-    int issued_end = 0;  // one past the last chunk issued
+    RingFills base, issued;  // fills per consumer warp: before the next item / issued so far
+    base.reset();
+    issued.reset();
     // A ticket is taken when the previous item has been issued: taking them
     // earlier reserves work a CTA cannot start yet and unbalances the end.
     auto next_item = [&](int4* item) {
@@ -938,18 +970,19 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       const int Ls = s_lens[d.x];
       const int new_tok =
           (p.k_new && d.z * pt + d.w == Ls && p.context_lens[d.x] == P + Ls) ? d.w - 1 : -1;
-      if (!produce_item<D, BS>(row, nblk, nchunks, gc, d.y, d.x, new_tok, p, s_ids, bars, stages,
-                               ring, &k_map, &v_map, policy, abort_flag, lane, &issued_end))
+      if (!produce_item<D, BS>(row, nblk, nchunks, base, d.y, d.x, new_tok, p, s_ids, bars,
+                               stages, ring, &k_map, &v_map, policy, abort_flag, lane, issued))
         break;
-      gc += nchunks;
+      base.advance(nchunks);
       have = next_item(&d);
     }
-    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued_end);
+    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued);
     return;
   }
 
   // ---------------- consumer warps ----------------
-  int gc = 0;
+  const int spw = stages / NW;
+  int mine = 0;  // fills of this warp's sub-ring consumed so far
   for (int it = 0;; ++it) {
     const int qs = it % IQ;
     bool stop = false, gave_up = false;
@@ -973,15 +1006,14 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&iempty[qs]));  // descriptor and query tile consumed
       const int nchunks = (d.w + CHUNK - 1) / CHUNK;
-      for (int j = 0; j < nchunks && !gave_up; ++j) {
-        const int c = gc + j;
-        const int st = c % stages;
-        if (st % NW != warp) continue;
+      // chunks warp, warp + NW, ... of the item: this warp's next fills, in order
+      for (int j = warp; j < nchunks; j += NW, ++mine) {
+        const int st = ring_stage(mine, warp, spw);
         if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {
           gave_up = true;
           break;
         }
-        const bool ok = mbar_wait(smem_u32(&bars[st]), (c / stages) & 1);
+        const bool ok = mbar_wait(smem_u32(&bars[st]), (mine / spw) & 1);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) {
             *abort_flag = 1;
@@ -995,7 +1027,6 @@ __global__ void __launch_bounds__((NW + 1) * 32)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars[stages + st]));
       }
-      gc += nchunks;
     }
     // All consumer warps decide together: the end of the work, or an abort anywhere.
     if (named_barrier_or(1, NW * 32, stop || gave_up)) break;

@@ -30,3 +30,18 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Prints the attention error figures the parity tests recorded (shown under -q too)."""
+    try:
+        from oracle_side import ERRORS
+    except ImportError:
+        return
+    if not ERRORS:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "attention vs the fp64 oracle: max abs / max rel error (|ref| > 1e-3)")
+    for name, n, abs_err, rel_err in ERRORS:
+        tr.write_line("%-44s %10d outputs  max abs %.3e  max rel %.3e" % (name, n, abs_err,
+                                                                           rel_err))

@@ -10,9 +10,6 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
-import workloads as wl
-from oracle_side import assert_attention_close
 from test_gpu_parity import DEV, SMALL, _bits, _fixed, _run_and_compare
 
 pytestmark = pytest.mark.gpu
@@ -33,25 +30,6 @@ def pkv():
 @pytest.mark.parametrize("w,part", SMALL, ids=[c[0].name for c in SMALL])
 def test_small_cases_fused(pkv, w, part):
     _run_and_compare(pkv, w, partition_size=part, fused=True)
-
-
-def test_llama7b_full_size_fused(pkv):
-    w = wl.get("llama7b")
-    lens = wl.context_lens(w)
-    _run_and_compare(pkv, w, sample=sorted({0, int(np.argmax(lens)), int(np.argmin(lens)), 255}),
-                     fused=True)
-
-
-def test_gqa_full_size_fused(pkv):
-    w = wl.get("gqa")
-    lens = wl.context_lens(w)
-    _run_and_compare(pkv, w, partition_size=w.partition_size,
-                     sample=sorted({0, int(np.argmax(lens)), int(np.argmin(lens)), 127}), fused=True)
-
-
-@pytest.mark.parametrize("bs", [8, 64])
-def test_block_size_sweep_fused(pkv, bs):
-    _run_and_compare(pkv, wl.bs_sweep(bs), sample=[0, 255], fused=True)
 
 
 def test_query_groups_split_over_ctas_write_one_row(pkv):
@@ -102,50 +80,3 @@ def test_fused_arguments_are_checked(pkv):
                                           gb.max_context_len, partition_size=24)  # not a multiple of 16
 
 
-def test_cow_workload_fused(pkv):
-    # copy-on-write step then the fused call, for all decode steps; afterwards the cache
-    # rows of chosen samples and their attention match the oracle
-    from batches import CowBatch
-    from oracle_side import compact_pools
-    w = wl.get("cow")
-    Hk, D, bs, N = w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks
-    gb = CowBatch(w, DEV)
-    model = oracle.BlockManagerModel(N, bs, free_order=wl.free_order(N, w.seed))
-    samples, prompt_of = [], {}
-    for p in range(w.prompts):
-        s = model.add_seq(w.prompt_len)
-        for x in [s] + model.fork(s, w.samples - 1):
-            samples.append(x)
-            prompt_of[x] = p
-    assert samples == gb.samples
-    news = []
-    for step in range(w.decode_steps):
-        host = gb.prepare_step()
-        assert host["slots"].tolist() == [model.append_token(s) for s in samples]
-        assert host["pairs"].tolist() == [list(x) for x in model.take_copies()]
-        dev = {k: torch.from_numpy(host[k]).to(DEV) for k in ("tables", "lens", "q", "k", "v")}
-        if len(host["pairs"]):
-            pkv.copy_blocks([gb.key_cache], [gb.value_cache],
-                            torch.from_numpy(host["pairs"]).to(DEV))
-        out = torch.empty_like(dev["q"])
-        pkv.paged_attention_decode_append(out, dev["q"], dev["k"], dev["v"], gb.key_cache,
-                                          gb.value_cache, dev["tables"], dev["lens"], w.scale,
-                                          gb.max_context_len)
-        news.append((host["k"], host["v"]))
-    torch.cuda.synchronize()
-    assert pkv.device_errors() == 0
-    chosen = [0, 7, 8, 100, 255]
-    entries = []
-    for i in chosen:
-        s = samples[i]
-        k0, v0 = wl.sequence_kv(w.seed, prompt_of[s], w.prompt_len, Hk, D)
-        entries.append((model.block_table(s), np.concatenate([k0, np.stack([k[i] for k, _ in news])]),
-                        np.concatenate([v0, np.stack([v[i] for _, v in news])])))
-    kc_o, vc_o, t_o, l_o, relabel = compact_pools(entries, bs, Hk, D)
-    # every block these samples use holds exactly the oracle's bytes
-    idx = torch.tensor(list(relabel), dtype=torch.long, device=DEV)
-    assert np.array_equal(_bits(gb.key_cache[idx]), kc_o.view(np.uint16))
-    assert np.array_equal(_bits(gb.value_cache[idx]), vc_o.view(np.uint16))
-    ref = oracle.paged_attention(host["q"][chosen], kc_o, vc_o, t_o, l_o, w.scale, bs, Hk,
-                                 nthreads=8)
-    assert_attention_close(out.cpu().numpy()[chosen], ref)

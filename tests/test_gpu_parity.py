@@ -4,7 +4,6 @@ Cache writes and block copies must match bit for bit (compared as raw fp16 bit
 patterns, NaN sentinels included); attention outputs must satisfy
 |gpu - oracle| <= 2e-3 + 1e-2 |oracle| element by element.
 """
-import math
 
 import numpy as np
 import pytest
@@ -59,17 +58,12 @@ def _run_and_compare(pkv, w, partition_size=0, sample=None, check_pool=True, fus
     torch.cuda.synchronize()
     assert pkv.device_errors() == 0
     if fused:
-        # the same kernels over the same (now updated) cache give the same outputs: bit for
-        # bit where the schedule is static; the persistent tensor-core kernel hands out work
-        # at run time, so which warp sums which chunk (the fp32 order) can differ
+        # the same kernels over the same (now updated) cache give the same outputs bit for
+        # bit: every kernel fixes which warp sums which chunk, whatever the work order
         fused_out = gb.out.clone()
         pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
                                    gb.context_lens, w.scale, gb.max_context_len, partition_size)
-        G = w.num_heads // w.num_kv_heads
-        if 2 <= G <= 8 and w.block_size >= 8 and w.num_seqs <= 1024:
-            assert_attention_close(fused_out.cpu().numpy(), gb.out.cpu().numpy())
-        else:
-            assert np.array_equal(_bits(fused_out), _bits(gb.out))
+        assert np.array_equal(_bits(fused_out), _bits(gb.out))
     if check_pool:
         idx = torch.tensor(ob.blocks, dtype=torch.long, device=DEV)
         assert np.array_equal(_bits(gb.key_cache[idx]), ob.key_cache.view(np.uint16))
@@ -156,6 +150,27 @@ def test_deterministic(pkv):
     assert np.array_equal(res[0], res[1]) and np.array_equal(res[0], res[2])
 
 
+@pytest.mark.parametrize("part", [512, 0, -1])
+def test_gqa_full_size_is_reproducible(pkv, part):
+    # the persistent tensor-core kernel hands out work items at run time; chunk j of an item
+    # always goes to consumer warp j mod 2, so three runs agree bit for bit
+    from batches import PagedBatch
+    w = wl.get("gqa")
+    gb = PagedBatch(w, DEV)
+    pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
+    res = []
+    for _ in range(3):
+        gb.out.fill_(float("nan"))
+        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                                   gb.context_lens, w.scale, gb.max_context_len, part)
+        res.append(_bits(gb.out))
+    assert pkv.device_errors() == 0
+    assert np.isfinite(gb.out.float().cpu().numpy()).all()
+    assert np.array_equal(res[0], res[1]) and np.array_equal(res[0], res[2])
+    del gb
+    torch.cuda.empty_cache()
+
+
 def test_block_table_figure_on_the_gpu(pkv):
     # the pages' example: 12 tokens at block_size 4 in physical blocks 7, 3, 1
     D, bs, N = 64, 4, 10
@@ -193,120 +208,7 @@ def test_context_of_one_is_exactly_v(pkv):
         assert np.array_equal(out[:, h], vnew[:, h // 4])
 
 
-# ---- full-size workloads, sampled ---------------------------------------------------
-
-def test_llama7b_full_size(pkv):
-    w = wl.get("llama7b")
-    lens = wl.context_lens(w)
-    sample = sorted({0, 1, int(np.argmax(lens)), int(np.argmin(lens)), 100, 255})
-    _run_and_compare(pkv, w, sample=sample)
-
-
-@pytest.mark.parametrize("bs", wl.SWEEP_BLOCK_SIZES)
-def test_block_size_sweep_full_size(pkv, bs):
-    _run_and_compare(pkv, wl.bs_sweep(bs), sample=[0, 77, 255])
-
-
-def test_gqa_full_size(pkv):
-    w = wl.get("gqa")
-    lens = wl.context_lens(w)
-    sample = sorted({0, int(np.argmax(lens)), int(np.argmin(lens)), 64, 127})
-    _run_and_compare(pkv, w, partition_size=w.partition_size, sample=sample)
-
-
-def test_gqa_full_size_automatic_split(pkv):
-    w = wl.get("gqa")
-    lens = wl.context_lens(w)
-    _run_and_compare(pkv, w, partition_size=0, sample=[int(np.argmax(lens)), 3], check_pool=False)
-
-
-# ---- copy-on-write workload ---------------------------------------------------------
-
-def test_cow_workload(pkv):
-    from batches import CowBatch
-    w = wl.get("cow")
-    Hk, D, bs, N = w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks
-    gb = CowBatch(w, DEV)
-    model = oracle.BlockManagerModel(N, bs, free_order=wl.free_order(N, w.seed))
-    samples, prompt_of, prompt_tail = [], {}, {}
-    for p in range(w.prompts):
-        s = model.add_seq(w.prompt_len)
-        prompt_tail[p] = model.block_table(s)[-1]
-        for x in [s] + model.fork(s, w.samples - 1):
-            samples.append(x)
-            prompt_of[x] = p
-    assert samples == gb.samples
-    prompt_kv = [wl.sequence_kv(w.seed, p, w.prompt_len, Hk, D) for p in range(w.prompts)]
-
-    # step 0: seven copies per prompt (the last sharer writes in place), then the new tokens
-    host = gb.prepare_step()
-    ref_slots = [model.append_token(s) for s in samples]
-    ref_pairs = model.take_copies()
-    assert host["slots"].tolist() == ref_slots
-    assert host["pairs"].tolist() == [list(x) for x in ref_pairs]
-    assert len(ref_pairs) == w.prompts * (w.samples - 1)
-    assert {a for a, _ in ref_pairs} == set(prompt_tail.values())
-    gb.run_cache_updates(host)
-    torch.cuda.synchronize()
-    assert pkv.device_errors() == 0
-
-    # expected tail blocks: prompt tails written, copied by the oracle, then the step's rows
-    blocks = sorted(set(prompt_tail.values()) | {b for _, b in ref_pairs})
-    relabel = {b: i for i, b in enumerate(blocks)}
-    first = (w.prompt_len // bs) * bs
-    kc = wl.sentinel_pool(len(blocks), Hk, bs, D)
-    vc = wl.sentinel_pool(len(blocks), Hk, bs, D)
-    kc, vc = oracle.reshape_and_cache(
-        kc, vc, np.concatenate([kv[0][first:] for kv in prompt_kv]),
-        np.concatenate([kv[1][first:] for kv in prompt_kv]),
-        np.concatenate([relabel[prompt_tail[p]] * bs + np.arange(w.prompt_len - first)
-                        for p in range(w.prompts)]), bs)
-    kcs, vcs = oracle.copy_blocks([kc], [vc], [(relabel[a], relabel[b]) for a, b in ref_pairs])
-    new_slots = [relabel[s // bs] * bs + s % bs for s in ref_slots]
-    kc, vc = oracle.reshape_and_cache(kcs[0], vcs[0], host["k"], host["v"], new_slots, bs)
-    idx = torch.tensor(blocks, dtype=torch.long, device=DEV)
-    assert np.array_equal(_bits(gb.key_cache[idx]), kc.view(np.uint16))
-    assert np.array_equal(_bits(gb.value_cache[idx]), vc.view(np.uint16))
-    # after the copies each prompt tail is referenced by one sample only
-    assert all(model.refcount[b] == 1 for b in prompt_tail.values())
-
-    new_kv = {0: (host["k"], host["v"])}
-    chosen = [0, 7, 8, 100, 255]
-
-    def check_attention(host, steps_done):
-        tables = torch.from_numpy(host["tables"]).to(DEV)
-        lens = torch.from_numpy(host["lens"]).to(DEV)
-        q = torch.from_numpy(host["q"]).to(DEV)
-        out = torch.empty_like(q)
-        pkv.paged_attention_decode(out, q, gb.key_cache, gb.value_cache, tables, lens, w.scale,
-                                   gb.max_context_len)
-        entries = []
-        for i in chosen:
-            s = samples[i]
-            k0, v0 = prompt_kv[prompt_of[s]]
-            kn = np.stack([new_kv[j][0][i] for j in range(steps_done)])
-            vn = np.stack([new_kv[j][1][i] for j in range(steps_done)])
-            entries.append((model.block_table(s), np.concatenate([k0, kn]),
-                            np.concatenate([v0, vn])))
-        kc_o, vc_o, t_o, l_o, _ = compact_pools(entries, bs, Hk, D)
-        assert l_o.tolist() == host["lens"][chosen].tolist()
-        ref = oracle.paged_attention(host["q"][chosen], kc_o, vc_o, t_o, l_o, w.scale, bs, Hk,
-                                     nthreads=8)
-        assert_attention_close(out.cpu().numpy()[chosen], ref)
-
-    check_attention(host, 1)
-    for step in range(1, w.decode_steps):
-        host = gb.prepare_step()
-        ref_slots = [model.append_token(s) for s in samples]
-        assert host["slots"].tolist() == ref_slots
-        assert host["pairs"].tolist() == [list(x) for x in model.take_copies()]
-        gb.run_cache_updates(host)
-        new_kv[step] = (host["k"], host["v"])
-    torch.cuda.synchronize()
-    assert pkv.device_errors() == 0
-    assert (host["lens"] == w.prompt_len + w.decode_steps).all()
-    check_attention(host, w.decode_steps)
-
+# (the full-size workloads, whole batches: test_gpu_full_size.py)
 
 # ---- edge cases and device-side checks ----------------------------------------------
 

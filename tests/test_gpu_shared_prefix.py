@@ -244,57 +244,6 @@ def test_inconsistent_groups_are_flagged_not_faulted(pkv):
     assert_attention_close(fb.out.cpu().numpy(), ref)
 
 
-def test_cow_workload_shared_prefix(pkv):
-    # all 200 decode steps of the copy-on-write workload through the fused shared-prefix
-    # call; afterwards the chosen samples' cache rows and attention match the oracle
-    from batches import CowBatch
-    w = wl.get("cow")
-    Hk, D, bs, N = w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks
-    gb = CowBatch(w, DEV)
-    model = oracle.BlockManagerModel(N, bs, free_order=wl.free_order(N, w.seed))
-    samples, prompt_of = [], {}
-    for p in range(w.prompts):
-        s = model.add_seq(w.prompt_len)
-        for x in [s] + model.fork(s, w.samples - 1):
-            samples.append(x)
-            prompt_of[x] = p
-    assert samples == gb.samples
-    news = []
-    for step in range(w.decode_steps):
-        host = gb.prepare_step()
-        assert host["slots"].tolist() == [model.append_token(s) for s in samples]
-        assert host["pairs"].tolist() == [list(x) for x in model.take_copies()]
-        pre, groups = pkv.prefix_groups(host["tables"], host["lens"], bs, 8)
-        assert len(groups) == w.prompts and (pre == 992).all()
-        mp, ms = 992, int((host["lens"] - pre).max())
-        dev = {k: torch.from_numpy(host[k]).to(DEV) for k in ("tables", "lens", "q", "k", "v")}
-        if len(host["pairs"]):
-            pkv.copy_blocks([gb.key_cache], [gb.value_cache], torch.from_numpy(host["pairs"]).to(DEV))
-        out = torch.empty_like(dev["q"])
-        pkv.paged_attention_decode_shared_prefix(
-            out, dev["q"], gb.key_cache, gb.value_cache, dev["tables"], dev["lens"],
-            torch.from_numpy(pre).to(DEV), torch.from_numpy(groups).to(DEV), w.scale,
-            gb.max_context_len, k_new=dev["k"], v_new=dev["v"], max_prefix_tokens=mp,
-            max_suffix_tokens=ms)
-        news.append((host["k"], host["v"]))
-    torch.cuda.synchronize()
-    assert pkv.device_errors() == 0
-    chosen = [0, 7, 8, 100, 255]
-    entries = []
-    for i in chosen:
-        s = samples[i]
-        k0, v0 = wl.sequence_kv(w.seed, prompt_of[s], w.prompt_len, Hk, D)
-        entries.append((model.block_table(s), np.concatenate([k0, np.stack([k[i] for k, _ in news])]),
-                        np.concatenate([v0, np.stack([v[i] for _, v in news])])))
-    kc_o, vc_o, t_o, l_o, relabel = compact_pools(entries, bs, Hk, D)
-    idx = torch.tensor(list(relabel), dtype=torch.long, device=DEV)
-    assert np.array_equal(_bits(gb.key_cache[idx]), kc_o.view(np.uint16))
-    assert np.array_equal(_bits(gb.value_cache[idx]), vc_o.view(np.uint16))
-    ref = oracle.paged_attention(host["q"][chosen], kc_o, vc_o, t_o, l_o, w.scale, bs, Hk,
-                                 nthreads=8)
-    assert_attention_close(out.cpu().numpy()[chosen], ref)
-
-
 @pytest.mark.parametrize("H,Hk", [(8, 8), (8, 2)], ids=["mha", "gqa"])
 def test_decode_session_with_shared_prefixes(pkv, H, Hk):
     # the host-buffer call: inputs from pinned host memory, groups built on the host per step

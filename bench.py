@@ -599,7 +599,7 @@ def measure_cow(args, w, dev, world, rank, local, step_kind, K, e2e_steps):
     else:
         need = pkv.paged_attention_workspace_bytes(B, H, Hk, D, w.block_size, gb.max_context_len,
                                                    cpart)
-    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
     plain_split = pkv.paged_attention_partition_tokens(B, H, Hk, D, w.block_size,
                                                        gb.max_context_len, cpart) > 0
     stream = torch.cuda.Stream(dev)

@@ -69,7 +69,9 @@ extern "C" {
                                          max_context_len / the table (clamped) */
 #define PAGEDKV_DEVERR_SLOT 4u        /* a slot beyond the pool: that token was skipped */
 #define PAGEDKV_DEVERR_TIMEOUT 8u     /* a pipeline wait gave up after ~2 s; output invalid */
-#define PAGEDKV_DEVERR_INTERNAL 16u   /* a kernel found its launch set-up inconsistent and did nothing */
+#define PAGEDKV_DEVERR_INTERNAL 16u   /* a kernel found its launch set-up inconsistent (did
+                                         nothing), or a workspace's work counters did not
+                                         start at zero (outputs invalid) */
 #define PAGEDKV_DEVERR_PREFIX 32u     /* a shared-prefix group or prefix length was inconsistent,
                                          or a host bound on the prefix / suffix lengths was below
                                          a real length: the affected outputs are invalid */
@@ -121,11 +123,16 @@ PAGEDKV_API int pagedkv_selftest_wait_timeout(unsigned int timeout_us, void *str
  *                  and of block_size), computed in parallel and merged by a
  *                  second kernel.
  *   workspace      device scratch of at least paged_attention_workspace_bytes(...)
- *                  bytes (16-byte aligned): the split-K partial results, and for
- *                  grouped queries (2..8 query heads per kv head) a work counter;
- *                  may be NULL when that function returns 0.  Its contents need no
- *                  initialization and are garbage afterwards; calls that may run
- *                  at the same time need separate workspaces.
+ *                  bytes (16-byte aligned); may be NULL when that function returns
+ *                  0.  Its first 16 bytes are work counters (grouped queries, 2..8
+ *                  query heads per kv head, take their work items from them): they
+ *                  must be zero before the workspace's first use -- allocate it
+ *                  zeroed or cudaMemsetAsync them once -- and every call leaves
+ *                  them zero again.  A launch that finds them not zero sets
+ *                  PAGEDKV_DEVERR_INTERNAL (its outputs are then invalid) and
+ *                  still leaves them zero.  The rest holds the split-K partial
+ *                  results, needs no initialization and is garbage afterwards.
+ *                  Calls that may run at the same time need separate workspaces.
  *
  * num_seqs == 0 is a no-op.  Errors: EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
  */
@@ -364,7 +371,8 @@ PAGEDKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, in
  *    capture on that device.
  *  - All calls on a device share the array and leave their partial results in
  *    it; calls that can overlap on the GPU (other streams, other threads) race.
- *    Nothing needs to start at zero.
+ *    Its work counters are cleared at that first call's set-up (on its stream)
+ *    and every call leaves them zero; nothing else needs to start at zero.
  */
 #define PAGEDKV_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 

@@ -177,7 +177,7 @@ def _decode(name, out, q, k_new, v_new, key_cache, value_cache, block_tables, co
     ws_ptr, ws_bytes = None, 0
     if need:
         if workspace is None:
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
         _cuda(workspace, "workspace", workspace.dtype)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     st = getattr(lib, name)(*ptrs, float(scale), bs, Hk, B, H, D, block_tables.shape[1], N,
@@ -246,7 +246,7 @@ def paged_attention_decode_shared_prefix(out, q, key_cache, value_cache, block_t
     ws_ptr, ws_bytes = None, 0
     if need:
         if workspace is None:
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
         _cuda(workspace, "workspace", workspace.dtype)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     st = lib.paged_attention_decode_shared_prefix(

@@ -236,9 +236,10 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     p.part_tokens = ((max_context_len + block_size - 1) / block_size) * block_size;
     p.num_parts = 1;
   }
-  // the tensor-core path runs persistent CTAs fed by a ticket word in the workspace
+  // the tensor-core path runs persistent CTAs fed by a work counter; the counters take the
+  // first WORK_COUNTER_BYTES of every workspace, the partials follow
   p.persistent = p.mma && num_seqs <= PERSISTENT_MAX_SEQS && PAGEDKV_TUNE_PERSISTENT;
-  if (p.persistent) p.ws_bytes = ((p.ws_bytes + 15) / 16) * 16 + 16;
+  if (p.persistent || p.ws_bytes > 0) p.ws_bytes += WORK_COUNTER_BYTES;
   // ring depth: few stages and many CTAs per SM stream best (measured)
   if (p.mma) {
     // a multiple of the consumer warps, so every warp owns the same number of stages
@@ -404,7 +405,7 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   if (plan.split) {
-    p.ws_o = static_cast<float*>(workspace);
+    p.ws_o = reinterpret_cast<float*>(static_cast<char*>(workspace) + WORK_COUNTER_BYTES);
     p.ws_ml = p.ws_o + (size_t)num_seqs * num_heads * plan.num_parts * head_dim;
   }
   p.err = err;
@@ -445,24 +446,15 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
     st = encode_pool_map(&vm, value_cache, rows, head_dim, block_size);
     if (st != PAGEDKV_OK) return st;
   }
-  unsigned int* ticket = nullptr;  // the persistent kernel's work counter
-  if (plan.mma && plan.persistent) {
-    const size_t parts_bytes =
-        plan.split ? (size_t)num_seqs * num_heads * plan.num_parts * (head_dim + 2) * sizeof(float)
-                   : 0;
-    ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
-                                             ((parts_bytes + 15) / 16) * 16);
-  }
+  // work counters (self-resetting: the last CTA of a persistent launch zeroes its pair):
+  // [0] [1] the decode pass's ticket and finished-CTA count, [2] [3] the prefix pass's
+  unsigned int* counters =
+      plan.ws_bytes > 0 ? reinterpret_cast<unsigned int*>(workspace) : nullptr;
   const bool prefix_pass = cascade && num_groups > 0;
   if (prefix_pass) {
     // Prefix pass first.  The suffix pass is its programmatic dependent: it may
     // start on the SMs the prefix pass frees and waits for it only before it
-    // reads the prefix partials; the merge follows the suffix pass.  The work
-    // counter is zeroed before the prefix pass so nothing sits between the two.
-    if (ticket) {
-      e = cudaMemsetAsync(ticket, 0, sizeof(unsigned int), s);
-      if (e != cudaSuccess) return cuda_fail(e, "work counter reset");
-    }
+    // reads the prefix partials; the merge follows the suffix pass.
     DecodeParams pp = p;
     pp.stages = plan.prefix_stages;
     pp.k_new = pp.v_new = nullptr;
@@ -478,7 +470,7 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
   }
   if (plan.mma) {
     if (plan.persistent) {
-      e = launch_mma_decode_persistent(p, km, vm, ticket, plan.split, s, prefix_pass);
+      e = launch_mma_decode_persistent(p, km, vm, counters, plan.split, s);
     } else {
       e = launch_mma_decode(p, km, vm, plan.split, s);
     }

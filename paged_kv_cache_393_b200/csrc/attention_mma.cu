@@ -747,9 +747,26 @@ __global__ void __launch_bounds__((NW + 1) * 32)
 // ---- persistent split-K kernel ---------------------------------------------------
 
 struct PersistentArgs {
-  unsigned int* ticket;  // zeroed before the launch
-  int write_zeros;       // no merge kernel may follow: write the zero outputs of empty contexts
+  unsigned int* ticket;    // next work item; zero at the start, zeroed again by the last CTA
+  unsigned int* finished;  // CTAs done taking tickets; likewise
+  int write_zeros;         // no merge kernel may follow: write the zero outputs of empty contexts
 };
+
+// Run by one thread of each CTA once the CTA takes no more tickets.  The last
+// CTA to get here zeroes both counters for the next launch on this workspace:
+// every CTA has taken its last ticket by then, so nothing can add to them.
+// Without an abort every CTA took exactly one ticket past the last item, so a
+// final count other than total + CTAs means the counter did not start at zero.
+__device__ __forceinline__ void release_counters(const PersistentArgs& pa, unsigned total,
+                                                 bool check, unsigned* err) {
+  __threadfence();
+  if (atomicAdd(pa.finished, 1u) == gridDim.x - 1) {
+    const unsigned taken = atomicExch(pa.ticket, 0u);
+    atomicExch(pa.finished, 0u);
+    if (check && taken != total + gridDim.x) flag_error(err, ERR_INTERNAL);
+    __threadfence();
+  }
+}
 
 // Work item of ticket t: every full partition (part_tokens tokens) comes first,
 // in (sequence, partition) order, then the partial last partitions, longest
@@ -794,7 +811,10 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = smem_raw;
   if (smem_u32(smem_raw) & 1023u) {
-    if (threadIdx.x == 0) flag_error(p.err, ERR_INTERNAL);
+    if (threadIdx.x == 0) {
+      flag_error(p.err, ERR_INTERNAL);
+      release_counters(pa, 0, false, p.err);
+    }
     return;
   }
   const int stages = p.stages;
@@ -929,11 +949,13 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     issued.reset();
     // A ticket is taken when the previous item has been issued: taking them
     // earlier reserves work a CTA cannot start yet and unbalances the end.
+    // (unsigned: whatever value the counter holds, a ticket is an item in range or the end)
     auto next_item = [&](int4* item) {
-      const int t = __shfl_sync(0xffffffffu, lane == 0 ? (int)atomicAdd(pa.ticket, 1u) : 0, 0);
-      *item = t < total ? item_of_ticket(t, p.num_kv_heads, B, pt, pref_f, by_tail, s_lens)
-                        : make_int4(0, 0, 0, 0);
-      return t < total;
+      const unsigned t = __shfl_sync(0xffffffffu, lane == 0 ? atomicAdd(pa.ticket, 1u) : 0u, 0);
+      const bool ok = t < (unsigned)total;
+      *item = ok ? item_of_ticket((int)t, p.num_kv_heads, B, pt, pref_f, by_tail, s_lens)
+                 : make_int4(0, 0, 0, 0);
+      return ok;
     };
     int4 d;
     bool have = next_item(&d);
@@ -976,7 +998,11 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       base.advance(nchunks);
       have = next_item(&d);
     }
-    if (lane == 0 && *abort_flag) drain_ring(bars, stages, issued);
+    if (lane == 0) {
+      const bool aborted = *abort_flag != 0;
+      if (aborted) drain_ring(bars, stages, issued);
+      release_counters(pa, (unsigned)total, !aborted, p.err);
+    }
     return;
   }
 
@@ -1073,8 +1099,8 @@ cudaError_t launch_mma_instance(const DecodeParams& p, const CUtensorMap& km,
 
 template <int D, int BS>
 cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap& km,
-                                       const CUtensorMap& vm, unsigned int* ticket, bool split,
-                                       cudaStream_t stream, bool ticket_zeroed) {
+                                       const CUtensorMap& vm, unsigned int* counters, bool split,
+                                       cudaStream_t stream) {
   static std::atomic<int> granted[MAX_DEVICES];
   static std::atomic<int> blocks_per_sm[MAX_DEVICES];
   static std::atomic<int> blocks_smem[MAX_DEVICES];
@@ -1100,12 +1126,9 @@ cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap&
   const long long items = (long long)p.num_kv_heads * p.num_seqs * p.num_parts;
   long long ctas = (long long)sms * blocks_per_sm[dev].load(std::memory_order_relaxed);
   if (ctas > items) ctas = items;
-  if (!ticket_zeroed) {
-    e = cudaMemsetAsync(ticket, 0, sizeof(unsigned int), stream);
-    if (e != cudaSuccess) return e;
-  }
   PersistentArgs pa;
-  pa.ticket = ticket;
+  pa.ticket = counters;
+  pa.finished = counters + 1;
   pa.write_zeros = (!split || p.seq_prefix_tokens) ? 1 : 0;
   return launch_kernel(p.after_prefix != 0, kernel, dim3((unsigned)ctas), dim3((NW + 1) * 32),
                        smem, stream, km, vm, p, pa);
@@ -1180,11 +1203,11 @@ cudaError_t launch_mma_prefix(const DecodeParams& p, const CUtensorMap& km, cons
 
 #define PKV_MMA_PERSISTENT_CASE(D_, BS_)        \
   if (p.head_dim == D_ && p.block_size == BS_) \
-    return launch_persistent_instance<D_, BS_>(p, km, vm, ticket, split, stream, ticket_zeroed);
+    return launch_persistent_instance<D_, BS_>(p, km, vm, counters, split, stream);
 
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& km,
-                                         const CUtensorMap& vm, unsigned int* ticket, bool split,
-                                         cudaStream_t stream, bool ticket_zeroed) {
+                                         const CUtensorMap& vm, unsigned int* counters, bool split,
+                                         cudaStream_t stream) {
   PKV_MMA_PERSISTENT_CASE(64, 8)
   PKV_MMA_PERSISTENT_CASE(64, 16)
   PKV_MMA_PERSISTENT_CASE(64, 32)

@@ -86,14 +86,19 @@ cudaError_t launch_simt_decode(const DecodeParams& p, int hpc, int kvc, bool spl
 cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& k_map,
                               const CUtensorMap& v_map, bool split, cudaStream_t stream);
 
+// Work counters at the start of every workspace: counters[0] is the ticket of the
+// persistent decode kernel and counters[1] its count of finished CTAs (the last
+// CTA zeroes both); counters[2..3] are the same pair for the shared-prefix pass.
+// They must be zero before a workspace's first use and every launch leaves
+// them zero.
+constexpr size_t WORK_COUNTER_BYTES = 16;
+
 // Persistent tensor-core kernel: a few CTAs per SM take (b, kv head, partition)
-// work items from `ticket` (a workspace word it zeroes first).  Without a
-// split every item is a whole context.
-// ticket_zeroed: the caller already zeroed the work counter on this stream.
+// work items from the ticket counters[0].  Without a split every item is a
+// whole context.
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& k_map,
-                                         const CUtensorMap& v_map, unsigned int* ticket,
-                                         bool split, cudaStream_t stream,
-                                         bool ticket_zeroed = false);
+                                         const CUtensorMap& v_map, unsigned int* counters,
+                                         bool split, cudaStream_t stream);
 size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs);
 constexpr int PERSISTENT_MAX_SEQS = 1024;
 

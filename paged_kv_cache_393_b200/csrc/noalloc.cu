@@ -16,9 +16,10 @@
 // needing more are rejected.  All calls on a device share it, and each call
 // leaves its partial results behind: calls that may run on the GPU at the same
 // time (different streams, or different host threads) corrupt each other's
-// results, so serialize them.  Nothing in it needs to start at zero: every
-// partial result a call reads was written earlier in that same call, and the
-// work counter is cleared on the stream before each launch that uses it.
+// results, so serialize them.  Its first 16 bytes are the work counters of the
+// grouped-query kernel, which must start at zero: they are cleared once, when a
+// device's address is looked up, and every call leaves them at zero.  Every
+// partial result a call reads was written earlier in that same call.
 #include "../../include/pagedkv.h"
 
 #include <cuda_runtime.h>
@@ -33,6 +34,7 @@ int record_error(int code, const char* message);
 namespace {
 
 constexpr size_t kScratchBytes = PAGEDKV_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kCounterBytes = 16;  // the work counters at the start of every workspace
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -48,8 +50,9 @@ int report(int code, const char* fmt, size_t a = 0, size_t b = 0) {
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name only stands for it; the address is looked up once per device,
-// with that device current, and cached.
-int scratch_address(void** out) {
+// with that device current, and cached; the work counters at its start are
+// cleared then, on the caller's stream, ahead of the first kernel that uses them.
+int scratch_address(void** out, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return report(PAGEDKV_ECUDA, "cudaGetDevice failed");
@@ -60,6 +63,8 @@ int scratch_address(void** out) {
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p)
       return report(PAGEDKV_ECUDA, "cudaGetSymbolAddress of the built-in scratch failed");
+    e = cudaMemsetAsync(p, 0, kCounterBytes, stream);
+    if (e != cudaSuccess) return report(PAGEDKV_ECUDA, "clearing the built-in scratch failed");
     g_scratch_address[dev] = p;
   }
   *out = g_scratch_address[dev];
@@ -93,7 +98,7 @@ extern "C" int paged_attention_decode_noalloc(
                   need, kScratchBytes);
   void* scratch = nullptr;
   if (need > 0) {
-    const int st = scratch_address(&scratch);
+    const int st = scratch_address(&scratch, static_cast<cudaStream_t>(stream));
     if (st != PAGEDKV_OK) return st;
   }
   return paged_attention_decode(out, q, key_cache, value_cache, block_tables, context_lens, scale,

@@ -42,8 +42,9 @@ class LayeredDecodeStep:
         self.context_lens = torch.ones(B, dtype=torch.int32, device=dev)
         self.pairs = torch.empty((max(max_pairs, 1), 2), dtype=torch.int64, device=dev)
         need = paged_attention_workspace_bytes(B, H, Hk, D, bs, max_context_len, partition_size)
-        # the layers run in order on one stream, so they share one workspace
-        self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        # the layers run in order on one stream, so they share one workspace (zeroed: its
+        # work counters must start at zero)
+        self.workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
         self.graph = None
         self._inputs_set = False
 

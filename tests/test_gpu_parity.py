@@ -171,6 +171,36 @@ def test_gqa_full_size_is_reproducible(pkv, part):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("part", [64, -1])
+def test_work_counters_are_left_zero_and_a_dirty_start_is_flagged(pkv, part):
+    # grouped queries take their work from counters at the start of the workspace: every
+    # launch leaves them zero (no reset between launches); a workspace whose counters do
+    # not start at zero is flagged, and the launch still leaves them zero
+    from batches import PagedBatch
+    w = _fixed("counters", 16, 2, 128, 16, [1, 300, 1030, 77])
+    gb = PagedBatch(w, DEV)
+    pkv.reshape_and_cache(gb.k_new, gb.v_new, gb.key_cache, gb.value_cache, gb.slots)
+    need = pkv.paged_attention_workspace_bytes(4, 16, 2, 128, 16, gb.max_context_len, part)
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+
+    def run():
+        pkv.paged_attention_decode(gb.out, gb.q, gb.key_cache, gb.value_cache, gb.block_tables,
+                                   gb.context_lens, w.scale, gb.max_context_len, part, ws)
+        torch.cuda.synchronize()
+
+    run()
+    assert pkv.device_errors() == 0 and (ws[:16] == 0).all()
+    ref = _bits(gb.out)
+    run()
+    assert pkv.device_errors() == 0 and np.array_equal(ref, _bits(gb.out))
+    ws[0] = 5                                      # a ticket count left by someone else
+    run()
+    assert pkv.device_errors() & pkv.DEVERR_INTERNAL
+    assert (ws[:16] == 0).all()
+    run()
+    assert pkv.device_errors() == 0 and np.array_equal(ref, _bits(gb.out))
+
+
 def test_block_table_figure_on_the_gpu(pkv):
     # the pages' example: 12 tokens at block_size 4 in physical blocks 7, 3, 1
     D, bs, N = 64, 4, 10

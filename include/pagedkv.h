@@ -219,11 +219,14 @@ PAGEDKV_API int paged_attention_decode_append(void *out, const void *q,
  *                  NULL when num_groups is 0.
  *   max_prefix_tokens, max_suffix_tokens  host upper bounds of the groups' prefix
  *                  lengths and of L_b - P_b over the batch (0 = max_context_len);
- *                  they size the launch grids.  A bound below a real length
- *                  leaves that work undone and sets PAGEDKV_DEVERR_PREFIX.  When
- *                  max_suffix_tokens fits one partition, the suffix pass folds
- *                  the prefix partials into every output itself and no merge
- *                  kernel is launched.
+ *                  they size the launch grids.  With up to 1024 groups the prefix
+ *                  pass runs on persistent CTAs that take every group's items
+ *                  from a queue, so max_prefix_tokens only sizes that grid; with
+ *                  more groups, and for max_suffix_tokens always, a bound below a
+ *                  real length leaves that work undone and sets
+ *                  PAGEDKV_DEVERR_PREFIX.  When max_suffix_tokens fits one
+ *                  partition, the suffix pass folds the prefix partials into
+ *                  every output itself and no merge kernel is launched.
  *   partition_size 0 or -1 = 512 tokens; else as for paged_attention_decode.
  *                  The call always splits.
  *   workspace      at least paged_attention_shared_prefix_workspace_bytes(...).

@@ -464,7 +464,12 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
       const int need = (max_prefix_tokens + plan.part_tokens - 1) / plan.part_tokens;
       if (need < prefix_parts) prefix_parts = need;
     }
-    e = launch_mma_prefix(pp, km, vm, prefix_parts, s);
+    // persistent CTAs stream the prefix items from a ticket queue; beyond the
+    // persistent grid's row limit, one CTA per item
+    if (num_groups <= PERSISTENT_MAX_SEQS)
+      e = launch_mma_prefix_persistent(pp, km, vm, counters, prefix_parts, s);
+    else
+      e = launch_mma_prefix(pp, km, vm, prefix_parts, s);
     if (e != cudaSuccess) return cuda_fail(e, "shared-prefix pass launch");
     p.after_prefix = 1;
   }

@@ -798,12 +798,86 @@ __device__ __forceinline__ int4 item_of_ticket(int t, int num_kv_heads, int num_
 
 constexpr int TAIL_KEYS = 64;  // partial partitions of 63+ chunks share the top key  // chunk-count keys of the partial-partition sort
 
-template <int D, int BS>
+// The shared-prefix pass's members of group g for one item (blocks blk0 ..
+// blk0+nblk-1 of the prefix, Pg prefix tokens): bit i of the result for member
+// slot i when that member is usable -- a sequence of the batch whose prefix
+// length is Pg and whose table entries over these blocks equal those of the
+// group's first usable member.  mem[i] gets every slot's sequence (all lanes).
+// Run by a whole warp; one round of loads for the entries of all members.
+template <int BS>
+__device__ unsigned prefix_members(const DecodeParams& p, int g, int Pg, int blk0, int nblk,
+                                   int max_members, int (&mem)[GROUP_MAX_MEMBERS], bool report,
+                                   int lane) {
+  const int32_t* gd = p.groups + (size_t)g * GROUP_WIDTH;
+  int m = -1;
+  bool ok = false;
+  if (lane < GROUP_MAX_MEMBERS) {
+    m = gd[1 + lane];
+    ok = lane < max_members && m >= 0 && m < p.num_seqs;
+    if (ok) {
+      const int L = min(p.context_lens[m], p.max_context_len);
+      bool bad = false;
+      ok = L > 0 && prefix_tokens_of(p.seq_prefix_tokens, m, L, BS, &bad) == Pg;
+    }
+    if (!ok && m != -1 && report) flag_error(p.err, ERR_PREFIX);
+  }
+  unsigned mask = __ballot_sync(0xffffffffu, ok) & ((1u << GROUP_MAX_MEMBERS) - 1);
+#pragma unroll
+  for (int i = 0; i < GROUP_MAX_MEMBERS; ++i) mem[i] = __shfl_sync(0xffffffffu, m, i);
+  if (mask == 0) return 0;
+  const int first = mem[__ffs(mask) - 1];
+  const int32_t* ref = p.block_tables + (size_t)first * p.max_blocks + blk0;
+  unsigned differ = 0;  // member slots whose entries differ from the first member's
+  for (int j = lane; j < nblk; j += 32) {
+    const int32_t r = ref[j];
+#pragma unroll
+    for (int i = 0; i < GROUP_MAX_MEMBERS; ++i)
+      if ((mask >> i) & 1)
+        differ |= (p.block_tables[(size_t)mem[i] * p.max_blocks + blk0 + j] != r) ? 1u << i : 0u;
+  }
+  differ = __reduce_or_sync(0xffffffffu, differ);
+  if (differ && lane == 0) flag_error(p.err, ERR_PREFIX);
+  return mask & ~differ;
+}
+
+// Query fragments (as load_q_fragments) of a tile whose column c is used only when
+// bit c of `cols` is set; other columns are zero.
+template <int D>
+__device__ __forceinline__ void load_q_masked(uint32_t (&qb)[D / 16][2], const __half* q_tile,
+                                              unsigned cols, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const bool use = (cols >> g) & 1;
+  const __half* qrow = q_tile + (size_t)g * D;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    qb[ks][0] = use ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
+    qb[ks][1] = use ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t + 8) : 0u;
+  }
+}
+
+// Columns of a prefix tile (member-major, G each) whose member slot is in `mask`.
+__device__ __forceinline__ unsigned member_columns(unsigned mask, int G) {
+  unsigned cols = 0;
+  for (int c = 0; c < (8 / G) * G; ++c)
+    if ((mask >> (c / G)) & 1) cols |= 1u << c;
+  return cols;
+}
+
+// PREFIX = false: the decode pass (suffix pass of a shared-prefix call), rows =
+// sequences.  PREFIX = true: the shared-prefix pass, rows = groups: an item is
+// (group, kv head, partition of the group's prefix); the producer checks the
+// members for the item (prefix length, table entries over the partition equal
+// to the first usable member's; a member failing either is left out and raises
+// PAGEDKV_DEVERR_PREFIX), the columns of the tile are the usable members' query
+// heads of that kv head (member-major), and each member's partial state goes
+// to its prefix slot `partition`.
+template <int D, int BS, bool PREFIX>
 __global__ void __launch_bounds__((NW + 1) * 32)
     mma_decode_persistent_kernel(const __grid_constant__ CUtensorMap k_map,
                                  const __grid_constant__ CUtensorMap v_map, const DecodeParams p,
                                  const PersistentArgs pa) {
   using Geo = StageGeom<D>;
+  constexpr int AUX = GROUP_MAX_MEMBERS + 1;  // PREFIX: member mask, then the members
   constexpr uint32_t QTILE_BYTES = 8 * D * 2;
   // The 128-byte TMA swizzle needs 1024-byte aligned stages; the dynamic
   // shared memory is declared with that alignment (no slack is allocated), and
@@ -817,8 +891,9 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     }
     return;
   }
+  if (PREFIX) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // suffix pass
   const int stages = p.stages;
-  const int B = p.num_seqs;
+  const int B = PREFIX ? p.num_groups : p.num_seqs;
   const uint32_t ring = smem_u32(smem);
   unsigned char* cur = smem + (size_t)stages * 2 * Geo::TILE_BYTES;
   __half* s_q = reinterpret_cast<__half*>(cur);  // [IQ][8][D]
@@ -829,6 +904,8 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   cur += Geo::MERGE_BYTES;
   int4* s_item = reinterpret_cast<int4*>(cur);   // [IQ]
   cur += IQ * sizeof(int4);
+  int* s_aux = reinterpret_cast<int*>(cur);      // PREFIX: [IQ][AUX] member mask, members
+  if (PREFIX) cur += IQ * AUX * sizeof(int);
   int* s_lens = reinterpret_cast<int*>(cur);     // [B]
   int* pref_f = s_lens + B;                      // [B + 1]
   int* by_tail = pref_f + B + 1;                 // [B]: sequences with a partial partition
@@ -849,18 +926,27 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   // per-sequence partition counts; the partial tails' chunk-count keys
   for (int k = threadIdx.x; k < TAIL_KEYS; k += blockDim.x) tail_run[k] = 0;
   __syncthreads();
-  // s_lens[b]: the tokens this kernel covers, L minus a shared prefix's tokens
+  // s_lens[b]: the tokens this kernel covers -- L minus a shared prefix's tokens, or
+  // (PREFIX) the group's prefix tokens
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    int L = p.context_lens[b];
-    if (L > p.max_context_len || L <= 0) {
-      if (blockIdx.x == 0) flag_error(p.err, ERR_CONTEXT_LEN);
-      L = L <= 0 ? 0 : p.max_context_len;
+    int L;
+    if (PREFIX) {
+      const int pb = p.groups[(size_t)b * GROUP_WIDTH];
+      const bool ok = pb > 0 && pb <= p.max_blocks;
+      if (!ok && blockIdx.x == 0) flag_error(p.err, ERR_PREFIX);
+      L = ok ? pb * BS : 0;
+    } else {
+      L = p.context_lens[b];
+      if (L > p.max_context_len || L <= 0) {
+        if (blockIdx.x == 0) flag_error(p.err, ERR_CONTEXT_LEN);
+        L = L <= 0 ? 0 : p.max_context_len;
+      }
+      bool bad_prefix = false;
+      L -= L > 0 ? prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad_prefix) : 0;
+      if (bad_prefix && blockIdx.x == 0) flag_error(p.err, ERR_PREFIX);
     }
-    bool bad_prefix = false;
-    L -= L > 0 ? prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad_prefix) : 0;
-    if (bad_prefix && blockIdx.x == 0) flag_error(p.err, ERR_PREFIX);
     s_lens[b] = L;
-    if (L == 0 && pa.write_zeros && blockIdx.x == 0) {
+    if (!PREFIX && L == 0 && pa.write_zeros && blockIdx.x == 0) {
       for (int i = 0; i < p.num_heads * D; ++i)
         p.out[(size_t)b * p.num_heads * D + i] = __float2half_rn(0.f);
     }
@@ -963,6 +1049,28 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       const bool done = !have || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
       if (done) d = make_int4(0, 0, 0, 0);
       const int qs = it % IQ;
+      // the item's table row, chunks and (PREFIX) usable members
+      const int nblk = (d.w + BS - 1) / BS;
+      int nchunks = (d.w + CHUNK - 1) / CHUNK;
+      const int32_t* row = nullptr;
+      int new_tok = -1;
+      unsigned mask = 0;
+      int mem[GROUP_MAX_MEMBERS];
+      if (!done) {
+        if (PREFIX) {
+          const int blk0 = d.z * pt / BS;
+          mask = prefix_members<BS>(p, d.x, s_lens[d.x], blk0, nblk, 8 / G, mem,
+                                    d.y == 0 && d.z == 0, lane);
+          if (mask) row = p.block_tables + (size_t)mem[__ffs(mask) - 1] * p.max_blocks + blk0;
+          else nchunks = 0;  // no usable member: nothing to stream
+        } else {
+          const int P = prefix_of(d.x);
+          row = p.block_tables + (size_t)d.x * p.max_blocks + (P + d.z * pt) / BS;
+          const int Ls = s_lens[d.x];
+          new_tok = (p.k_new && d.z * pt + d.w == Ls && p.context_lens[d.x] == P + Ls) ? d.w - 1
+                                                                                     : -1;
+        }
+      }
       bool ok = true;
       if (lane == 0) {
         if (it >= IQ && !mbar_wait(smem_u32(&iempty[qs]), ((it / IQ) - 1) & 1)) {
@@ -973,26 +1081,34 @@ __global__ void __launch_bounds__((NW + 1) * 32)
         if (ok) {
           s_item[qs] = d;
           const uint32_t full = smem_u32(&ifull[qs]);
-          if (!done) {
+          if (done) {
+            mbar_arrive(full);  // the end marker (tokens = 0)
+          } else if (PREFIX) {
+            s_aux[qs * AUX] = (int)mask;
+            for (int i = 0; i < GROUP_MAX_MEMBERS; ++i) s_aux[qs * AUX + 1 + i] = mem[i];
+            // the usable members' query rows of kv head d.y: columns i*G .. i*G+G-1
+            if (mask) {
+              mbar_arrive_expect_tx(full, (uint32_t)(__popc(mask) * G * D * 2));
+              for (int i = 0; i < GROUP_MAX_MEMBERS; ++i)
+                if ((mask >> i) & 1)
+                  bulk_load(smem_u32(s_q) + qs * QTILE_BYTES + (uint32_t)(i * G * D * 2),
+                            p.q + ((size_t)mem[i] * p.num_heads + d.y * G) * D,
+                            (uint32_t)(G * D * 2), full, policy);
+            } else {
+              mbar_arrive(full);
+            }
+          } else {
             mbar_arrive_expect_tx(full, (uint32_t)(G * D * 2));
             bulk_load(smem_u32(s_q) + qs * QTILE_BYTES,
                       p.q + ((size_t)d.x * p.num_heads + d.y * G) * D, (uint32_t)(G * D * 2), full,
                       policy);
-          } else {
-            mbar_arrive(full);  // the end marker (tokens = 0)
           }
         }
       }
       ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
       if (done || !ok) break;
-      const int nchunks = (d.w + CHUNK - 1) / CHUNK;
-      const int nblk = (d.w + BS - 1) / BS;
-      const int P = prefix_of(d.x);
-      const int32_t* row = p.block_tables + (size_t)d.x * p.max_blocks + (P + d.z * pt) / BS;
-      const int Ls = s_lens[d.x];
-      const int new_tok =
-          (p.k_new && d.z * pt + d.w == Ls && p.context_lens[d.x] == P + Ls) ? d.w - 1 : -1;
-      if (!produce_item<D, BS>(row, nblk, nchunks, base, d.y, d.x, new_tok, p, s_ids, bars,
+      if (nchunks > 0 &&
+          !produce_item<D, BS>(row, nblk, nchunks, base, d.y, d.x, new_tok, p, s_ids, bars,
                                stages, ring, &k_map, &v_map, policy, abort_flag, lane, issued))
         break;
       base.advance(nchunks);
@@ -1024,14 +1140,22 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       d = s_item[qs];
       stop = d.w == 0;
     }
+    unsigned mask = 0;                 // PREFIX: usable member slots of the item
+    int mem[GROUP_MAX_MEMBERS];        // PREFIX: the member slots' sequences
+    if (PREFIX && !stop) {
+      mask = (unsigned)s_aux[qs * AUX];
+#pragma unroll
+      for (int i = 0; i < GROUP_MAX_MEMBERS; ++i) mem[i] = s_aux[qs * AUX + 1 + i];
+    }
     Acc<D> a;
     a.reset();
     if (!stop) {
       uint32_t qb[Geo::MT][2];
-      load_q_fragments<D>(qb, s_q + qs * (8 * D), G, lane);
+      if (PREFIX) load_q_masked<D>(qb, s_q + qs * (8 * D), member_columns(mask, G), lane);
+      else load_q_fragments<D>(qb, s_q + qs * (8 * D), G, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&iempty[qs]));  // descriptor and query tile consumed
-      const int nchunks = (d.w + CHUNK - 1) / CHUNK;
+      const int nchunks = (PREFIX && !mask) ? 0 : (d.w + CHUNK - 1) / CHUNK;
       // chunks warp, warp + NW, ... of the item: this warp's next fills, in order
       for (int j = warp; j < nchunks; j += NW, ++mine) {
         const int st = ring_stage(mine, warp, spw);
@@ -1058,6 +1182,19 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     if (named_barrier_or(1, NW * 32, stop || gave_up)) break;
     write_state<D>(a, s_m, s_l, s_o, warp, lane);
     named_barrier_sync(1, NW * 32);
+    if (PREFIX) {
+      // each usable member's partial state goes to its prefix slot d.z
+      const int kvh = d.y;
+      store_columns<D>(
+          s_m, s_l, s_o, p, (8 / G) * G,
+          [&](int c) -> long long {
+            const int i = c / G;
+            return ((mask >> i) & 1) ? (long long)mem[i] * p.num_heads + (long long)kvh * G + c % G
+                                     : -1;
+          },
+          d.z, false);
+      continue;
+    }
     // a whole suffix (one item) is finished here, a shared prefix's partials folded in
     if (p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");  // prefix partials ready
     const int P = prefix_of(d.x);
@@ -1066,7 +1203,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     store_item<D>(s_m, s_l, s_o, p, d.x, d.y, np + d.z, G, whole, whole ? np : 0);
   }
   // the merge kernel may be scheduled once every CTA got here
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (!PREFIX) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 constexpr int MAX_DEVICES = 64;
@@ -1097,15 +1234,16 @@ cudaError_t launch_mma_instance(const DecodeParams& p, const CUtensorMap& km,
                        vm, p);
 }
 
-template <int D, int BS>
+template <int D, int BS, bool PREFIX>
 cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap& km,
                                        const CUtensorMap& vm, unsigned int* counters, bool split,
-                                       cudaStream_t stream) {
+                                       long long items, cudaStream_t stream) {
   static std::atomic<int> granted[MAX_DEVICES];
   static std::atomic<int> blocks_per_sm[MAX_DEVICES];
   static std::atomic<int> blocks_smem[MAX_DEVICES];
-  auto kernel = mma_decode_persistent_kernel<D, BS>;
-  const size_t smem = mma_persistent_smem_bytes(D, p.stages, p.num_seqs);
+  auto kernel = mma_decode_persistent_kernel<D, BS, PREFIX>;
+  const size_t smem =
+      mma_persistent_smem_bytes(D, p.stages, PREFIX ? p.num_groups : p.num_seqs, PREFIX);
   cudaError_t e = allow_smem(kernel, smem, granted);
   if (e != cudaSuccess) return e;
   int dev = 0;
@@ -1123,15 +1261,15 @@ cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap&
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   // no more CTAs than work items can exist
-  const long long items = (long long)p.num_kv_heads * p.num_seqs * p.num_parts;
   long long ctas = (long long)sms * blocks_per_sm[dev].load(std::memory_order_relaxed);
   if (ctas > items) ctas = items;
+  if (ctas < 1) ctas = 1;
   PersistentArgs pa;
-  pa.ticket = counters;
-  pa.finished = counters + 1;
-  pa.write_zeros = (!split || p.seq_prefix_tokens) ? 1 : 0;
-  return launch_kernel(p.after_prefix != 0, kernel, dim3((unsigned)ctas), dim3((NW + 1) * 32),
-                       smem, stream, km, vm, p, pa);
+  pa.ticket = counters + (PREFIX ? 2 : 0);
+  pa.finished = counters + (PREFIX ? 3 : 1);
+  pa.write_zeros = (!PREFIX && (!split || p.seq_prefix_tokens)) ? 1 : 0;
+  return launch_kernel(!PREFIX && p.after_prefix != 0, kernel, dim3((unsigned)ctas),
+                       dim3((NW + 1) * 32), smem, stream, km, vm, p, pa);
 }
 
 }  // namespace
@@ -1146,10 +1284,11 @@ size_t mma_smem_bytes(int head_dim, int block_size, int stages) {
          32 * sizeof(int) + 2ull * stages * sizeof(uint64_t) + 16;
 }
 
-size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs) {
+size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_rows, bool prefix) {
   const size_t merge = (size_t)NW * 8 * (2 + head_dim + 4) * sizeof(float);
   return (size_t)stages * mma_stage_bytes(head_dim, 16) + IQ * 8ull * head_dim * 2 + merge +
-         IQ * sizeof(int4) + (3ull * num_seqs + 1 + TAIL_KEYS + 1 + 32) * sizeof(int) + 8 +
+         IQ * sizeof(int4) + (prefix ? IQ * (GROUP_MAX_MEMBERS + 1) * sizeof(int) : 0) +
+         (3ull * num_rows + 1 + TAIL_KEYS + 1 + 32) * sizeof(int) + 8 +
          (2ull * stages + 2 * IQ) * sizeof(uint64_t) + 16;
 }
 
@@ -1201,9 +1340,10 @@ cudaError_t launch_mma_prefix(const DecodeParams& p, const CUtensorMap& km, cons
   return cudaErrorInvalidValue;
 }
 
-#define PKV_MMA_PERSISTENT_CASE(D_, BS_)        \
-  if (p.head_dim == D_ && p.block_size == BS_) \
-    return launch_persistent_instance<D_, BS_>(p, km, vm, counters, split, stream);
+#define PKV_MMA_PERSISTENT_CASE(D_, BS_)                                                      \
+  if (p.head_dim == D_ && p.block_size == BS_)                                               \
+    return launch_persistent_instance<D_, BS_, false>(                                       \
+        p, km, vm, counters, split, (long long)p.num_kv_heads * p.num_seqs * p.num_parts, stream);
 
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& km,
                                          const CUtensorMap& vm, unsigned int* counters, bool split,
@@ -1216,6 +1356,25 @@ cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMa
   PKV_MMA_PERSISTENT_CASE(128, 16)
   PKV_MMA_PERSISTENT_CASE(128, 32)
   PKV_MMA_PERSISTENT_CASE(128, 64)
+  return cudaErrorInvalidValue;
+}
+
+#define PKV_MMA_PREFIX_PERSISTENT_CASE(D_, BS_)                                             \
+  if (p.head_dim == D_ && p.block_size == BS_)                                             \
+    return launch_persistent_instance<D_, BS_, true>(                                      \
+        p, km, vm, counters, true, (long long)p.num_kv_heads * p.num_groups * prefix_parts, stream);
+
+cudaError_t launch_mma_prefix_persistent(const DecodeParams& p, const CUtensorMap& km,
+                                         const CUtensorMap& vm, unsigned int* counters,
+                                         int prefix_parts, cudaStream_t stream) {
+  PKV_MMA_PREFIX_PERSISTENT_CASE(64, 8)
+  PKV_MMA_PREFIX_PERSISTENT_CASE(64, 16)
+  PKV_MMA_PREFIX_PERSISTENT_CASE(64, 32)
+  PKV_MMA_PREFIX_PERSISTENT_CASE(64, 64)
+  PKV_MMA_PREFIX_PERSISTENT_CASE(128, 8)
+  PKV_MMA_PREFIX_PERSISTENT_CASE(128, 16)
+  PKV_MMA_PREFIX_PERSISTENT_CASE(128, 32)
+  PKV_MMA_PREFIX_PERSISTENT_CASE(128, 64)
   return cudaErrorInvalidValue;
 }
 

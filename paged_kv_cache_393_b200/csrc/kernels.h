@@ -99,7 +99,13 @@ constexpr size_t WORK_COUNTER_BYTES = 16;
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& k_map,
                                          const CUtensorMap& v_map, unsigned int* counters,
                                          bool split, cudaStream_t stream);
-size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_seqs);
+// Shared-prefix pass on the same persistent grid: work items (group, kv head,
+// prefix partition) from the ticket counters[2]; the columns of an item's tile
+// are the group's usable members' query heads of that kv head.
+cudaError_t launch_mma_prefix_persistent(const DecodeParams& p, const CUtensorMap& k_map,
+                                         const CUtensorMap& v_map, unsigned int* counters,
+                                         int prefix_parts, cudaStream_t stream);
+size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_rows, bool prefix = false);
 constexpr int PERSISTENT_MAX_SEQS = 1024;
 
 // Shared-prefix pass: CTA = (kv head, group, prefix partition); the members'

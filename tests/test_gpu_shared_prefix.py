@@ -189,17 +189,27 @@ def test_forked_batches(pkv, case, fused):
 
 
 @pytest.mark.parametrize("H,Hk", [(8, 8), (8, 2)], ids=["mha", "gqa"])
-def test_bounds_below_the_real_lengths_are_flagged(pkv, H, Hk):
+def test_bounds_below_the_real_lengths(pkv, H, Hk):
     fb = ForkBatch(pkv, H, Hk, 128, 16, [1000, 300], 4, lambda i: 100 * i)
     pre, groups = fb.groups()
     mp, ms = _bounds(fb, pre, groups)
     fb.write_new_tokens()
-    for bad in ((mp - 512, ms), (mp, 16)):           # one partition short
+    ref, _, _, _ = fb.expected(list(range(len(fb.seqs))))
+
+    def run(mp_, ms_):
+        fb.out.fill_(float("nan"))
         pkv.paged_attention_decode_shared_prefix(
             fb.out, fb.q, fb.kc, fb.vc, fb.tables, fb.lens, torch.from_numpy(pre).to(DEV),
             torch.from_numpy(groups).to(DEV), 1.0 / fb.D ** 0.5, fb.max_context_len, 64,
-            max_prefix_tokens=bad[0], max_suffix_tokens=bad[1])
-        assert pkv.device_errors() & pkv.DEVERR_PREFIX
+            max_prefix_tokens=mp_, max_suffix_tokens=ms_)
+        return pkv.device_errors()
+
+    # the persistent prefix pass takes every group's items from its queue: a prefix bound
+    # one partition short only sizes its grid, and the result is still complete
+    assert run(mp - 512, ms) == 0
+    assert_attention_close(fb.out.cpu().numpy(), ref)
+    # a suffix bound one partition short leaves work undone and says so
+    assert run(mp, 16) & pkv.DEVERR_PREFIX
 
 
 def test_more_sequences_than_the_persistent_grid(pkv):

@@ -91,6 +91,15 @@ class PagedBatch:
         self.out = torch.empty((B, w.num_heads, w.head_dim), dtype=torch.float16, device=dev)
 
 
+    @property
+    def scale(self) -> float:
+        return self.w.scale
+
+    def kv_bytes(self) -> int:
+        """Algorithmic K+V bytes one attention pass reads."""
+        return int(self.lens_host.astype(np.int64).sum()) * wl.kv_bytes_per_token(
+            self.w.num_kv_heads, self.w.head_dim)
+
 def _prefill(batches, chunk_tokens):
     """Writes the prompts of every batch, drawing each sequence's K/V values once (the
     batches differ only in block size and pool)."""
@@ -123,15 +132,6 @@ def paged_batches(ws, device, prefill_chunk_tokens: int = 1 << 17):
     for gb in out:
         gb._finish()
     return out
-
-    @property
-    def scale(self) -> float:
-        return self.w.scale
-
-    def kv_bytes(self) -> int:
-        """Algorithmic K+V bytes one attention pass reads."""
-        return int(self.lens_host.astype(np.int64).sum()) * wl.kv_bytes_per_token(
-            self.w.num_kv_heads, self.w.head_dim)
 
 
 class CowBatch:

@@ -124,14 +124,15 @@ PAGEDKV_API int pagedkv_selftest_wait_timeout(unsigned int timeout_us, void *str
  *                  second kernel.
  *   workspace      device scratch of at least paged_attention_workspace_bytes(...)
  *                  bytes (16-byte aligned); may be NULL when that function returns
- *                  0.  Its first 16 bytes are work counters (grouped queries, 2..8
+ *                  0.  Its first 32 bytes are work counters (grouped queries, 2..8
  *                  query heads per kv head, take their work items from them): they
  *                  must be zero before the workspace's first use -- allocate it
  *                  zeroed or cudaMemsetAsync them once -- and every call leaves
- *                  them zero again.  A launch that finds them not zero sets
- *                  PAGEDKV_DEVERR_INTERNAL (its outputs are then invalid) and
- *                  still leaves them zero.  The rest holds the split-K partial
- *                  results, needs no initialization and is garbage afterwards.
+ *                  them zero again.  A launch that finds its ticket not at zero
+ *                  sets PAGEDKV_DEVERR_INTERNAL (some outputs are then invalid);
+ *                  zero the counters again after that flag.  The rest holds the
+ *                  split-K partial results, needs no initialization and is
+ *                  garbage afterwards.
  *                  Calls that may run at the same time need separate workspaces.
  *
  * num_seqs == 0 is a no-op.  Errors: EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA.
@@ -207,7 +208,10 @@ PAGEDKV_API int paged_attention_decode_append(void *out, const void *q,
  *
  *   seq_prefix_tokens  device int32 [num_seqs]: P_b, the tokens of sequence b
  *                  that its group's prefix pass covers; 0 = none.  A multiple of
- *                  block_size and at most L_b - 1.
+ *                  block_size and at most L_b - 1.  A sequence with P_b > 0 must
+ *                  be a member of a group: one that no group lists is not
+ *                  detected on the device (its output is then invalid);
+ *                  paged_decode_step_host checks this on the host.
  *   groups         device int32 [num_groups][PAGEDKV_GROUP_WIDTH]: the group's
  *                  prefix length in blocks, then up to 8 member sequence indices
  *                  (-1 = unused).  A group may hold at most 8 / G members
@@ -314,7 +318,9 @@ PAGEDKV_API int pagedkv_prefix_groups(const int32_t *block_tables, const int32_t
  *                     destination repeated or used as a source (EINVAL otherwise).
  *   seq_prefix_tokens_host, groups_host, num_groups
  *                     NULL / NULL / 0 for the plain step; else host arrays as
- *                     pagedkv_prefix_groups writes them (num_groups <= num_seqs / 2)
+ *                     pagedkv_prefix_groups writes them (num_groups <= num_seqs / 2);
+ *                     a sequence with prefix tokens that no group lists with that
+ *                     prefix length is refused (EINVAL)
  *   key_cache,
  *   value_cache       device pools as for paged_attention_decode (one layer)
  *   staging           device buffer of paged_decode_step_staging_bytes(...) bytes,
@@ -374,8 +380,9 @@ PAGEDKV_API int paged_attention_partition_tokens(int num_seqs, int num_heads, in
  *    capture on that device.
  *  - All calls on a device share the array and leave their partial results in
  *    it; calls that can overlap on the GPU (other streams, other threads) race.
- *    Its work counters are cleared at that first call's set-up (on its stream)
- *    and every call leaves them zero; nothing else needs to start at zero.
+ *    Its work counters (the first 32 bytes) are cleared at that first call's
+ *    set-up (on its stream) and every call leaves them zero; nothing else needs
+ *    to start at zero.
  */
 #define PAGEDKV_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 

@@ -446,8 +446,8 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
     st = encode_pool_map(&vm, value_cache, rows, head_dim, block_size);
     if (st != PAGEDKV_OK) return st;
   }
-  // work counters (self-resetting: the last CTA of a persistent launch zeroes its pair):
-  // [0] [1] the decode pass's ticket and finished-CTA count, [2] [3] the prefix pass's
+  // work counters (self-resetting: the last CTA of a persistent launch zeroes its pass's
+  // 16 bytes): the decode pass's first, then the prefix pass's
   unsigned int* counters =
       plan.ws_bytes > 0 ? reinterpret_cast<unsigned int*>(workspace) : nullptr;
   const bool prefix_pass = cascade && num_groups > 0;
@@ -615,6 +615,25 @@ struct StepLayout {
   size_t ws_bytes, total;
 };
 
+// The plain host step splits a batch into chunks of sequences so that uploading
+// chunk c + 1 and downloading chunk c - 1 overlap the attention of chunk c: up to
+// STEP_MAX_CHUNKS chunks of at least STEP_CHUNK_SEQS sequences.  The shared-prefix
+// step runs whole (its groups span the batch).
+constexpr int STEP_MAX_CHUNKS = 4;
+constexpr int STEP_CHUNK_SEQS = 64;
+
+int step_chunks(int num_seqs, bool shared_prefix) {
+  if (shared_prefix) return 1;
+  const int c = num_seqs / STEP_CHUNK_SEQS;
+  return c < 1 ? 1 : (c > STEP_MAX_CHUNKS ? STEP_MAX_CHUNKS : c);
+}
+
+// Sequences [first, first + count) of chunk i of n.
+void chunk_range(int num_seqs, int n, int i, int* first, int* count) {
+  *first = (int)((long long)num_seqs * i / n);
+  *count = (int)((long long)num_seqs * (i + 1) / n) - *first;
+}
+
 int step_layout(StepLayout* lay, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                 int block_size, int max_blocks_per_seq, int max_context_len, int partition_size,
                 int max_pairs, bool shared_prefix) {
@@ -641,8 +660,20 @@ int step_layout(StepLayout* lay, int num_seqs, int num_heads, int num_kv_heads, 
   lay->out = take(B * H * D * 2);
   lay->prefix = shared_prefix ? take(B * 4) : 0;
   lay->groups = shared_prefix ? take((B / 2 > 0 ? B / 2 : 1) * GROUP_WIDTH * 4) : 0;
-  lay->ws = take(plan.ws_bytes);
-  lay->ws_bytes = plan.ws_bytes;
+  // the chunks run one after another and share the workspace: size it for the
+  // largest plan among the whole batch and its chunks
+  size_t ws = plan.ws_bytes;
+  const int n = step_chunks(num_seqs, shared_prefix);
+  for (int i = 0; i < n && n > 1; ++i) {
+    int first = 0, count = 0;
+    chunk_range(num_seqs, n, i, &first, &count);
+    Plan cp;
+    if (make_plan(&cp, count, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                  partition_size, false) == PAGEDKV_OK && cp.ws_bytes > ws)
+      ws = cp.ws_bytes;
+  }
+  lay->ws = take(ws);
+  lay->ws_bytes = ws;
   lay->total = off;
   return PAGEDKV_OK;
 }
@@ -670,6 +701,45 @@ int h2d(void* dst, const void* src, size_t bytes, cudaStream_t s, const char* wh
   const cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s);
   return e == cudaSuccess ? PAGEDKV_OK : cuda_fail(e, what);
 }
+
+// Copy streams and events of the pipelined host step, per host thread and device,
+// created at the first chunked call and kept until the process exits.
+struct StepAux {
+  cudaStream_t up, down;
+  cudaEvent_t start, small, done, in[STEP_MAX_CHUNKS], out[STEP_MAX_CHUNKS];
+  bool ready;
+};
+thread_local StepAux tl_step_aux[MAX_DEVICES];
+
+int step_aux(StepAux** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= MAX_DEVICES) return fail(PAGEDKV_ECUDA, "device id %d out of range", dev);
+  StepAux& a = tl_step_aux[dev];
+  if (!a.ready) {
+    if ((e = cudaStreamCreateWithFlags(&a.up, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&a.down, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "creating the copy streams");
+    cudaEvent_t* evs[3 + 2 * STEP_MAX_CHUNKS] = {&a.start, &a.small, &a.done};
+    for (int i = 0; i < STEP_MAX_CHUNKS; ++i) {
+      evs[3 + i] = &a.in[i];
+      evs[3 + STEP_MAX_CHUNKS + i] = &a.out[i];
+    }
+    for (cudaEvent_t* ev : evs)
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_fail(e, "creating the step's events");
+    a.ready = true;
+  }
+  *out = &a;
+  return PAGEDKV_OK;
+}
+
+#define PKV_CHECK_CUDA(call, what)                 \
+  do {                                             \
+    const cudaError_t e_ = (call);                 \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
 
 }  // namespace
 }  // namespace pkv
@@ -735,9 +805,23 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
       if (pb > 0 && (long long)pb * block_size > max_prefix)
         max_prefix = (int)std::min<long long>((long long)pb * block_size, max_context_len);
     }
+    // every sequence with a prefix must be a member of a group with that prefix length
+    // (the device path cannot see a sequence that no group lists)
+    std::vector<char> listed((size_t)num_seqs, 0);
+    for (int g = 0; g < num_groups; ++g) {
+      const int32_t* gd = groups_host + (size_t)g * GROUP_WIDTH;
+      for (int i = 1; i < GROUP_WIDTH; ++i) {
+        const int m = gd[i];
+        if (m >= 0 && m < num_seqs && seq_prefix_tokens_host[m] == gd[0] * block_size)
+          listed[(size_t)m] = 1;
+      }
+    }
     for (int b = 0; b < num_seqs; ++b) {
       const int P = seq_prefix_tokens_host[b];
       const int L = context_lens_host[b];
+      if (P != 0 && !listed[(size_t)b])
+        return fail(PAGEDKV_EINVAL, "sequence %d has %d prefix tokens but no group lists it", b,
+                    P);
       // a prefix length the kernels reject counts as 0 (they flag it)
       const int rest = (P > 0 && P % block_size == 0 && P <= L - 1) ? L - P : L;
       max_suffix = rest > max_suffix ? rest : max_suffix;
@@ -748,6 +832,73 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
   char* base = static_cast<char*>(staging);
   const size_t B = (size_t)num_seqs, H = (size_t)num_heads, Hk = (size_t)num_kv_heads,
                D = (size_t)head_dim;
+  const int nch = step_chunks(num_seqs, shared);
+  if (nch > 1) {
+    // Pipelined: the uploads run on a copy stream, chunk by chunk, and each chunk's
+    // attention starts as soon as its inputs have landed; each chunk's output is
+    // downloaded on a second copy stream while the next chunk computes.  The
+    // caller's stream waits for the last download, so work it enqueues later (the
+    // next step overwriting this staging) comes after all of it.
+    StepAux* aux = nullptr;
+    if ((st = step_aux(&aux)) != PAGEDKV_OK) return st;
+    const size_t row_q = H * D * 2, row_kv = Hk * D * 2, row_t = (size_t)max_blocks_per_seq * 4;
+    PKV_CHECK_CUDA(cudaEventRecord(aux->start, s), "step start");
+    PKV_CHECK_CUDA(cudaStreamWaitEvent(aux->up, aux->start, 0), "upload wait");
+    if ((st = h2d(base + lay.tables, block_tables_host, B * row_t, aux->up,
+                  "block table upload")) != PAGEDKV_OK ||
+        (st = h2d(base + lay.lens, context_lens_host, B * 4, aux->up, "context length upload")) !=
+            PAGEDKV_OK ||
+        (st = h2d(base + lay.pairs, copy_pairs_host, (size_t)num_pairs * 16, aux->up,
+                  "pair upload")) != PAGEDKV_OK)
+      return st;
+    PKV_CHECK_CUDA(cudaEventRecord(aux->small, aux->up), "upload event");
+    for (int c = 0; c < nch; ++c) {
+      int first = 0, count = 0;
+      chunk_range(num_seqs, nch, c, &first, &count);
+      const char* qh = static_cast<const char*>(q_host) + first * row_q;
+      const char* kh = static_cast<const char*>(k_new_host) + first * row_kv;
+      const char* vh = static_cast<const char*>(v_new_host) + first * row_kv;
+      if ((st = h2d(base + lay.q + first * row_q, qh, count * row_q, aux->up, "query upload")) !=
+              PAGEDKV_OK ||
+          (st = h2d(base + lay.k + first * row_kv, kh, count * row_kv, aux->up,
+                    "new K upload")) != PAGEDKV_OK ||
+          (st = h2d(base + lay.v + first * row_kv, vh, count * row_kv, aux->up,
+                    "new V upload")) != PAGEDKV_OK)
+        return st;
+      PKV_CHECK_CUDA(cudaEventRecord(aux->in[c], aux->up), "upload event");
+    }
+    PKV_CHECK_CUDA(cudaStreamWaitEvent(s, aux->small, 0), "compute wait");
+    if (num_pairs > 0) {
+      void* kc[1] = {key_cache};
+      void* vc[1] = {value_cache};
+      st = copy_blocks(kc, vc, reinterpret_cast<const int64_t*>(base + lay.pairs), num_pairs, 1,
+                       (size_t)num_kv_heads * block_size * head_dim, num_blocks, stream);
+      if (st != PAGEDKV_OK) return st;
+    }
+    void* ws = lay.ws_bytes ? base + lay.ws : nullptr;
+    for (int c = 0; c < nch; ++c) {
+      int first = 0, count = 0;
+      chunk_range(num_seqs, nch, c, &first, &count);
+      PKV_CHECK_CUDA(cudaStreamWaitEvent(s, aux->in[c], 0), "compute wait");
+      st = paged_attention_decode_append(
+          base + lay.out + first * row_q, base + lay.q + first * row_q,
+          base + lay.k + first * row_kv, base + lay.v + first * row_kv, key_cache, value_cache,
+          reinterpret_cast<const int32_t*>(base + lay.tables + first * row_t),
+          reinterpret_cast<const int32_t*>(base + lay.lens) + first, scale, block_size,
+          num_kv_heads, count, num_heads, head_dim, max_blocks_per_seq, num_blocks,
+          max_context_len, partition_size, ws, lay.ws_bytes, stream);
+      if (st != PAGEDKV_OK) return st;
+      PKV_CHECK_CUDA(cudaEventRecord(aux->out[c], s), "compute event");
+      PKV_CHECK_CUDA(cudaStreamWaitEvent(aux->down, aux->out[c], 0), "download wait");
+      PKV_CHECK_CUDA(cudaMemcpyAsync(static_cast<char*>(out_host) + first * row_q,
+                                     base + lay.out + first * row_q, count * row_q,
+                                     cudaMemcpyDeviceToHost, aux->down),
+                     "output download");
+    }
+    PKV_CHECK_CUDA(cudaEventRecord(aux->done, aux->down), "download event");
+    PKV_CHECK_CUDA(cudaStreamWaitEvent(s, aux->done, 0), "step join");
+    return PAGEDKV_OK;
+  }
   // 1. the step's inputs, host to device (small arrays first)
   if ((st = h2d(base + lay.tables, block_tables_host, B * max_blocks_per_seq * 4, s,
                 "block table upload")) != PAGEDKV_OK ||

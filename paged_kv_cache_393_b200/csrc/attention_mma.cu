@@ -747,23 +747,28 @@ __global__ void __launch_bounds__((NW + 1) * 32)
 // ---- persistent split-K kernel ---------------------------------------------------
 
 struct PersistentArgs {
-  unsigned int* ticket;    // next work item; zero at the start, zeroed again by the last CTA
-  unsigned int* finished;  // CTAs done taking tickets; likewise
+  unsigned int* ticket;          // next work item; zero at the start, zeroed by the last CTA
+  unsigned long long* finished;  // (CTAs done << 32) + items they processed; likewise
   int write_zeros;         // no merge kernel may follow: write the zero outputs of empty contexts
 };
 
-// Run by one thread of each CTA once the CTA takes no more tickets.  The last
-// CTA to get here zeroes both counters for the next launch on this workspace:
-// every CTA has taken its last ticket by then, so nothing can add to them.
-// Without an abort every CTA took exactly one ticket past the last item, so a
-// final count other than total + CTAs means the counter did not start at zero.
+// Run by one thread of each CTA once the CTA takes no more tickets, with the
+// number of items the CTA processed.  The last CTA to get here zeroes both
+// counters for the next launch on this workspace: every CTA has taken its last
+// ticket by then, so nothing can add to them.  Without an abort the CTAs
+// processed every item once and took one ticket each past the last, so any
+// other count means the counters did not start at zero (some items were
+// skipped).
 __device__ __forceinline__ void release_counters(const PersistentArgs& pa, unsigned total,
-                                                 bool check, unsigned* err) {
+                                                 unsigned items, bool check, unsigned* err) {
   __threadfence();
-  if (atomicAdd(pa.finished, 1u) == gridDim.x - 1) {
+  const unsigned long long before = atomicAdd(pa.finished, (1ull << 32) | items);
+  if ((before >> 32) == gridDim.x - 1) {
+    const unsigned processed = (unsigned)(before & 0xffffffffull) + items;
     const unsigned taken = atomicExch(pa.ticket, 0u);
-    atomicExch(pa.finished, 0u);
-    if (check && taken != total + gridDim.x) flag_error(err, ERR_INTERNAL);
+    atomicExch(pa.finished, 0ull);
+    if (check && (processed != total || taken != total + gridDim.x))
+      flag_error(err, ERR_INTERNAL);
     __threadfence();
   }
 }
@@ -887,7 +892,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   if (smem_u32(smem_raw) & 1023u) {
     if (threadIdx.x == 0) {
       flag_error(p.err, ERR_INTERNAL);
-      release_counters(pa, 0, false, p.err);
+      release_counters(pa, 0, 0, false, p.err);
     }
     return;
   }
@@ -1045,6 +1050,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     };
     int4 d;
     bool have = next_item(&d);
+    unsigned items = 0;  // items taken (lane 0's count is the one reported)
     for (int it = 0;; ++it) {
       const bool done = !have || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
       if (done) d = make_int4(0, 0, 0, 0);
@@ -1112,12 +1118,13 @@ __global__ void __launch_bounds__((NW + 1) * 32)
                                stages, ring, &k_map, &v_map, policy, abort_flag, lane, issued))
         break;
       base.advance(nchunks);
+      ++items;
       have = next_item(&d);
     }
     if (lane == 0) {
       const bool aborted = *abort_flag != 0;
       if (aborted) drain_ring(bars, stages, issued);
-      release_counters(pa, (unsigned)total, !aborted, p.err);
+      release_counters(pa, (unsigned)total, items, !aborted, p.err);
     }
     return;
   }
@@ -1265,8 +1272,8 @@ cudaError_t launch_persistent_instance(const DecodeParams& p, const CUtensorMap&
   if (ctas > items) ctas = items;
   if (ctas < 1) ctas = 1;
   PersistentArgs pa;
-  pa.ticket = counters + (PREFIX ? 2 : 0);
-  pa.finished = counters + (PREFIX ? 3 : 1);
+  pa.ticket = counters + (PREFIX ? 4 : 0);
+  pa.finished = reinterpret_cast<unsigned long long*>(counters + (PREFIX ? 6 : 2));
   pa.write_zeros = (!PREFIX && (!split || p.seq_prefix_tokens)) ? 1 : 0;
   return launch_kernel(!PREFIX && p.after_prefix != 0, kernel, dim3((unsigned)ctas),
                        dim3((NW + 1) * 32), smem, stream, km, vm, p, pa);

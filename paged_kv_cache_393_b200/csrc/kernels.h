@@ -67,8 +67,12 @@ inline cudaError_t launch_kernel(bool pdl, void (*kernel)(KArgs...), dim3 grid, 
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Consumer warps of the grouped-query (tensor-core) kernel; plus one producer warp.
-constexpr int MMA_CONSUMER_WARPS = 2;
+// Consumer warps of the grouped-query (tensor-core) kernel; plus one producer warp
+// (fixed at build time; 2 measured best).
+#ifndef PAGEDKV_TUNE_MMA_WARPS
+#define PAGEDKV_TUNE_MMA_WARPS 2
+#endif
+constexpr int MMA_CONSUMER_WARPS = PAGEDKV_TUNE_MMA_WARPS;
 
 // Shared-memory bytes of one ring stage / the whole launch.
 size_t simt_stage_bytes(int head_dim, int block_size, int kvc);
@@ -86,21 +90,22 @@ cudaError_t launch_simt_decode(const DecodeParams& p, int hpc, int kvc, bool spl
 cudaError_t launch_mma_decode(const DecodeParams& p, const CUtensorMap& k_map,
                               const CUtensorMap& v_map, bool split, cudaStream_t stream);
 
-// Work counters at the start of every workspace: counters[0] is the ticket of the
-// persistent decode kernel and counters[1] its count of finished CTAs (the last
-// CTA zeroes both); counters[2..3] are the same pair for the shared-prefix pass.
+// Work counters at the start of every workspace, 16 bytes per persistent pass
+// (the decode pass, then the shared-prefix pass): a 32-bit ticket, 4 unused
+// bytes, and a 64-bit word of finished CTAs (high half) and items they
+// processed (low half); the last CTA of a launch zeroes its pass's counters.
 // They must be zero before a workspace's first use and every launch leaves
 // them zero.
-constexpr size_t WORK_COUNTER_BYTES = 16;
+constexpr size_t WORK_COUNTER_BYTES = 32;
 
 // Persistent tensor-core kernel: a few CTAs per SM take (b, kv head, partition)
-// work items from the ticket counters[0].  Without a split every item is a
+// work items from the decode pass's ticket (counters[0]).  Without a split every item is a
 // whole context.
 cudaError_t launch_mma_decode_persistent(const DecodeParams& p, const CUtensorMap& k_map,
                                          const CUtensorMap& v_map, unsigned int* counters,
                                          bool split, cudaStream_t stream);
 // Shared-prefix pass on the same persistent grid: work items (group, kv head,
-// prefix partition) from the ticket counters[2]; the columns of an item's tile
+// prefix partition) from the prefix pass's ticket (counters[4]); the columns of an item's tile
 // are the group's usable members' query heads of that kv head.
 cudaError_t launch_mma_prefix_persistent(const DecodeParams& p, const CUtensorMap& k_map,
                                          const CUtensorMap& v_map, unsigned int* counters,

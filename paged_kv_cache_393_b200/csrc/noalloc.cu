@@ -16,7 +16,7 @@
 // needing more are rejected.  All calls on a device share it, and each call
 // leaves its partial results behind: calls that may run on the GPU at the same
 // time (different streams, or different host threads) corrupt each other's
-// results, so serialize them.  Its first 16 bytes are the work counters of the
+// results, so serialize them.  Its first 32 bytes are the work counters of the
 // grouped-query kernel, which must start at zero: they are cleared once, when a
 // device's address is looked up, and every call leaves them at zero.  Every
 // partial result a call reads was written earlier in that same call.
@@ -34,7 +34,7 @@ int record_error(int code, const char* message);
 namespace {
 
 constexpr size_t kScratchBytes = PAGEDKV_NOALLOC_SCRATCH_BYTES;
-constexpr size_t kCounterBytes = 16;  // the work counters at the start of every workspace
+constexpr size_t kCounterBytes = 32;  // the work counters at the start of every workspace
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 

@@ -128,10 +128,15 @@ size_t split_merge_smem_bytes(int num_parts) {
 cudaError_t launch_split_reduce(const DecodeParams& p, cudaStream_t stream) {
   const long long rows = (long long)p.num_seqs * p.num_heads;
   const dim3 grid((unsigned)((rows + MERGE_WARPS - 1) / MERGE_WARPS));
+  // A programmatic dependent of the partition pass, except after a shared-prefix
+  // pass: then the merge also reads the prefix pass's partials, and a suffix
+  // CTA that exits early never waits for that pass, so the merge is ordered
+  // behind both the ordinary way (its griddepcontrol.wait then returns at once).
+  const bool pdl = p.after_prefix == 0;
   if (p.head_dim == 64)
-    return launch_kernel(true, split_merge_kernel<64>, grid, dim3(MERGE_WARPS * 32), 0, stream, p);
+    return launch_kernel(pdl, split_merge_kernel<64>, grid, dim3(MERGE_WARPS * 32), 0, stream, p);
   if (p.head_dim == 128)
-    return launch_kernel(true, split_merge_kernel<128>, grid, dim3(MERGE_WARPS * 32), 0, stream,
+    return launch_kernel(pdl, split_merge_kernel<128>, grid, dim3(MERGE_WARPS * 32), 0, stream,
                          p);
   return cudaErrorInvalidValue;
 }

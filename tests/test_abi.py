@@ -134,13 +134,13 @@ def test_shared_prefix_rejects_bad_arguments_on_the_host(lib, kw, code):
 
 
 def test_shared_prefix_workspace_bytes(lib):
-    # 16 bytes of work counters, then the partials: always split at 512 (or the given size),
+    # 32 bytes of work counters, then the partials: always split at 512 (or the given size),
     # with one extra slot per (sequence, head)
     f = lib.paged_attention_shared_prefix_workspace_bytes
-    assert f(4, 8, 8, 128, 16, 1200, 0) == 16 + 4 * 8 * (3 + 1) * 130 * 4
-    assert f(4, 8, 8, 128, 16, 1200, -1) == 16 + 4 * 8 * (3 + 1) * 130 * 4
-    assert f(4, 8, 8, 64, 16, 1200, 256) == 16 + 4 * 8 * (5 + 1) * 66 * 4
-    assert f(4, 16, 8, 128, 16, 1200, 0) == 16 + 4 * 16 * 4 * 130 * 4
+    assert f(4, 8, 8, 128, 16, 1200, 0) == 32 + 4 * 8 * (3 + 1) * 130 * 4
+    assert f(4, 8, 8, 128, 16, 1200, -1) == 32 + 4 * 8 * (3 + 1) * 130 * 4
+    assert f(4, 8, 8, 64, 16, 1200, 256) == 32 + 4 * 8 * (5 + 1) * 66 * 4
+    assert f(4, 16, 8, 128, 16, 1200, 0) == 32 + 4 * 16 * 4 * 130 * 4
     assert f(4, 8, 8, 128, 4, 1200, 0) == 0            # rejected: block_size 4
 
 
@@ -154,28 +154,28 @@ def test_empty_batch_is_a_no_op(lib):
 
 
 def test_workspace_bytes(lib):
-    # every workspace starts with 16 bytes of work counters, then the split-K partials
+    # every workspace starts with 32 bytes of work counters, then the split-K partials
     # single pass over one kv head per query head: no workspace
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, -1) == 0
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 512, 0) == 0
     # CUDA-core kernel, automatic: 512-token partitions for the 256-sequence batch, halved to
     # 128 for 32 sequences (2 kv heads per CTA: 512 CTAs per partition, ~4 waves wanted)
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, 0) == \
-        16 + 256 * 32 * 3 * 130 * 4
+        32 + 256 * 32 * 3 * 130 * 4
     assert pkv.paged_attention_workspace_bytes(32, 32, 32, 128, 16, 1524, 0) == \
-        16 + 32 * 32 * 12 * 130 * 4
+        32 + 32 * 32 * 12 * 130 * 4
     # explicit split: B * H * P * (D + 2) floats (CUDA-core kernel, MHA)
-    assert pkv.paged_attention_workspace_bytes(4, 8, 8, 64, 16, 1000, 256) == 16 + 4 * 8 * 4 * 66 * 4
+    assert pkv.paged_attention_workspace_bytes(4, 8, 8, 64, 16, 1000, 256) == 32 + 4 * 8 * 4 * 66 * 4
     # tensor-core split-K (persistent CTAs fed by the work counter)
-    assert pkv.paged_attention_workspace_bytes(4, 8, 2, 64, 16, 1000, 256) == 16 + 4 * 8 * 4 * 66 * 4
+    assert pkv.paged_attention_workspace_bytes(4, 8, 2, 64, 16, 1000, 256) == 32 + 4 * 8 * 4 * 66 * 4
     # long GQA contexts split automatically into 512-token partitions
     assert pkv.paged_attention_workspace_bytes(128, 64, 8, 128, 16, 16384, 0) == \
-        16 + 128 * 64 * 32 * 130 * 4
+        32 + 128 * 64 * 32 * 130 * 4
     # grouped queries in a single pass still take their work from the counter
-    assert pkv.paged_attention_workspace_bytes(128, 64, 8, 128, 16, 2048, -1) == 16
+    assert pkv.paged_attention_workspace_bytes(128, 64, 8, 128, 16, 2048, -1) == 32
     # beyond 1024 sequences the tensor-core split runs one CTA per item (the counters unused)
     assert pkv.paged_attention_workspace_bytes(1100, 16, 2, 64, 16, 1000, 512) == \
-        16 + 1100 * 16 * 2 * 66 * 4
+        32 + 1100 * 16 * 2 * 66 * 4
     assert pkv.paged_attention_workspace_bytes(1, 8, 3, 64, 16, 100, 0) == 0     # rejected shape
 
 
@@ -275,3 +275,12 @@ def test_host_step_staging_bytes(lib):
     assert f(B, H, Hk, D, bs, maxblk, maxlen, 0, 224, 1) == \
         want - r(ws) + r(B * 4) + r(B // 2 * 9 * 4) + r(ws2)
     assert f(B, H, Hk, 96, bs, maxblk, maxlen, 0, 0, 0) == 0    # rejected head_dim
+
+
+def test_host_step_refuses_a_prefix_no_group_lists(lib):
+    import numpy as np
+    # sequence 1 claims 16 prefix tokens, but the only group lists sequences 0 and 2
+    groups = np.array([[1, 0, 2, -1, -1, -1, -1, -1, -1]], np.int32)
+    assert _host_step(lib, lens=[40, 40, 40, 40], pre=[16, 16, 16, 0], groups=groups, ng=1) == \
+        nat.EINVAL
+    assert b"no group" in lib.pagedkv_last_error()

@@ -189,14 +189,14 @@ def test_work_counters_are_left_zero_and_a_dirty_start_is_flagged(pkv, part):
         torch.cuda.synchronize()
 
     run()
-    assert pkv.device_errors() == 0 and (ws[:16] == 0).all()
+    assert pkv.device_errors() == 0 and (ws[:32] == 0).all()
     ref = _bits(gb.out)
     run()
     assert pkv.device_errors() == 0 and np.array_equal(ref, _bits(gb.out))
     ws[0] = 5                                      # a ticket count left by someone else
     run()
     assert pkv.device_errors() & pkv.DEVERR_INTERNAL
-    assert (ws[:16] == 0).all()
+    assert (ws[:32] == 0).all()
     run()
     assert pkv.device_errors() == 0 and np.array_equal(ref, _bits(gb.out))
 

@@ -120,6 +120,9 @@ constexpr size_t MAX_SMEM = 227 * 1024;
 #ifndef PAGEDKV_TUNE_PERSISTENT
 #define PAGEDKV_TUNE_PERSISTENT 1
 #endif
+#ifndef PAGEDKV_TUNE_PREFIX_HALF
+#define PAGEDKV_TUNE_PREFIX_HALF 0          // 1: shared prefixes in half-size partitions
+#endif
 
 struct Plan {
   bool mma = false;
@@ -127,6 +130,7 @@ struct Plan {
   int hpc = 1, kvc = 1;      // CUDA-core kernel: query heads / kv heads per CTA
   bool split = false;
   int part_tokens = 0;
+  int prefix_part_tokens = 0;  // shared-prefix decode: tokens per prefix partition
   int num_parts = 1;
   int stages = 2;
   size_t smem = 0;
@@ -162,6 +166,9 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
                 "head (block_size %d, %d)", block_size, G);
   Plan p;
   p.cascade = cascade;
+  // tensor cores for query groups (running the suffix pass of a shared-prefix call for one kv
+  // head per query head on them too was measured slower: every suffix item folds the prefix
+  // partials, so the persistent suffix CTAs wait for the whole prefix pass)
   p.mma = G >= 2 && G <= 8 && block_size >= 8;
   if (!p.mma) {
     if (G == 1) {
@@ -225,9 +232,18 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
                 partition_size);
   }
   (void)unit;
+  // A shared prefix can be split into partitions of its own size (finer prefix items
+  // balance the persistent grid better, but measured slower overall: more prefix partials
+  // to write and to fold in).
+  p.prefix_part_tokens = p.part_tokens;
+  if (PAGEDKV_TUNE_PREFIX_HALF && cascade && partition_size <= 0 &&
+      (p.part_tokens / 2) % align == 0)
+    p.prefix_part_tokens = p.part_tokens / 2;
   if (p.split) {
-    // a shared prefix can end inside a partition: one more slot per (sequence, head)
-    p.num_parts = (max_context_len + p.part_tokens - 1) / p.part_tokens + (cascade ? 1 : 0);
+    // slots: the prefix partitions, then the rest's; a shared prefix can end inside a
+    // partition, so one more slot per (sequence, head)
+    p.num_parts = cascade ? (max_context_len + p.prefix_part_tokens - 1) / p.prefix_part_tokens + 1
+                          : (max_context_len + p.part_tokens - 1) / p.part_tokens;
     if (p.num_parts > MAX_PARTITIONS)
       return fail(PAGEDKV_EUNSUPPORTED, "%d partitions exceed %d: use a larger partition_size",
                   p.num_parts, MAX_PARTITIONS);
@@ -419,6 +435,7 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
   p.num_blocks = num_blocks;
   p.max_context_len = max_context_len;
   p.part_tokens = plan.part_tokens;
+  p.prefix_part_tokens = plan.prefix_part_tokens;
   p.num_parts = plan.num_parts;
   p.grid_parts = plan.num_parts;
   if (cascade && max_suffix_tokens > 0) {
@@ -459,9 +476,10 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
     pp.stages = plan.prefix_stages;
     pp.k_new = pp.v_new = nullptr;
     pp.no_merge = 0;  // its partial results are always folded in later
-    int prefix_parts = (max_context_len + plan.part_tokens - 1) / plan.part_tokens;
+    const int ppt = plan.prefix_part_tokens;
+    int prefix_parts = (max_context_len + ppt - 1) / ppt;
     if (max_prefix_tokens > 0) {
-      const int need = (max_prefix_tokens + plan.part_tokens - 1) / plan.part_tokens;
+      const int need = (max_prefix_tokens + ppt - 1) / ppt;
       if (need < prefix_parts) prefix_parts = need;
     }
     // persistent CTAs stream the prefix items from a ticket queue; beyond the
@@ -611,14 +629,16 @@ size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
 // Offsets of the regions of the caller's staging buffer (each 256-byte aligned).
 struct StepLayout {
-  size_t q, k, v, tables, lens, pairs, out, prefix, groups, ws;
+  size_t q, k, v, tables, lens, pairs, out, prefix, groups, ws, ws2;
   size_t ws_bytes, total;
 };
 
 // The plain host step splits a batch into chunks of sequences so that uploading
 // chunk c + 1 and downloading chunk c - 1 overlap the attention of chunk c: up to
-// STEP_MAX_CHUNKS chunks of at least STEP_CHUNK_SEQS sequences.  The shared-prefix
-// step runs whole (its groups span the batch).
+// STEP_MAX_CHUNKS chunks of at least STEP_CHUNK_SEQS sequences, alternating over
+// two compute streams (each with its own workspace) so that one chunk's last
+// CTAs and merge overlap the next chunk's start.  The shared-prefix step runs
+// whole (its groups span the batch).
 constexpr int STEP_MAX_CHUNKS = 4;
 constexpr int STEP_CHUNK_SEQS = 64;
 
@@ -673,6 +693,7 @@ int step_layout(StepLayout* lay, int num_seqs, int num_heads, int num_kv_heads, 
       ws = cp.ws_bytes;
   }
   lay->ws = take(ws);
+  lay->ws2 = n > 1 ? take(ws) : lay->ws;  // the second compute stream's workspace
   lay->ws_bytes = ws;
   lay->total = off;
   return PAGEDKV_OK;
@@ -705,8 +726,8 @@ int h2d(void* dst, const void* src, size_t bytes, cudaStream_t s, const char* wh
 // Copy streams and events of the pipelined host step, per host thread and device,
 // created at the first chunked call and kept until the process exits.
 struct StepAux {
-  cudaStream_t up, down;
-  cudaEvent_t start, small, done, in[STEP_MAX_CHUNKS], out[STEP_MAX_CHUNKS];
+  cudaStream_t up, down, comp;  // uploads, downloads, the second compute stream
+  cudaEvent_t start, small, copied, done, in[STEP_MAX_CHUNKS], out[STEP_MAX_CHUNKS];
   bool ready;
 };
 thread_local StepAux tl_step_aux[MAX_DEVICES];
@@ -719,12 +740,13 @@ int step_aux(StepAux** out) {
   StepAux& a = tl_step_aux[dev];
   if (!a.ready) {
     if ((e = cudaStreamCreateWithFlags(&a.up, cudaStreamNonBlocking)) != cudaSuccess ||
-        (e = cudaStreamCreateWithFlags(&a.down, cudaStreamNonBlocking)) != cudaSuccess)
-      return cuda_fail(e, "creating the copy streams");
-    cudaEvent_t* evs[3 + 2 * STEP_MAX_CHUNKS] = {&a.start, &a.small, &a.done};
+        (e = cudaStreamCreateWithFlags(&a.down, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&a.comp, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "creating the step's streams");
+    cudaEvent_t* evs[4 + 2 * STEP_MAX_CHUNKS] = {&a.start, &a.small, &a.copied, &a.done};
     for (int i = 0; i < STEP_MAX_CHUNKS; ++i) {
-      evs[3 + i] = &a.in[i];
-      evs[3 + STEP_MAX_CHUNKS + i] = &a.out[i];
+      evs[4 + i] = &a.in[i];
+      evs[4 + STEP_MAX_CHUNKS + i] = &a.out[i];
     }
     for (cudaEvent_t* ev : evs)
       if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
@@ -875,26 +897,32 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
                        (size_t)num_kv_heads * block_size * head_dim, num_blocks, stream);
       if (st != PAGEDKV_OK) return st;
     }
-    void* ws = lay.ws_bytes ? base + lay.ws : nullptr;
+    // the second compute stream starts after the copies (and after earlier work on s)
+    PKV_CHECK_CUDA(cudaEventRecord(aux->copied, s), "copy event");
+    PKV_CHECK_CUDA(cudaStreamWaitEvent(aux->comp, aux->copied, 0), "compute wait");
     for (int c = 0; c < nch; ++c) {
       int first = 0, count = 0;
       chunk_range(num_seqs, nch, c, &first, &count);
-      PKV_CHECK_CUDA(cudaStreamWaitEvent(s, aux->in[c], 0), "compute wait");
+      // even chunks on the caller's stream, odd ones on the second, each with its workspace
+      cudaStream_t cs = (c & 1) ? aux->comp : s;
+      void* ws = lay.ws_bytes ? base + ((c & 1) ? lay.ws2 : lay.ws) : nullptr;
+      PKV_CHECK_CUDA(cudaStreamWaitEvent(cs, aux->in[c], 0), "compute wait");
       st = paged_attention_decode_append(
           base + lay.out + first * row_q, base + lay.q + first * row_q,
           base + lay.k + first * row_kv, base + lay.v + first * row_kv, key_cache, value_cache,
           reinterpret_cast<const int32_t*>(base + lay.tables + first * row_t),
           reinterpret_cast<const int32_t*>(base + lay.lens) + first, scale, block_size,
           num_kv_heads, count, num_heads, head_dim, max_blocks_per_seq, num_blocks,
-          max_context_len, partition_size, ws, lay.ws_bytes, stream);
+          max_context_len, partition_size, ws, lay.ws_bytes, cs);
       if (st != PAGEDKV_OK) return st;
-      PKV_CHECK_CUDA(cudaEventRecord(aux->out[c], s), "compute event");
+      PKV_CHECK_CUDA(cudaEventRecord(aux->out[c], cs), "compute event");
       PKV_CHECK_CUDA(cudaStreamWaitEvent(aux->down, aux->out[c], 0), "download wait");
       PKV_CHECK_CUDA(cudaMemcpyAsync(static_cast<char*>(out_host) + first * row_q,
                                      base + lay.out + first * row_q, count * row_q,
                                      cudaMemcpyDeviceToHost, aux->down),
                      "output download");
     }
+    // the caller's stream joins the downloads (which follow every chunk's kernels)
     PKV_CHECK_CUDA(cudaEventRecord(aux->done, aux->down), "download event");
     PKV_CHECK_CUDA(cudaStreamWaitEvent(s, aux->done, 0), "step join");
     return PAGEDKV_OK;

@@ -92,7 +92,9 @@ struct StageGeom {
   static constexpr uint32_t TILE_BYTES = NSL * SLICE_BYTES;    // K (or V) of one stage
   static constexpr int MT = D / 16;                            // 16-wide slices of D
   static constexpr int OSTRIDE = D + 4;                        // padded merge rows
-  static constexpr uint32_t MERGE_BYTES = NW * 8 * (2 + OSTRIDE) * 4;
+  // one consumer warp's softmax state for the per-item merge: max[8], sum[8], o[8][OSTRIDE]
+  static constexpr int STATE_FLOATS = 16 + 8 * OSTRIDE;
+  static_assert(STATE_FLOATS * 4 <= 2 * TILE_BYTES, "a warp's state must fit one ring stage");
 };
 
 // ---- producer side ---------------------------------------------------------------
@@ -350,10 +352,10 @@ __device__ __forceinline__ void load_q_column(uint32_t (&qb)[D / 16][2], const _
   }
 }
 
-// Each warp's state into the merge buffers (after the per-head sums are reduced).
+// A warp's state into its merge buffer (after the per-head sums are reduced):
+// buf[0..7] the maxima, buf[8..15] the sums, buf[16..] the [8][OSTRIDE] outputs.
 template <int D>
-__device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, float* s_o, int warp,
-                                            int lane) {
+__device__ __forceinline__ void write_state(Acc<D>& a, float* buf, int lane) {
   using Geo = StageGeom<D>;
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -362,12 +364,12 @@ __device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, f
     a.l1 += __shfl_xor_sync(0xffffffffu, a.l1, off);
   }
   if (g == 0) {
-    s_m[warp * 8 + 2 * t] = a.m0;
-    s_m[warp * 8 + 2 * t + 1] = a.m1;
-    s_l[warp * 8 + 2 * t] = a.l0;
-    s_l[warp * 8 + 2 * t + 1] = a.l1;
+    buf[2 * t] = a.m0;
+    buf[2 * t + 1] = a.m1;
+    buf[8 + 2 * t] = a.l0;
+    buf[8 + 2 * t + 1] = a.l1;
   }
-  float* so = s_o + warp * 8 * Geo::OSTRIDE;
+  float* so = buf + 16;
 #pragma unroll
   for (int mt = 0; mt < Geo::MT; ++mt) {
     so[(2 * t) * Geo::OSTRIDE + mt * 16 + g] = a.o[mt][0];
@@ -381,9 +383,10 @@ __device__ __forceinline__ void write_state(Acc<D>& a, float* s_m, float* s_l, f
 // the fp16 output when the item covers the whole context, else the partition's
 // (max, sum, unnormalised output) for the merge.
 template <int D, typename ColumnRow>
-__device__ __forceinline__ void store_columns(const float* s_m, const float* s_l, const float* s_o,
-                                              const DecodeParams& p, int ncols, ColumnRow row_of,
-                                              int part, bool whole, int prefix_slots = 0) {
+__device__ __forceinline__ void store_columns(float* const (&bufs)[NW], const DecodeParams& p,
+                                              int ncols, ColumnRow row_of, int part, bool whole,
+                                              int prefix_slots = 0) {
+  // bufs[w]: consumer warp w's state (write_state), NULL when it had no chunk of the item.
   // row_of(c): the (sequence * num_heads + head) row of column c, or -1 to skip it.
   // prefix_slots > 0 (with whole): fold in that many finished shared-prefix partials first.
   // Each thread takes 4 consecutive dims of one column.
@@ -397,18 +400,21 @@ __device__ __forceinline__ void store_columns(const float* s_m, const float* s_l
     if (bh < 0) continue;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * 8 + col]);
+    for (int w = 0; w < NW; ++w)
+      if (bufs[w]) M = fmaxf(M, bufs[w][col]);
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
     float den = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      const float a = rescale_factor(s_m[w * 8 + col], M);
-      const float4 o = *reinterpret_cast<const float4*>(s_o + (w * 8 + col) * Geo::OSTRIDE + d0);
+      if (!bufs[w]) continue;
+      const float a = rescale_factor(bufs[w][col], M);
+      const float4 o =
+          *reinterpret_cast<const float4*>(bufs[w] + 16 + col * Geo::OSTRIDE + d0);
       num.x = fmaf(a, o.x, num.x);
       num.y = fmaf(a, o.y, num.y);
       num.z = fmaf(a, o.z, num.z);
       num.w = fmaf(a, o.w, num.w);
-      den = fmaf(a, s_l[w * 8 + col], den);
+      den = fmaf(a, bufs[w][8 + col], den);
     }
     if (prefix_slots > 0) {
       const size_t base = (size_t)bh * p.num_parts;
@@ -448,12 +454,19 @@ __device__ __forceinline__ void store_columns(const float* s_m, const float* s_l
 // Merges the consumer warps' states of one item (columns = the G query heads
 // of kv head kvh of sequence b) into out, or into partial slot `part`.
 template <int D>
-__device__ __forceinline__ void store_item(const float* s_m, const float* s_l, const float* s_o,
-                                           const DecodeParams& p, int b, int kvh, int part, int G,
-                                           bool whole, int prefix_slots = 0) {
+__device__ __forceinline__ void store_item(float* const (&bufs)[NW], const DecodeParams& p, int b,
+                                           int kvh, int part, int G, bool whole,
+                                           int prefix_slots = 0) {
   const long long row0 = (long long)b * p.num_heads + (long long)kvh * G;
-  store_columns<D>(s_m, s_l, s_o, p, G, [&](int c) { return row0 + c; }, part, whole,
-                   prefix_slots);
+  store_columns<D>(bufs, p, G, [&](int c) { return row0 + c; }, part, whole, prefix_slots);
+}
+
+// The drained ring as merge buffers, one per consumer warp (the one-CTA-per-item kernels).
+template <int D>
+__device__ __forceinline__ void ring_state_buffers(float* (&bufs)[NW], unsigned char* smem) {
+#pragma unroll
+  for (int w = 0; w < NW; ++w)
+    bufs[w] = reinterpret_cast<float*>(smem) + w * StageGeom<D>::STATE_FLOATS;
 }
 
 // ---- one CTA per (sequence, kv head, partition) ---------------------------------
@@ -472,9 +485,8 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_ids + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * stages);
   // merge buffers, placed over the ring once every stage has been consumed
-  float* s_m = reinterpret_cast<float*>(smem);  // [NW][8]
-  float* s_l = s_m + NW * 8;                    // [NW][8]
-  float* s_o = s_l + NW * 8;                    // [NW][8][OSTRIDE]
+  float* bufs[NW];
+  ring_state_buffers<D>(bufs, smem);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -508,7 +520,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   if (ntok <= 0) return;
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
   const int nblk = (ntok + BS - 1) / BS;
-  const int np = (P + p.part_tokens - 1) / p.part_tokens;  // prefix slots
+  const int np = (P + p.prefix_part_tokens - 1) / p.prefix_part_tokens;  // prefix slots
   const int slot_part = np + part;
   // covering a shared prefix's whole suffix: fold in the finished prefix partials here
   const bool merge_prefix = SPLIT && P > 0 && L - P <= p.part_tokens;
@@ -575,10 +587,10 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   if (named_barrier_or(1, NW * 32, gave_up)) return;
   // the merge kernel (if any) may be scheduled once every CTA got here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  write_state<D>(a, s_m, s_l, s_o, warp, lane);
+  write_state<D>(a, bufs[warp], lane);
   named_barrier_sync(1, NW * 32);
   if (p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");  // prefix partials ready
-  store_item<D>(s_m, s_l, s_o, p, b, kvh, slot_part, G,
+  store_item<D>(bufs, p, b, kvh, slot_part, G,
                 !SPLIT || (P == 0 && L <= p.part_tokens) || merge_prefix, merge_prefix ? np : 0);
 }
 
@@ -612,9 +624,8 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   int* s_ids = reinterpret_cast<int*>(smem + (size_t)stages * 2 * Geo::TILE_BYTES);  // [32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_ids + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * stages);
-  float* s_m = reinterpret_cast<float*>(smem);  // merge buffers over the drained ring
-  float* s_l = s_m + NW * 8;
-  float* s_o = s_l + NW * 8;
+  float* bufs[NW];  // merge buffers over the drained ring
+  ring_state_buffers<D>(bufs, smem);
 
   // the suffix pass may start on the SMs this grid frees; it waits for this grid
   // before it reads the partial results
@@ -633,11 +644,12 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     return;
   }
   const int P = pblocks * BS;
-  const int tok0 = part * p.part_tokens;
-  if (part == gridDim.z - 1 && tok0 + p.part_tokens < P && threadIdx.x == 0 && kvh == 0)
+  const int ppt = p.prefix_part_tokens;
+  const int tok0 = part * ppt;
+  if (part == gridDim.z - 1 && tok0 + ppt < P && threadIdx.x == 0 && kvh == 0)
     flag_error(p.err, ERR_PREFIX);  // the grid was sized below this prefix
   if (tok0 >= P) return;
-  const int ntok = min(P, tok0 + p.part_tokens) - tok0;
+  const int ntok = min(P, tok0 + ppt) - tok0;
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
   const int nblk = (ntok + BS - 1) / BS;
   const int blk0 = tok0 / BS;
@@ -733,10 +745,10 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     if (lane == 0) mbar_arrive(smem_u32(&bars[stages + st]));
   }
   if (named_barrier_or(1, NW * 32, gave_up)) return;
-  write_state<D>(a, s_m, s_l, s_o, warp, lane);
+  write_state<D>(a, bufs[warp], lane);
   named_barrier_sync(1, NW * 32);
   store_columns<D>(
-      s_m, s_l, s_o, p, max_members * G,
+      bufs, p, max_members * G,
       [&](int c) -> long long {
         const int m = s_member[c / G];
         return m < 0 ? -1 : (long long)m * p.num_heads + (long long)kvh * G + c % G;
@@ -782,7 +794,7 @@ __device__ __forceinline__ void release_counters(const PersistentArgs& pa, unsig
 // partial partition in that order.  Returns (b, kvh, part, tokens).
 __device__ __forceinline__ int4 item_of_ticket(int t, int num_kv_heads, int num_seqs,
                                                int part_tokens, const int* pref_f,
-                                               const int* by_tail, const int* lens) {
+                                               const uint16_t* by_tail, const int* lens) {
   const int kvh = t % num_kv_heads;
   int u = t / num_kv_heads;
   const int total_f = pref_f[num_seqs];
@@ -903,18 +915,17 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   unsigned char* cur = smem + (size_t)stages * 2 * Geo::TILE_BYTES;
   __half* s_q = reinterpret_cast<__half*>(cur);  // [IQ][8][D]
   cur += IQ * QTILE_BYTES;
-  float* s_m = reinterpret_cast<float*>(cur);    // [NW][8]
-  float* s_l = s_m + NW * 8;                     // [NW][8]
-  float* s_o = s_l + NW * 8;                     // [NW][8][OSTRIDE]
-  cur += Geo::MERGE_BYTES;
+  float* s_merge = reinterpret_cast<float*>(cur);  // [NW][STATE_FLOATS]: the per-item merge
+  cur += NW * Geo::STATE_FLOATS * sizeof(float);
   int4* s_item = reinterpret_cast<int4*>(cur);   // [IQ]
   cur += IQ * sizeof(int4);
   int* s_aux = reinterpret_cast<int*>(cur);      // PREFIX: [IQ][AUX] member mask, members
   if (PREFIX) cur += IQ * AUX * sizeof(int);
   int* s_lens = reinterpret_cast<int*>(cur);     // [B]
   int* pref_f = s_lens + B;                      // [B + 1]
-  int* by_tail = pref_f + B + 1;                 // [B]: sequences with a partial partition
-  int* tail_run = by_tail + B;                   // [TAIL_KEYS]: counts, then insert positions
+  // [B]: rows with a partial partition (16-bit: rows < PERSISTENT_MAX_SEQS)
+  uint16_t* by_tail = reinterpret_cast<uint16_t*>(pref_f + B + 1);
+  int* tail_run = pref_f + B + 1 + (B + 1) / 2;  // [TAIL_KEYS]: counts, then insert positions
   int* s_num_tail = tail_run + TAIL_KEYS;        // [1]: sequences with a partial partition
   int* s_ids = s_num_tail + 1;                   // [32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(
@@ -926,7 +937,8 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = p.num_heads / p.num_kv_heads;
-  const int pt = p.part_tokens;
+  // the partitions this kernel's items cover (a prefix pass: the prefix's own)
+  const int pt = PREFIX ? p.prefix_part_tokens : p.part_tokens;
 
   // per-sequence partition counts; the partial tails' chunk-count keys
   for (int k = threadIdx.x; k < TAIL_KEYS; k += blockDim.x) tail_run[k] = 0;
@@ -1011,7 +1023,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       const unsigned same = __match_any_sync(0xffffffffu, key);
       if (tail) {
         const int rank = __popc(same & ((1u << lane) - 1));
-        by_tail[tail_run[key] + rank] = b;
+        by_tail[tail_run[key] + rank] = (uint16_t)b;
       }
       __syncwarp();
       if (tail && (same & ((1u << lane) - 1)) == 0) tail_run[key] += __popc(same);
@@ -1055,28 +1067,12 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       const bool done = !have || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
       if (done) d = make_int4(0, 0, 0, 0);
       const int qs = it % IQ;
-      // the item's table row, chunks and (PREFIX) usable members
-      const int nblk = (d.w + BS - 1) / BS;
-      int nchunks = (d.w + CHUNK - 1) / CHUNK;
-      const int32_t* row = nullptr;
-      int new_tok = -1;
+      // (PREFIX) the item's usable members, checked before its slot is written
       unsigned mask = 0;
       int mem[GROUP_MAX_MEMBERS];
-      if (!done) {
-        if (PREFIX) {
-          const int blk0 = d.z * pt / BS;
-          mask = prefix_members<BS>(p, d.x, s_lens[d.x], blk0, nblk, 8 / G, mem,
-                                    d.y == 0 && d.z == 0, lane);
-          if (mask) row = p.block_tables + (size_t)mem[__ffs(mask) - 1] * p.max_blocks + blk0;
-          else nchunks = 0;  // no usable member: nothing to stream
-        } else {
-          const int P = prefix_of(d.x);
-          row = p.block_tables + (size_t)d.x * p.max_blocks + (P + d.z * pt) / BS;
-          const int Ls = s_lens[d.x];
-          new_tok = (p.k_new && d.z * pt + d.w == Ls && p.context_lens[d.x] == P + Ls) ? d.w - 1
-                                                                                     : -1;
-        }
-      }
+      if (PREFIX && !done)
+        mask = prefix_members<BS>(p, d.x, s_lens[d.x], d.z * pt / BS, (d.w + BS - 1) / BS, 8 / G,
+                                  mem, d.y == 0 && d.z == 0, lane);
       bool ok = true;
       if (lane == 0) {
         if (it >= IQ && !mbar_wait(smem_u32(&iempty[qs]), ((it / IQ) - 1) & 1)) {
@@ -1113,6 +1109,22 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       }
       ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
       if (done || !ok) break;
+      // the item's table row, chunks and (fused append) new token
+      const int nblk = (d.w + BS - 1) / BS;
+      int nchunks = (d.w + CHUNK - 1) / CHUNK;
+      const int32_t* row;
+      int new_tok = -1;
+      if (PREFIX) {
+        row = p.block_tables + (size_t)mem[mask ? __ffs(mask) - 1 : 0] * p.max_blocks +
+              d.z * pt / BS;
+        if (!mask) nchunks = 0;  // no usable member: nothing to stream
+      } else {
+        const int P = prefix_of(d.x);
+        row = p.block_tables + (size_t)d.x * p.max_blocks + (P + d.z * pt) / BS;
+        const int Ls = s_lens[d.x];
+        new_tok =
+            (p.k_new && d.z * pt + d.w == Ls && p.context_lens[d.x] == P + Ls) ? d.w - 1 : -1;
+      }
       if (nchunks > 0 &&
           !produce_item<D, BS>(row, nblk, nchunks, base, d.y, d.x, new_tok, p, s_ids, bars,
                                stages, ring, &k_map, &v_map, policy, abort_flag, lane, issued))
@@ -1130,6 +1142,8 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   }
 
   // ---------------- consumer warps ----------------
+  // (Keeping each warp's last stage of an item as its merge buffer, instead of a
+  // buffer of its own, fits 6 CTAs per SM instead of 5 but measured slower.)
   const int spw = stages / NW;
   int mine = 0;  // fills of this warp's sub-ring consumed so far
   for (int it = 0;; ++it) {
@@ -1187,27 +1201,30 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     }
     // All consumer warps decide together: the end of the work, or an abort anywhere.
     if (named_barrier_or(1, NW * 32, stop || gave_up)) break;
-    write_state<D>(a, s_m, s_l, s_o, warp, lane);
+    float* bufs[NW];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) bufs[w] = s_merge + w * Geo::STATE_FLOATS;
+    write_state<D>(a, s_merge + warp * Geo::STATE_FLOATS, lane);
     named_barrier_sync(1, NW * 32);
     if (PREFIX) {
       // each usable member's partial state goes to its prefix slot d.z
       const int kvh = d.y;
       store_columns<D>(
-          s_m, s_l, s_o, p, (8 / G) * G,
+          bufs, p, (8 / G) * G,
           [&](int c) -> long long {
             const int i = c / G;
             return ((mask >> i) & 1) ? (long long)mem[i] * p.num_heads + (long long)kvh * G + c % G
                                      : -1;
           },
           d.z, false);
-      continue;
+    } else {
+      // a whole suffix (one item) is finished here, a shared prefix's partials folded in
+      if (p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");  // prefix partials
+      const int P = prefix_of(d.x);
+      const int np = (P + p.prefix_part_tokens - 1) / p.prefix_part_tokens;
+      const bool whole = s_lens[d.x] <= pt;
+      store_item<D>(bufs, p, d.x, d.y, np + d.z, G, whole, whole ? np : 0);
     }
-    // a whole suffix (one item) is finished here, a shared prefix's partials folded in
-    if (p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");  // prefix partials ready
-    const int P = prefix_of(d.x);
-    const int np = (P + pt - 1) / pt;
-    const bool whole = s_lens[d.x] <= pt;
-    store_item<D>(s_m, s_l, s_o, p, d.x, d.y, np + d.z, G, whole, whole ? np : 0);
   }
   // the merge kernel may be scheduled once every CTA got here
   if (!PREFIX) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -1292,10 +1309,10 @@ size_t mma_smem_bytes(int head_dim, int block_size, int stages) {
 }
 
 size_t mma_persistent_smem_bytes(int head_dim, int stages, int num_rows, bool prefix) {
-  const size_t merge = (size_t)NW * 8 * (2 + head_dim + 4) * sizeof(float);
+  const size_t merge = (size_t)NW * (16 + 8 * (head_dim + 4)) * sizeof(float);
   return (size_t)stages * mma_stage_bytes(head_dim, 16) + IQ * 8ull * head_dim * 2 + merge +
          IQ * sizeof(int4) + (prefix ? IQ * (GROUP_MAX_MEMBERS + 1) * sizeof(int) : 0) +
-         (3ull * num_rows + 1 + TAIL_KEYS + 1 + 32) * sizeof(int) + 8 +
+         (2ull * num_rows + 1 + (num_rows + 1) / 2 + TAIL_KEYS + 1 + 32) * sizeof(int) + 8 +
          (2ull * stages + 2 * IQ) * sizeof(uint64_t) + 16;
 }
 

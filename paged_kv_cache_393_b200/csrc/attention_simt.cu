@@ -116,7 +116,7 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
     flag_error(p.err, ERR_PREFIX);                  // the grid was sized below this suffix
   const int ntok = min(L, tok0 + p.part_tokens) - tok0;
   if (ntok <= 0) return;                            // partition beyond this context
-  const int np = (P + p.part_tokens - 1) / p.part_tokens;  // prefix slots
+  const int np = (P + p.prefix_part_tokens - 1) / p.prefix_part_tokens;  // prefix slots
   const int slot_part = np + part;
   // A CTA that covers a shared prefix's whole suffix finishes the output itself:
   // the prefix pass ran to completion before this launch, so its partial

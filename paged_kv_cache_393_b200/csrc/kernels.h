@@ -26,6 +26,7 @@ struct DecodeParams {
   int num_seqs, num_heads, num_kv_heads, head_dim, block_size;
   int max_blocks, num_blocks, max_context_len;
   int part_tokens;             // tokens per partition (a multiple of 16 and of bs)
+  int prefix_part_tokens;      // tokens per partition of a shared prefix (its slots come first)
   int num_parts;               // partial-result slots per (sequence, head)
   int grid_parts;              // partitions in the launch grid (<= num_parts)
   int no_merge;                // no merge kernel follows: a partial result here is an error

@@ -31,7 +31,6 @@ constexpr int MERGE_GROUPS = 4;  // lane groups per warp, each over every 4th pa
 
 template <int D>
 __global__ void __launch_bounds__(MERGE_WARPS * 32) split_merge_kernel(const DecodeParams p) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the partition pass
   constexpr int V4 = D / 4;                           // float4 columns of one output row
   constexpr int GL = 32 / MERGE_GROUPS;               // lanes per group
   constexpr int CPL = V4 / GL;                        // float4 columns per lane
@@ -42,12 +41,15 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) split_merge_kernel(const Dec
   const long long row = (long long)blockIdx.x * MERGE_WARPS + (threadIdx.x >> 5);  // b * H + h
   if (row >= (long long)p.num_seqs * p.num_heads) return;
   const int b = (int)(row / p.num_heads);
+  // the lengths and prefix lengths are inputs no earlier kernel of the step writes: read
+  // them while the partition pass may still run, then wait for its partials
   int L = p.context_lens[b];
   if (L > p.max_context_len) L = p.max_context_len;  // flagged by the partition pass
   // partial slots: a shared prefix's partitions (if any), then the rest of the context's
   bool bad = false;
   const int pre = L <= 0 ? 0 : prefix_tokens_of(p.seq_prefix_tokens, b, L, p.block_size, &bad);
-  const int np = (pre + p.part_tokens - 1) / p.part_tokens;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the partition pass
+  const int np = (pre + p.prefix_part_tokens - 1) / p.prefix_part_tokens;
   const int ns = L <= 0 ? 0 : (L - pre + p.part_tokens - 1) / p.part_tokens;
   const int P = np + ns;
   if (ns == 1) return;  // one partition after any prefix: finished by the partition pass

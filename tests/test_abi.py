@@ -134,8 +134,8 @@ def test_shared_prefix_rejects_bad_arguments_on_the_host(lib, kw, code):
 
 
 def test_shared_prefix_workspace_bytes(lib):
-    # 32 bytes of work counters, then the partials: always split at 512 (or the given size),
-    # with one extra slot per (sequence, head)
+    # 32 bytes of work counters, then the partials: always split at 512 tokens (or the given
+    # size), with one extra slot per (sequence, head): a prefix can end inside a partition
     f = lib.paged_attention_shared_prefix_workspace_bytes
     assert f(4, 8, 8, 128, 16, 1200, 0) == 32 + 4 * 8 * (3 + 1) * 130 * 4
     assert f(4, 8, 8, 128, 16, 1200, -1) == 32 + 4 * 8 * (3 + 1) * 130 * 4
@@ -268,12 +268,13 @@ def test_host_step_staging_bytes(lib):
     r = lambda n: (n + 255) // 256 * 256  # noqa: E731
     B, H, Hk, D, bs, maxblk, maxlen = 256, 32, 32, 128, 16, 96, 1524
     ws = lib.paged_attention_workspace_bytes(B, H, Hk, D, bs, maxlen, 0)
+    # the plain step pipelines 4 chunks over two compute streams: two workspaces
     want = (r(B * H * D * 2) * 2 + r(B * Hk * D * 2) * 2 + r(B * maxblk * 4) + r(B * 4) +
-            r(224 * 16) + r(ws))
+            r(224 * 16) + 2 * r(ws))
     assert f(B, H, Hk, D, bs, maxblk, maxlen, 0, 224, 0) == want
     ws2 = lib.paged_attention_shared_prefix_workspace_bytes(B, H, Hk, D, bs, maxlen, 0)
     assert f(B, H, Hk, D, bs, maxblk, maxlen, 0, 224, 1) == \
-        want - r(ws) + r(B * 4) + r(B // 2 * 9 * 4) + r(ws2)
+        want - 2 * r(ws) + r(B * 4) + r(B // 2 * 9 * 4) + r(ws2)
     assert f(B, H, Hk, 96, bs, maxblk, maxlen, 0, 0, 0) == 0    # rejected head_dim
 
 

@@ -120,6 +120,10 @@ constexpr size_t MAX_SMEM = 227 * 1024;
 #ifndef PAGEDKV_TUNE_PERSISTENT
 #define PAGEDKV_TUNE_PERSISTENT 1
 #endif
+#ifndef PAGEDKV_TUNE_MHA_SUFFIX_MMA
+#define PAGEDKV_TUNE_MHA_SUFFIX_MMA 0       // 1: a shared-prefix call's MHA suffix pass on the
+                                            // persistent tensor-core kernel, not folding
+#endif
 #ifndef PAGEDKV_TUNE_PREFIX_HALF
 #define PAGEDKV_TUNE_PREFIX_HALF 0          // 1: shared prefixes in half-size partitions
 #endif
@@ -136,6 +140,7 @@ struct Plan {
   size_t smem = 0;
   size_t ws_bytes = 0;
   bool cascade = false;      // shared-prefix decode: prefix pass + suffix pass + merge
+  bool fold_prefix = true;   // the suffix pass folds the prefix partials (single-partition suffixes)
   int prefix_stages = 0;     // ring depth of the prefix pass
 };
 
@@ -169,7 +174,8 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
   // tensor cores for query groups (running the suffix pass of a shared-prefix call for one kv
   // head per query head on them too was measured slower: every suffix item folds the prefix
   // partials, so the persistent suffix CTAs wait for the whole prefix pass)
-  p.mma = G >= 2 && G <= 8 && block_size >= 8;
+  p.mma = (G >= 2 || (cascade && PAGEDKV_TUNE_MHA_SUFFIX_MMA)) && G <= 8 && block_size >= 8;
+  p.fold_prefix = !(cascade && G == 1 && PAGEDKV_TUNE_MHA_SUFFIX_MMA);
   if (!p.mma) {
     if (G == 1) {
       // widest contiguous kv-head group whose stage stays within 16 KB
@@ -444,7 +450,9 @@ int decode(void* out, const void* q, const void* k_new, const void* v_new, const
   }
   // With a shared prefix and every suffix within one partition, the partition
   // pass finishes every output itself: no merge.
-  const bool merged = cascade && max_suffix_tokens > 0 && max_suffix_tokens <= plan.part_tokens;
+  const bool merged = cascade && plan.fold_prefix && max_suffix_tokens > 0 &&
+                      max_suffix_tokens <= plan.part_tokens;
+  p.fold_prefix = plan.fold_prefix ? 1 : 0;
   p.no_merge = merged ? 1 : 0;
   p.stages = plan.stages;
   p.k_new = static_cast<const __half*>(k_new);
@@ -639,8 +647,14 @@ struct StepLayout {
 // two compute streams (each with its own workspace) so that one chunk's last
 // CTAs and merge overlap the next chunk's start.  The shared-prefix step runs
 // whole (its groups span the batch).
-constexpr int STEP_MAX_CHUNKS = 4;
-constexpr int STEP_CHUNK_SEQS = 64;
+#ifndef PAGEDKV_TUNE_STEP_CHUNKS
+#define PAGEDKV_TUNE_STEP_CHUNKS 4
+#endif
+#ifndef PAGEDKV_TUNE_STEP_CHUNK_SEQS
+#define PAGEDKV_TUNE_STEP_CHUNK_SEQS 64
+#endif
+constexpr int STEP_MAX_CHUNKS = PAGEDKV_TUNE_STEP_CHUNKS;
+constexpr int STEP_CHUNK_SEQS = PAGEDKV_TUNE_STEP_CHUNK_SEQS;
 
 int step_chunks(int num_seqs, bool shared_prefix) {
   if (shared_prefix) return 1;

@@ -523,7 +523,7 @@ __global__ void __launch_bounds__((NW + 1) * 32)
   const int np = (P + p.prefix_part_tokens - 1) / p.prefix_part_tokens;  // prefix slots
   const int slot_part = np + part;
   // covering a shared prefix's whole suffix: fold in the finished prefix partials here
-  const bool merge_prefix = SPLIT && P > 0 && L - P <= p.part_tokens;
+  const bool merge_prefix = SPLIT && P > 0 && L - P <= p.part_tokens && p.fold_prefix;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -1219,10 +1219,11 @@ __global__ void __launch_bounds__((NW + 1) * 32)
           d.z, false);
     } else {
       // a whole suffix (one item) is finished here, a shared prefix's partials folded in
-      if (p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");  // prefix partials
+      // (only that waits for the prefix pass)
       const int P = prefix_of(d.x);
       const int np = (P + p.prefix_part_tokens - 1) / p.prefix_part_tokens;
-      const bool whole = s_lens[d.x] <= pt;
+      const bool whole = s_lens[d.x] <= pt && (P == 0 || p.fold_prefix);
+      if (whole && P > 0 && p.after_prefix) asm volatile("griddepcontrol.wait;" ::: "memory");
       store_item<D>(bufs, p, d.x, d.y, np + d.z, G, whole, whole ? np : 0);
     }
   }

@@ -121,7 +121,7 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
   // A CTA that covers a shared prefix's whole suffix finishes the output itself:
   // the prefix pass ran to completion before this launch, so its partial
   // results can be folded in here and no merge is needed.
-  const bool merge_prefix = SPLIT && P > 0 && L - P <= p.part_tokens;
+  const bool merge_prefix = SPLIT && P > 0 && L - P <= p.part_tokens && p.fold_prefix;
   const bool direct = !SPLIT || (P == 0 && L <= p.part_tokens) || merge_prefix;
   const int nchunks = (ntok + CHUNK - 1) / CHUNK;
   const int blk0 = tok0 / BS;

@@ -32,6 +32,8 @@ struct DecodeParams {
   int no_merge;                // no merge kernel follows: a partial result here is an error
   int after_prefix;            // launched as a programmatic dependent of the shared-prefix pass:
                                // wait for it (griddepcontrol.wait) before reading its partials
+  int fold_prefix;             // a suffix within one partition folds the prefix partials into
+                               // the output itself; 0: it leaves a partial, the merge combines
   int stages;                  // depth of the shared-memory ring
   // Fused append (NULL = none): this step's new K/V rows, [B][Hk][D], which the
   // kernel writes to position L_b - 1 through the block table before reading it.

@@ -52,7 +52,8 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) split_merge_kernel(const Dec
   const int np = (pre + p.prefix_part_tokens - 1) / p.prefix_part_tokens;
   const int ns = L <= 0 ? 0 : (L - pre + p.part_tokens - 1) / p.part_tokens;
   const int P = np + ns;
-  if (ns == 1) return;  // one partition after any prefix: finished by the partition pass
+  // one partition after any prefix: finished by the partition pass (prefix partials folded)
+  if (ns == 1 && (np == 0 || p.fold_prefix)) return;
   __half* out = p.out + row * D;
   if (P == 0) {
     if (lane < V4) *reinterpret_cast<uint2*>(out + lane * 4) = make_uint2(0u, 0u);

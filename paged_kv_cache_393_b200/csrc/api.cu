@@ -662,10 +662,22 @@ int step_chunks(int num_seqs, bool shared_prefix) {
   return c < 1 ? 1 : (c > STEP_MAX_CHUNKS ? STEP_MAX_CHUNKS : c);
 }
 
-// Sequences [first, first + count) of chunk i of n.
+#ifndef PAGEDKV_TUNE_STEP_HALF_ENDS
+#define PAGEDKV_TUNE_STEP_HALF_ENDS 0   // 1: first and last chunks half-size
+#endif
+
+// Sequences [first, first + count) of chunk i of n.  With half-size end chunks the
+// first chunk's upload and the last chunk's download, which nothing overlaps, shrink.
 void chunk_range(int num_seqs, int n, int i, int* first, int* count) {
-  *first = (int)((long long)num_seqs * i / n);
-  *count = (int)((long long)num_seqs * (i + 1) / n) - *first;
+  auto edge = [&](int k) -> int {  // first sequence of chunk k
+    if (!PAGEDKV_TUNE_STEP_HALF_ENDS || n < 3) return (int)((long long)num_seqs * k / n);
+    // weights 1, 2, ..., 2, 1 (in halves): chunk k starts at (2k - 1) / (2n - 2) of the batch
+    if (k == 0) return 0;
+    if (k == n) return num_seqs;
+    return (int)((long long)num_seqs * (2 * k - 1) / (2 * n - 2));
+  };
+  *first = edge(i);
+  *count = edge(i + 1) - *first;
 }
 
 int step_layout(StepLayout* lay, int num_seqs, int num_heads, int num_kv_heads, int head_dim,

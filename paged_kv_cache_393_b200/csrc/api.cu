@@ -653,6 +653,9 @@ struct StepLayout {
 #ifndef PAGEDKV_TUNE_STEP_CHUNK_SEQS
 #define PAGEDKV_TUNE_STEP_CHUNK_SEQS 64
 #endif
+#ifndef PAGEDKV_TUNE_STEP_END_QUARTERS
+#define PAGEDKV_TUNE_STEP_END_QUARTERS 2  // half-size end chunks (measured faster than equal)
+#endif
 constexpr int STEP_MAX_CHUNKS = PAGEDKV_TUNE_STEP_CHUNKS;
 constexpr int STEP_CHUNK_SEQS = PAGEDKV_TUNE_STEP_CHUNK_SEQS;
 
@@ -662,19 +665,16 @@ int step_chunks(int num_seqs, bool shared_prefix) {
   return c < 1 ? 1 : (c > STEP_MAX_CHUNKS ? STEP_MAX_CHUNKS : c);
 }
 
-#ifndef PAGEDKV_TUNE_STEP_HALF_ENDS
-#define PAGEDKV_TUNE_STEP_HALF_ENDS 1   // first and last chunks half-size (measured faster)
-#endif
-
-// Sequences [first, first + count) of chunk i of n.  With half-size end chunks the
-// first chunk's upload and the last chunk's download, which nothing overlaps, shrink.
+// Sequences [first, first + count) of chunk i of n.  The first and last chunks weigh
+// E = PAGEDKV_TUNE_STEP_END_QUARTERS quarters of a middle chunk: smaller end chunks
+// shrink the first upload and the last download, which nothing overlaps.
 void chunk_range(int num_seqs, int n, int i, int* first, int* count) {
+  const long long E = PAGEDKV_TUNE_STEP_END_QUARTERS;
+  const long long total = n < 2 ? 1 : 2 * E + 4LL * (n - 2);
   auto edge = [&](int k) -> int {  // first sequence of chunk k
-    if (!PAGEDKV_TUNE_STEP_HALF_ENDS || n < 3) return (int)((long long)num_seqs * k / n);
-    // weights 1, 2, ..., 2, 1 (in halves): chunk k starts at (2k - 1) / (2n - 2) of the batch
-    if (k == 0) return 0;
-    if (k == n) return num_seqs;
-    return (int)((long long)num_seqs * (2 * k - 1) / (2 * n - 2));
+    if (k <= 0) return 0;
+    if (k >= n) return num_seqs;
+    return (int)((long long)num_seqs * (E + 4LL * (k - 1)) / total);
   };
   *first = edge(i);
   *count = edge(i + 1) - *first;
@@ -753,7 +753,7 @@ int h2d(void* dst, const void* src, size_t bytes, cudaStream_t s, const char* wh
 // created at the first chunked call and kept until the process exits.
 struct StepAux {
   cudaStream_t up, down, comp;  // uploads, downloads, the second compute stream
-  cudaEvent_t start, small, copied, done, in[STEP_MAX_CHUNKS], out[STEP_MAX_CHUNKS];
+  cudaEvent_t start, copied, done, in[STEP_MAX_CHUNKS], out[STEP_MAX_CHUNKS];
   bool ready;
 };
 thread_local StepAux tl_step_aux[MAX_DEVICES];
@@ -769,10 +769,10 @@ int step_aux(StepAux** out) {
         (e = cudaStreamCreateWithFlags(&a.down, cudaStreamNonBlocking)) != cudaSuccess ||
         (e = cudaStreamCreateWithFlags(&a.comp, cudaStreamNonBlocking)) != cudaSuccess)
       return cuda_fail(e, "creating the step's streams");
-    cudaEvent_t* evs[4 + 2 * STEP_MAX_CHUNKS] = {&a.start, &a.small, &a.copied, &a.done};
+    cudaEvent_t* evs[3 + 2 * STEP_MAX_CHUNKS] = {&a.start, &a.copied, &a.done};
     for (int i = 0; i < STEP_MAX_CHUNKS; ++i) {
-      evs[4 + i] = &a.in[i];
-      evs[4 + STEP_MAX_CHUNKS + i] = &a.out[i];
+      evs[3 + i] = &a.in[i];
+      evs[3 + STEP_MAX_CHUNKS + i] = &a.out[i];
     }
     for (cudaEvent_t* ev : evs)
       if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
@@ -882,40 +882,47 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
                D = (size_t)head_dim;
   const int nch = step_chunks(num_seqs, shared);
   if (nch > 1) {
-    // Pipelined: the uploads run on a copy stream, chunk by chunk, and each chunk's
-    // attention starts as soon as its inputs have landed; each chunk's output is
-    // downloaded on a second copy stream while the next chunk computes.  The
-    // caller's stream waits for the last download, so work it enqueues later (the
-    // next step overwriting this staging) comes after all of it.
+    // Pipelined: the uploads run chunk by chunk, and each chunk's attention starts as
+    // soon as its inputs have landed; each chunk's output is downloaded on a copy
+    // stream while the next chunk computes.  The caller's stream waits for the last
+    // download, so work it enqueues later (the next step overwriting this staging)
+    // comes after all of it.
     StepAux* aux = nullptr;
     if ((st = step_aux(&aux)) != PAGEDKV_OK) return st;
     const size_t row_q = H * D * 2, row_kv = Hk * D * 2, row_t = (size_t)max_blocks_per_seq * 4;
+    // uploads of chunk c: its table rows, lengths, q and new K/V rows
+    auto upload = [&](int c, cudaStream_t us) -> int {
+      int first = 0, count = 0, r = PAGEDKV_OK;
+      chunk_range(num_seqs, nch, c, &first, &count);
+      if ((r = h2d(base + lay.tables + first * row_t,
+                   reinterpret_cast<const char*>(block_tables_host) + first * row_t,
+                   count * row_t, us, "block table upload")) != PAGEDKV_OK ||
+          (r = h2d(base + lay.lens + first * 4, context_lens_host + first, count * 4, us,
+                   "context length upload")) != PAGEDKV_OK ||
+          (r = h2d(base + lay.q + first * row_q, static_cast<const char*>(q_host) + first * row_q,
+                   count * row_q, us, "query upload")) != PAGEDKV_OK ||
+          (r = h2d(base + lay.k + first * row_kv,
+                   static_cast<const char*>(k_new_host) + first * row_kv, count * row_kv, us,
+                   "new K upload")) != PAGEDKV_OK ||
+          (r = h2d(base + lay.v + first * row_kv,
+                   static_cast<const char*>(v_new_host) + first * row_kv, count * row_kv, us,
+                   "new V upload")) != PAGEDKV_OK)
+        return r;
+      return PAGEDKV_OK;
+    };
+    // The pairs and the first chunk's inputs go up on the caller's stream, ahead of its
+    // kernels with no cross-stream wait (and after the previous step on it, which read
+    // this staging); the copy stream takes the other chunks once they have landed.
+    if ((st = h2d(base + lay.pairs, copy_pairs_host, (size_t)num_pairs * 16, s,
+                  "pair upload")) != PAGEDKV_OK ||
+        (st = upload(0, s)) != PAGEDKV_OK)
+      return st;
     PKV_CHECK_CUDA(cudaEventRecord(aux->start, s), "step start");
     PKV_CHECK_CUDA(cudaStreamWaitEvent(aux->up, aux->start, 0), "upload wait");
-    if ((st = h2d(base + lay.tables, block_tables_host, B * row_t, aux->up,
-                  "block table upload")) != PAGEDKV_OK ||
-        (st = h2d(base + lay.lens, context_lens_host, B * 4, aux->up, "context length upload")) !=
-            PAGEDKV_OK ||
-        (st = h2d(base + lay.pairs, copy_pairs_host, (size_t)num_pairs * 16, aux->up,
-                  "pair upload")) != PAGEDKV_OK)
-      return st;
-    PKV_CHECK_CUDA(cudaEventRecord(aux->small, aux->up), "upload event");
-    for (int c = 0; c < nch; ++c) {
-      int first = 0, count = 0;
-      chunk_range(num_seqs, nch, c, &first, &count);
-      const char* qh = static_cast<const char*>(q_host) + first * row_q;
-      const char* kh = static_cast<const char*>(k_new_host) + first * row_kv;
-      const char* vh = static_cast<const char*>(v_new_host) + first * row_kv;
-      if ((st = h2d(base + lay.q + first * row_q, qh, count * row_q, aux->up, "query upload")) !=
-              PAGEDKV_OK ||
-          (st = h2d(base + lay.k + first * row_kv, kh, count * row_kv, aux->up,
-                    "new K upload")) != PAGEDKV_OK ||
-          (st = h2d(base + lay.v + first * row_kv, vh, count * row_kv, aux->up,
-                    "new V upload")) != PAGEDKV_OK)
-        return st;
+    for (int c = 1; c < nch; ++c) {
+      if ((st = upload(c, aux->up)) != PAGEDKV_OK) return st;
       PKV_CHECK_CUDA(cudaEventRecord(aux->in[c], aux->up), "upload event");
     }
-    PKV_CHECK_CUDA(cudaStreamWaitEvent(s, aux->small, 0), "compute wait");
     if (num_pairs > 0) {
       void* kc[1] = {key_cache};
       void* vc[1] = {value_cache};
@@ -932,7 +939,7 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
       // even chunks on the caller's stream, odd ones on the second, each with its workspace
       cudaStream_t cs = (c & 1) ? aux->comp : s;
       void* ws = lay.ws_bytes ? base + ((c & 1) ? lay.ws2 : lay.ws) : nullptr;
-      PKV_CHECK_CUDA(cudaStreamWaitEvent(cs, aux->in[c], 0), "compute wait");
+      if (c > 0) PKV_CHECK_CUDA(cudaStreamWaitEvent(cs, aux->in[c], 0), "compute wait");
       st = paged_attention_decode_append(
           base + lay.out + first * row_q, base + lay.q + first * row_q,
           base + lay.k + first * row_kv, base + lay.v + first * row_kv, key_cache, value_cache,

@@ -219,6 +219,20 @@ def test_more_sequences_than_the_persistent_grid(pkv):
     _run(pkv, fb, True, 32, sample=[0, 1, 2, 3, 517, 1039])
 
 
+@pytest.mark.parametrize("part", [0, 64])
+def test_many_short_suffixes(pkv, part):
+    # 320 sequences x 16 head pairs: several waves of suffix CTAs, every suffix within one
+    # partition (folded in place, no merge), over 40 groups whose prefixes end at assorted
+    # block counts.  The 9-token prompts share no whole block, so their samples have no
+    # prefix and sit among the grouped ones.
+    prompts = [9 + 53 * (i % 13) for i in range(40)]
+    fb = ForkBatch(pkv, 32, 32, 128, 16, prompts, 8, lambda i: (11 * i) % 41)
+    assert len(fb.seqs) == 320
+    pre, _ = fb.groups()
+    assert (pre == 0).sum() >= 8 and (pre > 0).sum() >= 200
+    _run(pkv, fb, True, part)
+
+
 def test_inconsistent_groups_are_flagged_not_faulted(pkv):
     fb = ForkBatch(pkv, 8, 8, 128, 16, [300, 200], 4, lambda i: i)
     pre, groups = fb.groups()

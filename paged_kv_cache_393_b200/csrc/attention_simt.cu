@@ -92,7 +92,9 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
   const int kv0 = h0 / G;
   const bool reporter = threadIdx.x == 0 && blockIdx.x == 0 && part == 0;
 
+  // the length and the shared-prefix entry are loaded together (one round trip)
   int L = p.context_lens[b];
+  const int P_entry = p.seq_prefix_tokens ? p.seq_prefix_tokens[b] : 0;
   if (L > p.max_context_len) {
     if (reporter) flag_error(p.err, ERR_CONTEXT_LEN);
     L = p.max_context_len;
@@ -109,7 +111,7 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
   // the suffix [P, L): its partitions start at P, and their partial results go
   // after the prefix partitions' slots.
   bool bad_prefix = false;
-  const int P = prefix_tokens_of(p.seq_prefix_tokens, b, L, BS, &bad_prefix);
+  const int P = prefix_tokens_checked(P_entry, L, BS, &bad_prefix);
   if (bad_prefix && reporter) flag_error(p.err, ERR_PREFIX);
   const int tok0 = P + part * p.part_tokens;        // first token of this partition
   if (SPLIT && part == gridDim.z - 1 && tok0 + p.part_tokens < L && threadIdx.x == 0)
@@ -326,26 +328,28 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
     const size_t bh = (size_t)b * p.num_heads + h;
     if (direct) {
       if (merge_prefix) {
+        // the prefix partials folded in online, one partition at a time: each
+        // partition's loads are independent of the others', so they are in flight
+        // together instead of a round of maxima before a round of outputs
         const float* ml = p.ws_ml + bh * p.num_parts * 2;
-        float M = m;
-        for (int i = 0; i < np; ++i) M = fmaxf(M, ml[2 * i]);
-        const float a = rescale_factor(m, M);
-        l *= a;
-#pragma unroll
-        for (int d = 0; d < 8; ++d) acc[d] *= a;
+#pragma unroll 4
         for (int i = 0; i < np; ++i) {
-          const float w = rescale_factor(ml[2 * i], M);
-          const float4* o = reinterpret_cast<const float4*>(p.ws_o + (bh * p.num_parts + i) * D + col);
+          const float mi = ml[2 * i], li = ml[2 * i + 1];
+          const float4* o =
+              reinterpret_cast<const float4*>(p.ws_o + (bh * p.num_parts + i) * D + col);
           const float4 o0 = o[0], o1 = o[1];
-          l = fmaf(w, ml[2 * i + 1], l);
-          acc[0] = fmaf(w, o0.x, acc[0]);
-          acc[1] = fmaf(w, o0.y, acc[1]);
-          acc[2] = fmaf(w, o0.z, acc[2]);
-          acc[3] = fmaf(w, o0.w, acc[3]);
-          acc[4] = fmaf(w, o1.x, acc[4]);
-          acc[5] = fmaf(w, o1.y, acc[5]);
-          acc[6] = fmaf(w, o1.z, acc[6]);
-          acc[7] = fmaf(w, o1.w, acc[7]);
+          const float M = fmaxf(m, mi);
+          const float a = rescale_factor(m, M), w = rescale_factor(mi, M);
+          l = fmaf(w, li, l * a);
+          acc[0] = fmaf(w, o0.x, acc[0] * a);
+          acc[1] = fmaf(w, o0.y, acc[1] * a);
+          acc[2] = fmaf(w, o0.z, acc[2] * a);
+          acc[3] = fmaf(w, o0.w, acc[3] * a);
+          acc[4] = fmaf(w, o1.x, acc[4] * a);
+          acc[5] = fmaf(w, o1.y, acc[5] * a);
+          acc[6] = fmaf(w, o1.z, acc[6] * a);
+          acc[7] = fmaf(w, o1.w, acc[7] * a);
+          m = M;
         }
       }
       uint4 packed;

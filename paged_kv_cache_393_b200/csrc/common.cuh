@@ -32,16 +32,22 @@ __device__ __forceinline__ void flag_error(unsigned* err, unsigned bit) {
 // Tokens of a sequence that its shared-prefix group covers (0 = none): a whole
 // number of blocks that leaves at least the last token to the sequence itself.
 // Any other value is reported through *bad and treated as 0 by every kernel.
-__device__ __forceinline__ int prefix_tokens_of(const int32_t* seq_prefix_tokens, int b, int L,
-                                                int bs, bool* bad) {
-  if (!seq_prefix_tokens) return 0;
-  const int P = seq_prefix_tokens[b];
+// The shared-prefix tokens of a sequence of length L, given its entry P of
+// seq_prefix_tokens: 0 when it has none or when P is not a whole number of blocks
+// below L (then *bad is set).
+__device__ __forceinline__ int prefix_tokens_checked(int P, int L, int bs, bool* bad) {
   if (P == 0) return 0;
   if (P < 0 || P % bs != 0 || P > L - 1) {
     *bad = true;
     return 0;
   }
   return P;
+}
+
+__device__ __forceinline__ int prefix_tokens_of(const int32_t* seq_prefix_tokens, int b, int L,
+                                                int bs, bool* bad) {
+  if (!seq_prefix_tokens) return 0;
+  return prefix_tokens_checked(seq_prefix_tokens[b], L, bs, bad);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

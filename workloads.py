@@ -18,7 +18,9 @@ Workloads (shapes of the pages' Llama-2-7B / 70B-like decode batches):
                 sequences), then 200 decode steps; 32 = 32 heads, head_dim 128,
                 block_size 16, pool of 32768 blocks.
 * ``llama7b_small`` / ``gqa_small``  32- and 16-sequence cuts of those batches
-                (pools of about 1 GB) for profiler captures.
+                (pools of about 1 GB) for profiler captures; ``cow_small`` an
+                8-prompt cut of ``cow``, ``cow_compact`` the whole ``cow`` batch in
+                a 6144-block pool.
 * ``gqa``       128 sequences, 64 query heads over 8 kv heads, head_dim 128,
                 block_size 16, context lengths round(LogNormal(ln 1024, 1))
                 clipped to [64, 16384], split into 512-token partitions,
@@ -91,6 +93,10 @@ WORKLOADS = {
     # an 8-prompt cut of cow (64 samples) for profiler captures of the shared-prefix pass
     "cow_small": Workload("cow_small", 64, 32, 32, 128, 16, 8192, 1004, "cow",
                           prompts=8, prompt_len=1000, samples=8, decode_steps=200),
+    # the whole cow batch in a pool of 6144 blocks (1.6 GB; 200 steps need 5312): the
+    # prefix pass's full item count, for multi-pass profiler captures
+    "cow_compact": Workload("cow_compact", 256, 32, 32, 128, 16, 6144, 1004, "cow",
+                            prompts=32, prompt_len=1000, samples=8, decode_steps=200),
     "gqa": Workload("gqa", 128, 64, 8, 128, 16, 131072, 1005, "lognormal",
                     lognormal_median=1024.0, lognormal_sigma=1.0, len_lo=64, len_hi=16384,
                     partition_size=512),

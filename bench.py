@@ -307,7 +307,10 @@ def time_decode(gb, part, step_kind, K, warmup, dev, stream, world, local):
     if flags:
         raise SystemExit("device error flags %#x during the timed steps (%s)" % (flags, w.name))
 
-    attn_ms = sum(a.elapsed_time(b) for a, b in ev_a) / K
+    per_launch = sorted(a.elapsed_time(b) for a, b in ev_a)
+    attn_ms = sum(per_launch) / K
+    attn_median_ms = per_launch[K // 2] if K % 2 else 0.5 * (per_launch[K // 2 - 1] +
+                                                             per_launch[K // 2])
     kv_bytes = gb.kv_bytes()
     # the attention call's algorithmic bytes per launch: K+V rows read, q read, out
     # written, table entries and lengths read, new rows, split partials written and read
@@ -321,7 +324,8 @@ def time_decode(gb, part, step_kind, K, warmup, dev, stream, world, local):
     if pt > 0:
         parts = (gb.lens_host + pt - 1) // pt
         partial_bytes = int(parts[parts > 1].sum()) * H * (D + 2) * 4 * 2
-    return {"ms_total": t0.elapsed_time(t1), "K": K, "attn_ms": attn_ms, "kv_bytes": kv_bytes,
+    return {"ms_total": t0.elapsed_time(t1), "K": K, "attn_ms": attn_ms,
+            "attn_median_ms": attn_median_ms, "kv_bytes": kv_bytes,
             "attn_bytes": attn_bytes, "partial_bytes": partial_bytes,
             "launches": K * launches_per_step, "clocks": clocks, "kernel_file": kernel_file,
             "partition_tokens": pt}
@@ -335,7 +339,8 @@ def roofline_of(res, workload):
             "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
             "traffic": recorded_traffic(res["kernel_file"], workload),
             "algorithmic_bytes": res["attn_bytes"], "split_partial_bytes": res["partial_bytes"],
-            "avg_launch_ms": round(res["attn_ms"], 5)}
+            "avg_launch_ms": round(res["attn_ms"], 5),
+            "median_launch_ms": round(res["attn_median_ms"], 5)}
 
 
 def sub_entry(w, res, step_kind):

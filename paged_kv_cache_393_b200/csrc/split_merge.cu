@@ -9,13 +9,13 @@
 // slots of a (sequence, head) are its prefix partitions, then the partitions
 // of the rest of its context.
 //
-// One warp per (sequence, head), four per CTA.  The lanes stride over the
-// partitions for the maximum (warp shuffles), and each lane turns its own
-// partitions' maxima into weights; then the warp splits into four groups of
-// eight lanes, group g taking partitions g, g+4, g+8, ... with their weights
-// broadcast by shuffle and each lane D/32 float4 columns of them, so a long
+// One warp per (sequence, head), four per CTA.  The warp splits into four
+// groups of eight lanes; group g folds partitions g, g+4, g+8, ... online
+// (running maximum, rescaled sum and columns), each lane D/32 float4 columns of
+// them, and a partition's (max, sum) and columns are loaded together, so a long
 // context (tens of partitions) is a short chain of independent loads with many
-// in flight; two shuffles add the groups up.
+// in flight.  Shuffles bring the four groups to the overall maximum and add
+// them up.
 // No shared memory and no CTA barrier, and the grid fits the GPU in about one
 // wave.  The kernel is launched as a programmatic dependent of the partition
 // pass: its CTAs can be resident before that pass ends and wait
@@ -60,47 +60,50 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) split_merge_kernel(const Dec
     return;
   }
   const float* ml = p.ws_ml + row * p.num_parts * 2;
-  // lane i owns partitions i, i + 32, ...: their (max, sum) come in one round of loads
-  float M = -INFINITY;
-  for (int i = lane; i < P; i += 32) M = fmaxf(M, ml[2 * i]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const float4* src = reinterpret_cast<const float4*>(p.ws_o + row * p.num_parts * D);
-  float den = 0.f;  // this lane's partitions' share of the denominator
+  // Group g folds partitions g, g + 4, g + 8, ... online: each partition's (max, sum)
+  // and output columns are loaded together, so a context's partials are one round of
+  // independent loads.  Then the four groups are combined by shuffles.
+  float M = -INFINITY;  // this group's running maximum
+  float den = 0.f;      // this group's sum, scaled to 2^-M
   float4 acc[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int base = 0; base < P; base += 32) {
-    // weight of partition base + lane, computed by its owner and broadcast by shuffle, so
-    // the loop below issues only independent loads of the partial outputs
-    const int own = base + lane;
-    const float w_own = own < P ? rescale_factor(ml[2 * own], M) : 0.f;
-    if (own < P) den = fmaf(w_own, ml[2 * own + 1], den);
-    const int cnt = min(32, P - base);
-    // group g takes partitions base + g, base + g + 4, ...; the trip count is warp-uniform
 #pragma unroll 4
-    for (int j = 0; j < (cnt + MERGE_GROUPS - 1) / MERGE_GROUPS; ++j) {
-      const int k = j * MERGE_GROUPS + grp;
-      const float w = __shfl_sync(0xffffffffu, w_own, k & 31);
-      if (k < cnt) {
-        float4 x[CPL];
+  for (int k = grp; k < P; k += MERGE_GROUPS) {
+    const float mk = ml[2 * k], lk = ml[2 * k + 1];
+    float4 x[CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) x[c] = src[(size_t)(base + k) * V4 + c * GL + sub];
+    for (int c = 0; c < CPL; ++c) x[c] = src[(size_t)k * V4 + c * GL + sub];
+    const float Mn = fmaxf(M, mk);
+    const float a = rescale_factor(M, Mn), w = rescale_factor(mk, Mn);
+    den = fmaf(w, lk, den * a);
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          acc[c].x = fmaf(w, x[c].x, acc[c].x);
-          acc[c].y = fmaf(w, x[c].y, acc[c].y);
-          acc[c].z = fmaf(w, x[c].z, acc[c].z);
-          acc[c].w = fmaf(w, x[c].w, acc[c].w);
-        }
-      }
+    for (int c = 0; c < CPL; ++c) {
+      acc[c].x = fmaf(w, x[c].x, acc[c].x * a);
+      acc[c].y = fmaf(w, x[c].y, acc[c].y * a);
+      acc[c].z = fmaf(w, x[c].z, acc[c].z * a);
+      acc[c].w = fmaf(w, x[c].w, acc[c].w * a);
     }
+    M = Mn;
+  }
+  // the groups' maxima, sums and columns brought to the overall maximum and added up
+  // (lanes sub, sub + 8, sub + 16, sub + 24 hold the same columns)
+  float Mall = M;
+#pragma unroll
+  for (int o = GL; o < 32; o <<= 1) Mall = fmaxf(Mall, __shfl_xor_sync(0xffffffffu, Mall, o));
+  const float a = rescale_factor(M, Mall);
+  den *= a;
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    acc[c].x *= a;
+    acc[c].y *= a;
+    acc[c].z *= a;
+    acc[c].w *= a;
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  // add up the four groups (lanes sub, sub + 8, sub + 16, sub + 24 hold the same columns)
-#pragma unroll
   for (int o = GL; o < 32; o <<= 1) {
+    den += __shfl_xor_sync(0xffffffffu, den, o);
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
       acc[c].x += __shfl_xor_sync(0xffffffffu, acc[c].x, o);

@@ -42,6 +42,26 @@ CASES = [
 ]
 
 
+def _ragged(n, hi, seed):
+    """n context lengths in [1, hi], with block-edge lengths at the chunks' first and last
+    sequences (whatever the chunking) and at the batch's ends."""
+    lens = np.random.default_rng(seed).integers(1, hi + 1, n)
+    edges = [1, 15, 16, 17, 31, 32, 33, 2]
+    for i, j in enumerate([0, n - 1, n // 6, n // 6 - 1, n // 2, n // 2 - 1, 5 * n // 6,
+                           5 * n // 6 - 1]):
+        lens[j] = edges[i]
+    return [int(x) for x in lens]
+
+
+# at least 128 sequences: the host step splits the batch into chunks (3 or 4 here) pipelined
+# over two copy streams and two compute streams
+CASES += [
+    (_fixed("host_chunked_mha", 8, 8, 64, 16, _ragged(200, 400, 1)), 0),
+    (_fixed("host_chunked_mha_split", 8, 8, 128, 16, _ragged(256, 700, 2)), 64),
+    (_fixed("host_chunked_gqa", 16, 2, 128, 16, _ragged(256, 900, 3)), 0),
+]
+
+
 @pytest.mark.parametrize("pinned", [True, False], ids=["pinned", "pageable"])
 @pytest.mark.parametrize("w,part", CASES, ids=[c[0].name for c in CASES])
 def test_host_step_matches_the_oracle(pkv, w, part, pinned):
@@ -64,12 +84,21 @@ def test_host_step_matches_the_oracle(pkv, w, part, pinned):
     assert_attention_close(out.numpy().astype(np.float64), ob.attention())
 
 
+# the copy-on-write workload's shape at 8 prompts (64 samples, one chunk), and 16 prompts of
+# 100 tokens (128 samples: two chunks, the copies ahead of both)
+COW = {"cow_small": lambda: wl.get("cow_small"),
+       "cow_128_chunked": lambda: wl.Workload("cow_128_chunked", 128, 8, 8, 64, 16, 2048, 1004,
+                                              "cow", prompts=16, prompt_len=100, samples=8,
+                                              decode_steps=3)}
+
+
+@pytest.mark.parametrize("cow", list(COW))
 @pytest.mark.parametrize("shared", [False, True], ids=["plain", "shared_prefix"])
-def test_host_step_copy_on_write_steps(pkv, shared):
-    # the copy-on-write workload's shape at 8 prompts (64 samples): step 0 copies the 56
-    # shared partial tails, then two more steps; every step goes through the host call
+def test_host_step_copy_on_write_steps(pkv, shared, cow):
+    # step 0 copies the shared partial tails (7 per prompt), then two more steps; every
+    # step goes through the host call
     from batches import CowBatch
-    w = wl.get("cow_small")
+    w = COW[cow]()
     B, H, Hk, D, bs, N = w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, w.block_size, \
         w.num_blocks
     gb = CowBatch(w, DEV)

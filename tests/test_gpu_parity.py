@@ -104,6 +104,10 @@ SMALL = [
     (_fixed("gqa8_bs4_cuda_cores", 16, 2, 64, 4, [1, 4, 5, 90]), 0),
     (_fixed("gqa16_cuda_cores", 32, 2, 64, 16, [2, 17, 250]), 0),
     (_fixed("gqa16_cuda_cores_split", 32, 2, 64, 16, [2, 17, 250]), 32),
+    # CUDA-core CTAs of 2 and 4 query heads over one kv head (G = 2 at bs 4; G = 10, 12)
+    (_fixed("gqa2_bs4_cuda_cores", 4, 2, 128, 4, [1, 4, 5, 63]), 0),
+    (_fixed("gqa10_cuda_cores_split", 20, 2, 128, 16, [3, 16, 17, 300]), 64),
+    (_fixed("gqa12_cuda_cores", 24, 2, 64, 16, [2, 33, 190]), 0),
     # long single passes: every stage of the ring is refilled many times
     (_fixed("gqa8_d128_bs64_long", 16, 2, 128, 64, [700, 1500]), -1),
     (_fixed("gqa4_d128_bs32_long", 8, 2, 128, 32, [999, 1800]), -1),

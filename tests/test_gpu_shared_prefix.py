@@ -233,6 +233,15 @@ def test_many_short_suffixes(pkv, part):
     _run(pkv, fb, True, part)
 
 
+def test_more_groups_than_the_persistent_grid(pkv):
+    # 1100 prompts of 16-55 tokens, 2 samples each: 1100 groups, so the prefix pass runs
+    # one CTA per item (the persistent grid takes up to 1024 groups)
+    fb = ForkBatch(pkv, 4, 4, 64, 16, [16 + i % 40 for i in range(1100)], 2, lambda i: i % 3)
+    pre, groups = fb.groups()
+    assert len(groups) == 1100
+    _run(pkv, fb, True, 0)
+
+
 def test_inconsistent_groups_are_flagged_not_faulted(pkv):
     fb = ForkBatch(pkv, 8, 8, 128, 16, [300, 200], 4, lambda i: i)
     pre, groups = fb.groups()

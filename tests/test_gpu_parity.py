@@ -101,6 +101,8 @@ SMALL = [
     (_fixed("gqa2_d128_bs32", 4, 2, 128, 32, [1, 31, 32, 33, 410]), 0),
     (_fixed("gqa2_d128_bs64_split", 4, 2, 128, 64, [1, 63, 64, 65, 410]), 128),
     (_fixed("gqa3_d64_bs16", 6, 2, 64, 16, [7, 40, 129]), 0),
+    (_fixed("gqa4_d64_bs32", 8, 2, 64, 32, [1, 31, 32, 33, 500]), 0),
+    (_fixed("gqa8_d64_bs64_split", 16, 2, 64, 64, [1, 63, 64, 65, 700]), 128),
     (_fixed("gqa8_bs4_cuda_cores", 16, 2, 64, 4, [1, 4, 5, 90]), 0),
     (_fixed("gqa16_cuda_cores", 32, 2, 64, 16, [2, 17, 250]), 0),
     (_fixed("gqa16_cuda_cores_split", 32, 2, 64, 16, [2, 17, 250]), 32),

@@ -175,6 +175,9 @@ CASES = [
     ("gqa2_d128_bs32", 8, 4, 128, 32, [900, 100], 6, lambda i: (5 * i) % 40, 0),
     ("gqa4_d64_bs16_p128", 16, 4, 64, 16, [600], 4, lambda i: i, 128),
     ("gqa8_no_groups", 16, 2, 128, 16, [300], 3, lambda i: i, 0),
+    ("mha64_bs32", 4, 4, 64, 32, [500, 70], 4, lambda i: (9 * i) % 50, 0),
+    ("mha64_bs64_p128", 4, 4, 64, 64, [600, 130], 3, lambda i: 30 * i, 128),
+    ("gqa2_d128_bs8", 8, 4, 128, 8, [400, 45], 4, lambda i: (3 * i) % 20, 0),
     ("single_samples", 4, 4, 128, 16, [50, 60, 70], 1, lambda i: 0, 0),
 ]
 

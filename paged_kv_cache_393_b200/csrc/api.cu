@@ -656,6 +656,7 @@ struct StepLayout {
 #ifndef PAGEDKV_TUNE_STEP_END_QUARTERS
 #define PAGEDKV_TUNE_STEP_END_QUARTERS 2  // half-size end chunks (measured faster than equal)
 #endif
+constexpr size_t STEP_SMALL_COPY = 65536;  // host copies below this are staged by the CPU
 constexpr int STEP_MAX_CHUNKS = PAGEDKV_TUNE_STEP_CHUNKS;
 constexpr int STEP_CHUNK_SEQS = PAGEDKV_TUNE_STEP_CHUNK_SEQS;
 
@@ -890,15 +891,24 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
     StepAux* aux = nullptr;
     if ((st = step_aux(&aux)) != PAGEDKV_OK) return st;
     const size_t row_q = H * D * 2, row_kv = Hk * D * 2, row_t = (size_t)max_blocks_per_seq * 4;
-    // uploads of chunk c: its table rows, lengths, q and new K/V rows
+    // Table rows go up with each chunk when every chunk's rows are a large copy of their
+    // own; otherwise the whole table goes once, ahead of the first chunk.  (Copies below
+    // STEP_SMALL_COPY bytes are staged by the host CPU, several microseconds each.)
+    int min_count = num_seqs;
+    for (int c = 0; c < nch; ++c) {
+      int first = 0, count = 0;
+      chunk_range(num_seqs, nch, c, &first, &count);
+      min_count = count < min_count ? count : min_count;
+    }
+    const bool rows_per_chunk = (size_t)min_count * row_t >= STEP_SMALL_COPY;
+    // uploads of chunk c: its table rows (when they go per chunk), q and new K/V rows
     auto upload = [&](int c, cudaStream_t us) -> int {
       int first = 0, count = 0, r = PAGEDKV_OK;
       chunk_range(num_seqs, nch, c, &first, &count);
-      if ((r = h2d(base + lay.tables + first * row_t,
-                   reinterpret_cast<const char*>(block_tables_host) + first * row_t,
-                   count * row_t, us, "block table upload")) != PAGEDKV_OK ||
-          (r = h2d(base + lay.lens + first * 4, context_lens_host + first, count * 4, us,
-                   "context length upload")) != PAGEDKV_OK ||
+      if ((rows_per_chunk &&
+           (r = h2d(base + lay.tables + first * row_t,
+                    reinterpret_cast<const char*>(block_tables_host) + first * row_t,
+                    count * row_t, us, "block table upload")) != PAGEDKV_OK) ||
           (r = h2d(base + lay.q + first * row_q, static_cast<const char*>(q_host) + first * row_q,
                    count * row_q, us, "query upload")) != PAGEDKV_OK ||
           (r = h2d(base + lay.k + first * row_kv,
@@ -910,11 +920,16 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
         return r;
       return PAGEDKV_OK;
     };
-    // The pairs and the first chunk's inputs go up on the caller's stream, ahead of its
-    // kernels with no cross-stream wait (and after the previous step on it, which read
-    // this staging); the copy stream takes the other chunks once they have landed.
+    // The pairs, the lengths, the table (unless it goes per chunk) and the first chunk's
+    // inputs go up on the caller's stream, ahead of its kernels with no cross-stream wait
+    // (and after the previous step on it, which read this staging); the copy stream
+    // takes the other chunks once they have landed.
     if ((st = h2d(base + lay.pairs, copy_pairs_host, (size_t)num_pairs * 16, s,
                   "pair upload")) != PAGEDKV_OK ||
+        (st = h2d(base + lay.lens, context_lens_host, B * 4, s, "context length upload")) !=
+            PAGEDKV_OK ||
+        (!rows_per_chunk && (st = h2d(base + lay.tables, block_tables_host, B * row_t, s,
+                                      "block table upload")) != PAGEDKV_OK) ||
         (st = upload(0, s)) != PAGEDKV_OK)
       return st;
     PKV_CHECK_CUDA(cudaEventRecord(aux->start, s), "step start");

@@ -168,17 +168,22 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
         const int tok = c * CHUNK;
         const int phys = s_ids[tok / BS - w0];
         const int r0 = tok % BS;
-        mbar_arrive_expect_tx(full, 2 * TILE_BYTES);
-        if (BS == CHUNK) {  // the KVC heads of one block are one contiguous tile
+        // the partition's last stage copies only its rows in the context (the rest of
+        // the tile is never read), each kv head's rows one contiguous copy
+        const int rows = min(CHUNK, ntok - tok);
+        if (BS == CHUNK && rows == CHUNK) {  // the KVC heads of one block: one contiguous tile
           const size_t off = ((size_t)phys * p.num_kv_heads + kv0) * (size_t)(BS * D);
+          mbar_arrive_expect_tx(full, 2 * TILE_BYTES);
           bulk_load(kdst, p.k_cache + off, TILE_BYTES, full, policy);
           bulk_load(vdst, p.v_cache + off, TILE_BYTES, full, policy);
         } else {
+          const uint32_t bytes = (uint32_t)rows * D * 2;
+          mbar_arrive_expect_tx(full, 2u * KVC * bytes);
 #pragma unroll
           for (int h = 0; h < KVC; ++h) {
             const size_t off = (((size_t)phys * p.num_kv_heads + kv0 + h) * BS + r0) * (size_t)D;
-            bulk_load(kdst + h * CHUNK * D * 2, p.k_cache + off, CHUNK * D * 2, full, policy);
-            bulk_load(vdst + h * CHUNK * D * 2, p.v_cache + off, CHUNK * D * 2, full, policy);
+            bulk_load(kdst + h * CHUNK * D * 2, p.k_cache + off, bytes, full, policy);
+            bulk_load(vdst + h * CHUNK * D * 2, p.v_cache + off, bytes, full, policy);
           }
         }
       } else {

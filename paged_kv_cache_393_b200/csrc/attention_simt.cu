@@ -189,12 +189,29 @@ __global__ void __launch_bounds__((HPC + 1) * 32)
       } else {
         const int first = c * NB;                // first block of the stage
         const int nb = min(NB, nblk - first);
-        mbar_arrive_expect_tx(full, 2u * nb * SUB_BYTES);
+        // only the partition's last block can be partly in the context: its kv heads'
+        // rows in the context are one copy each, the rest of the sub-tile is never read
+        const int last_rows = ntok - (nblk - 1) * BS;
+        const bool part_last = first + nb == nblk && last_rows < BS;
+        const uint32_t last_bytes = (uint32_t)last_rows * D * 2;
+        mbar_arrive_expect_tx(full, part_last ? 2u * ((nb - 1) * SUB_BYTES + KVC * last_bytes)
+                                              : 2u * nb * SUB_BYTES);
         for (int k = 0; k < nb; ++k) {
           const size_t off =
               ((size_t)s_ids[first + k - w0] * p.num_kv_heads + kv0) * (size_t)(BS * D);
-          bulk_load(kdst + k * SUB_BYTES, p.k_cache + off, SUB_BYTES, full, policy);
-          bulk_load(vdst + k * SUB_BYTES, p.v_cache + off, SUB_BYTES, full, policy);
+          if (part_last && k == nb - 1) {
+#pragma unroll
+            for (int h = 0; h < KVC; ++h) {
+              const uint32_t hs = (uint32_t)h * CB * D * 2;
+              bulk_load(kdst + k * SUB_BYTES + hs, p.k_cache + off + (size_t)h * BS * D,
+                        last_bytes, full, policy);
+              bulk_load(vdst + k * SUB_BYTES + hs, p.v_cache + off + (size_t)h * BS * D,
+                        last_bytes, full, policy);
+            }
+          } else {
+            bulk_load(kdst + k * SUB_BYTES, p.k_cache + off, SUB_BYTES, full, policy);
+            bulk_load(vdst + k * SUB_BYTES, p.v_cache + off, SUB_BYTES, full, policy);
+          }
         }
       }
       issued = c + 1;

@@ -639,6 +639,7 @@ size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 struct StepLayout {
   size_t q, k, v, tables, lens, pairs, out, prefix, groups, ws, ws2;
   size_t ws_bytes, total;
+  int chunk_part;  // partition_size of every chunk's call: the whole batch's partitioning
 };
 
 // The plain host step splits a batch into chunks of sequences so that uploading
@@ -707,8 +708,10 @@ int step_layout(StepLayout* lay, int num_seqs, int num_heads, int num_kv_heads, 
   lay->out = take(B * H * D * 2);
   lay->prefix = shared_prefix ? take(B * 4) : 0;
   lay->groups = shared_prefix ? take((B / 2 > 0 ? B / 2 : 1) * GROUP_WIDTH * 4) : 0;
-  // the chunks run one after another and share the workspace: size it for the
-  // largest plan among the whole batch and its chunks
+  // Every chunk is split as the whole batch would be (its partition size, or a single
+  // pass), so that each (sequence, head) is computed exactly as by one call over the
+  // batch.  The chunks share two workspaces: size them for the largest chunk plan.
+  lay->chunk_part = partition_size != 0 ? partition_size : (plan.split ? plan.part_tokens : -1);
   size_t ws = plan.ws_bytes;
   const int n = step_chunks(num_seqs, shared_prefix);
   for (int i = 0; i < n && n > 1; ++i) {
@@ -716,7 +719,7 @@ int step_layout(StepLayout* lay, int num_seqs, int num_heads, int num_kv_heads, 
     chunk_range(num_seqs, n, i, &first, &count);
     Plan cp;
     if (make_plan(&cp, count, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
-                  partition_size, false) == PAGEDKV_OK && cp.ws_bytes > ws)
+                  lay->chunk_part, false) == PAGEDKV_OK && cp.ws_bytes > ws)
       ws = cp.ws_bytes;
   }
   lay->ws = take(ws);
@@ -961,7 +964,7 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
           reinterpret_cast<const int32_t*>(base + lay.tables + first * row_t),
           reinterpret_cast<const int32_t*>(base + lay.lens) + first, scale, block_size,
           num_kv_heads, count, num_heads, head_dim, max_blocks_per_seq, num_blocks,
-          max_context_len, partition_size, ws, lay.ws_bytes, cs);
+          max_context_len, lay.chunk_part, ws, lay.ws_bytes, cs);
       if (st != PAGEDKV_OK) return st;
       PKV_CHECK_CUDA(cudaEventRecord(aux->out[c], cs), "compute event");
       PKV_CHECK_CUDA(cudaStreamWaitEvent(aux->down, aux->out[c], 0), "download wait");

@@ -84,6 +84,37 @@ def test_host_step_matches_the_oracle(pkv, w, part, pinned):
     assert_attention_close(out.numpy().astype(np.float64), ob.attention())
 
 
+CHUNKED = [c for c in CASES if c[0].num_seqs >= 128]
+
+
+@pytest.mark.parametrize("w,part", CHUNKED, ids=[c[0].name for c in CHUNKED])
+def test_chunked_step_equals_one_call(pkv, w, part):
+    # every chunk is split as the whole batch is, so the pipelined step computes each
+    # (sequence, head) exactly as one fused call over the batch does: the outputs agree
+    # bit for bit
+    from batches import PagedBatch
+    gb = PagedBatch(w, DEV)
+    B, H, D = w.num_seqs, w.num_heads, w.head_dim
+    sess = pkv.DecodeSession(gb.key_cache, gb.value_cache, B, H, gb.max_blocks,
+                             gb.max_context_len, w.scale, part)
+    out = _host(np.full((B, H, D), np.nan, np.float16), True)
+    stream = torch.cuda.Stream()
+    sess.step(_host(gb.q_host, True), _host(gb.k_new_host, True), _host(gb.v_new_host, True),
+              _host(gb.tables_host, True), _host(gb.lens_host, True), out, stream=stream)
+    stream.synchronize()
+    # one call over the whole batch (it stores the same new rows again)
+    need = pkv.paged_attention_workspace_bytes(B, H, w.num_kv_heads, D, w.block_size,
+                                               gb.max_context_len, part)
+    ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=DEV)
+    one = torch.full((B, H, D), float("nan"), dtype=torch.float16, device=DEV)
+    pkv.paged_attention_decode_append(one, gb.q, gb.k_new, gb.v_new, gb.key_cache,
+                                      gb.value_cache, gb.block_tables, gb.context_lens, w.scale,
+                                      gb.max_context_len, part, ws)
+    torch.cuda.synchronize()
+    assert pkv.device_errors() == 0
+    assert np.array_equal(out.numpy().view(np.uint16), _bits(one))
+
+
 # the copy-on-write workload's shape at 8 prompts (64 samples, one chunk), and 16 prompts of
 # 100 tokens (128 samples: two chunks, the copies ahead of both)
 COW = {"cow_small": lambda: wl.get("cow_small"),

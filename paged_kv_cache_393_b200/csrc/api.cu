@@ -214,10 +214,11 @@ int make_plan(Plan* plan, int num_seqs, int num_heads, int num_kv_heads, int hea
     const int auto_part = AUTO_PARTITION % align == 0 ? AUTO_PARTITION : align;
     if (!p.mma) {
       // CUDA-core kernel: split every context longer than a partition -- smaller, more uniform
-      // CTAs balance the end of the launch (measured faster at 256 and at 32 sequences) -- and
-      // halve the partition (down to 128 tokens) until there are ~4 waves of CTAs.
+      // CTAs balance the end of the launch (measured faster at 256 and at 32 sequences) --
+      // starting from 1024 tokens and halving (down to 128) until there are ~4 waves of CTAs.
+      // (256 sequences of 500..1524 tokens: 1024 beat 512, 1280, 2048 and a single pass.)
       const long long groups = (long long)num_seqs * (num_heads / p.hpc);
-      int pt = auto_part;
+      int pt = 2 * auto_part;
       while (pt > 128 && pt / 2 % align == 0 &&
              groups * ((max_context_len + pt - 1) / pt) < 4LL * NUM_SMS_HINT * SIMT_CTAS_PER_SM)
         pt /= 2;

@@ -158,10 +158,10 @@ def test_workspace_bytes(lib):
     # single pass over one kv head per query head: no workspace
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, -1) == 0
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 512, 0) == 0
-    # CUDA-core kernel, automatic: 512-token partitions for the 256-sequence batch, halved to
+    # CUDA-core kernel, automatic: 1024-token partitions for the 256-sequence batch, halved to
     # 128 for 32 sequences (2 kv heads per CTA: 512 CTAs per partition, ~4 waves wanted)
     assert pkv.paged_attention_workspace_bytes(256, 32, 32, 128, 16, 1524, 0) == \
-        32 + 256 * 32 * 3 * 130 * 4
+        32 + 256 * 32 * 2 * 130 * 4
     assert pkv.paged_attention_workspace_bytes(32, 32, 32, 128, 16, 1524, 0) == \
         32 + 32 * 32 * 12 * 130 * 4
     # explicit split: B * H * P * (D + 2) floats (CUDA-core kernel, MHA)
@@ -180,16 +180,16 @@ def test_workspace_bytes(lib):
 
 
 def test_noalloc_falls_back_to_a_single_pass_for_the_automatic_plan(lib):
-    # 256 MHA sequences up to 2500 tokens: the automatic 512-token split needs ~21 MB, more
+    # 256 MHA sequences up to 4000 tokens: the automatic 1024-token split needs ~17 MB, more
     # than the 16 MiB built-in scratch, so the call runs a single pass instead of refusing.
     # Without a GPU here it then fails on the device lookup, never with EWORKSPACE.
-    B, H, D, bs, maxlen = 256, 32, 128, 16, 2500
+    B, H, D, bs, maxlen = 256, 32, 128, 16, 4000
     assert lib.paged_attention_workspace_bytes(B, H, H, D, bs, maxlen, 0) > (16 << 20)
     fn = lib.paged_attention_decode_noalloc
     P, I = ctypes.c_void_p, ctypes.c_int
     fn.argtypes = [P, P, P, P, P, P, ctypes.c_float] + [I] * 9 + [P]
     fn.restype = I
-    args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, bs, H, B, H, D, 160, 65536, maxlen)
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, bs, H, B, H, D, 256, 65536, maxlen)
     st = fn(*args, 0, None)
     assert st != nat.EWORKSPACE
     assert fn(*args, 512, None) == nat.EWORKSPACE     # an explicit split is kept, and refused
@@ -198,7 +198,7 @@ def test_noalloc_falls_back_to_a_single_pass_for_the_automatic_plan(lib):
 def test_partition_tokens(lib):
     f = pkv.paged_attention_partition_tokens
     assert f(256, 32, 32, 128, 16, 1524, -1) == 0          # single pass asked for
-    assert f(256, 32, 32, 128, 16, 1524, 0) == 512         # automatic split
+    assert f(256, 32, 32, 128, 16, 1524, 0) == 1024        # automatic split
     assert f(32, 32, 32, 128, 16, 1524, 0) == 128          # small batch: smaller partitions
     assert f(128, 64, 8, 128, 16, 16384, 0) == 512         # long grouped-query contexts
     assert f(256, 32, 32, 128, 16, 1524, 256) == 256

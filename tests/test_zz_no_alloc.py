@@ -46,9 +46,9 @@ CASES = [
     (_workload("auto", 8, 8, 128, 16, [17, 2500]), 0),                 # library's choice (splits)
     (_workload("single", 4, 4, 128, 16, [40, 90]), -1),                # no scratch needed
     (_workload("gqa_single", 16, 2, 128, 16, [40, 900]), -1),          # only the work counter
-    # the library's split would need ~19 MB of scratch (128 x 32 heads x 9 partitions):
-    # more than the built-in 16 MiB, so the call falls back to a single pass
-    (_workload("auto_fallback", 32, 32, 128, 16, [4100] + [5 + i % 40 for i in range(127)]), 0),
+    # the library's split would need ~19 MB of scratch (128 x 32 heads x 9 partitions of 1024
+    # tokens): more than the built-in 16 MiB, so the call falls back to a single pass
+    (_workload("auto_fallback", 32, 32, 128, 16, [8200] + [5 + i % 40 for i in range(127)]), 0),
 ]
 
 

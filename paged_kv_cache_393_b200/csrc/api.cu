@@ -894,6 +894,21 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
     // comes after all of it.
     StepAux* aux = nullptr;
     if ((st = step_aux(&aux)) != PAGEDKV_OK) return st;
+    // On an error return after work was enqueued, the caller's stream still waits for
+    // whatever the side streams hold (best effort), so that its next use of this
+    // staging comes after it.
+    struct SideJoin {
+      cudaStream_t s;
+      StepAux* aux;
+      bool armed;
+      ~SideJoin() {
+        if (!armed) return;
+        for (cudaStream_t side : {aux->up, aux->comp, aux->down}) {
+          if (cudaEventRecord(aux->done, side) == cudaSuccess)
+            cudaStreamWaitEvent(s, aux->done, 0);
+        }
+      }
+    } side_join{s, aux, true};
     const size_t row_q = H * D * 2, row_kv = Hk * D * 2, row_t = (size_t)max_blocks_per_seq * 4;
     // Table rows go up with each chunk when every chunk's rows are a large copy of their
     // own; otherwise the whole table goes once, ahead of the first chunk.  (Copies below
@@ -977,6 +992,7 @@ int paged_decode_step_host(void* out_host, const void* q_host, const void* k_new
     // the caller's stream joins the downloads (which follow every chunk's kernels)
     PKV_CHECK_CUDA(cudaEventRecord(aux->done, aux->down), "download event");
     PKV_CHECK_CUDA(cudaStreamWaitEvent(s, aux->done, 0), "step join");
+    side_join.armed = false;
     return PAGEDKV_OK;
   }
   // 1. the step's inputs, host to device (small arrays first)

@@ -301,6 +301,17 @@ PAGEDKV_API int pagedkv_prefix_groups(const int32_t *block_tables, const int32_t
  *      taken from the host arrays);
  *   4. a device -> host copy of the output into out_host.
  *
+ * A plain step (no shared prefixes) of at least 128 sequences runs those steps
+ * for up to 4 chunks of sequences, pipelined: the first chunk's inputs go up on
+ * `stream`, the other chunks' on an internal copy stream; the chunks' attention
+ * alternates between `stream` and an internal compute stream, each chunk
+ * starting when its inputs have landed; each chunk's output comes back on an
+ * internal copy stream.  The internal streams are created per host thread and
+ * device at the first such call and kept until the process exits.  `stream`
+ * waits for all of it, also after an error return.  Every chunk is split as
+ * the whole batch would be, so the output equals that of one
+ * paged_attention_decode_append call over the batch, bit for bit.
+ *
  * The call returns once everything is enqueued; out_host is valid after the
  * stream synchronizes.  With pinned (page-locked) host buffers every copy is
  * asynchronous; pageable buffers work too, with copies the driver stages.

@@ -40,7 +40,7 @@ def test_context_length_recipes():
 
 
 def test_pool_fits_every_workload():
-    for name in ("tiny", "llama7b", "gqa"):
+    for name in ("tiny", "llama7b", "gqa", "llama7b_small", "gqa_small"):
         w = wl.get(name)
         need = sum(-(-int(L) // w.block_size) for L in wl.context_lens(w))
         assert need <= w.num_blocks, name
@@ -48,10 +48,14 @@ def test_pool_fits_every_workload():
         w = wl.bs_sweep(bs)
         need = sum(-(-int(L) // bs) for L in wl.context_lens(w))
         assert need <= w.num_blocks
-    w = wl.get("cow")
-    prefix = w.prompts * -(-w.prompt_len // w.block_size)
-    grown = w.num_seqs * (-(-(w.prompt_len + w.decode_steps) // w.block_size) - w.prompt_len // w.block_size)
-    assert prefix + grown <= w.num_blocks
+    for name in ("cow", "cow_small", "cow_compact"):
+        # prompts written once; every sample then owns its copied tail block and the
+        # blocks its 200 steps grow into
+        w = wl.get(name)
+        prefix = w.prompts * -(-w.prompt_len // w.block_size)
+        grown = w.num_seqs * (-(-(w.prompt_len + w.decode_steps) // w.block_size)
+                              - w.prompt_len // w.block_size)
+        assert prefix + grown <= w.num_blocks, name
 
 
 def test_generators_are_deterministic_and_length_independent():

@@ -93,7 +93,7 @@ WORKLOADS = {
     # an 8-prompt cut of cow (64 samples) for profiler captures of the shared-prefix pass
     "cow_small": Workload("cow_small", 64, 32, 32, 128, 16, 8192, 1004, "cow",
                           prompts=8, prompt_len=1000, samples=8, decode_steps=200),
-    # the whole cow batch in a pool of 6144 blocks (1.6 GB; 200 steps need 5312): the
+    # the whole cow batch in a pool of 6144 blocks (1.6 GB; 200 steps need 5344): the
     # prefix pass's full item count, for multi-pass profiler captures
     "cow_compact": Workload("cow_compact", 256, 32, 32, 128, 16, 6144, 1004, "cow",
                             prompts=32, prompt_len=1000, samples=8, decode_steps=200),
